@@ -1,0 +1,168 @@
+/*
+ * pp.h - C ABI of libpp, exact softmax attention over a preference-packed sequence on B200 (sm_100a).
+ *
+ * Problem (pages: "Preference Packing: Efficient Preference Optimization for LLMs", abstract and method digest;
+ * "prefix_grouper_utils.py", section 1 building position ids, section 2 building the grouper, and the
+ * prefix-sharing diagram; "PackInfer: Compute- and I/O-Efficient Attention for Batched LLM Inference", abstract):
+ * a batch of G groups is packed into one flat sequence of T tokens. Group g stores its prompt prefix P_g once,
+ * followed by its k_g responses S_g1..S_gk. A prefix token attends causally within the prefix; a token of S_i
+ * attends to the whole prefix and causally within S_i, never to a sibling response or to another group. Position
+ * ids run 0..P_g-1 on the prefix and restart at P_g for every response.
+ *
+ * Conventions for every call
+ *   - Ownership: the caller owns all memory. The library allocates nothing on the device or the host (apart from a
+ *     few small static tables of its own); every buffer is passed in as a raw pointer with its size.
+ *   - Pointers: "_d" names and every tensor argument are DEVICE pointers on the current CUDA device, except where a
+ *     comment says host. Tensors are dense and row-major:
+ *       Q, O, dO, dQ: [T, Hq, d]; K, V, dK, dV: [T, Hkv, d]; LSE: [Hq, T] fp32; pos ids: int32 [T].
+ *     The packed order is group by group: prefix, then the responses in order.
+ *   - Asynchrony: every call only enqueues work on `stream` (a cudaStream_t; NULL = legacy default stream) and
+ *     returns without synchronising, except pp_get_status().
+ *   - Errors: arguments are validated on the host before anything is enqueued; an invalid argument returns
+ *     PP_ERR_INVALID_ARG (or PP_ERR_UNSUPPORTED / PP_ERR_WORKSPACE) and enqueues nothing. A failed launch returns
+ *     PP_ERR_CUDA. Problems only the device can see (inconsistent descriptors, a bounded wait that ran out) set a
+ *     device error word that pp_get_status() reads. pp_last_error() returns a message for the calling thread.
+ *   - Limits: T < 2^31 - 256; d in {64, 128}; Hq % Hkv == 0; Hq <= 256.
+ */
+#ifndef PP_H_
+#define PP_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PP_API __attribute__((visibility("default")))
+#else
+#define PP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PP_OK = 0,
+    PP_ERR_INVALID_ARG = -1,   /* host-side validation failed; nothing was enqueued */
+    PP_ERR_UNSUPPORTED = -2,   /* valid but unsupported combination (e.g. backward in fp32) */
+    PP_ERR_CUDA = -3,          /* a CUDA runtime/driver call failed */
+    PP_ERR_DEVICE_TIMEOUT = -4,/* a kernel's bounded wait ran out (reported by pp_get_status) */
+    PP_ERR_WORKSPACE = -5,     /* a buffer is smaller than the size the library asked for */
+    PP_ERR_DEVICE_INPUT = -6   /* the device found inconsistent descriptors (reported by pp_get_status) */
+} pp_status;
+
+typedef enum { PP_BF16 = 0, PP_FP32 = 1 } pp_dtype;
+
+/* One group's descriptor ("prefix_grouper_utils.py" section 1: each group carries its prefix length and its
+ * responses' lengths). The response lengths themselves are the segments of cu_seqlens. */
+typedef struct {
+    int32_t prefix_len;    /* P_g >= 0 */
+    int32_t num_suffixes;  /* k_g >= 0 */
+} pp_group_desc;
+
+/* Which pass a workspace size is asked for. */
+enum { PP_PASS_FWD = 0, PP_PASS_BWD = 1 };
+
+/* ---------------------------------------------------------------------------------------------------------------
+ * pp_meta_bounds (host only, no device work)
+ * Upper bound on the bytes of the metadata buffer that pp_build_meta fills, from the sizes alone.
+ *   num_groups G >= 1, num_segments = sum_g (1 + k_g), total_tokens T >= 0, num_heads_q / num_heads_kv as for the
+ *   attention calls. *meta_bytes (host pointer) receives the size. Errors: PP_ERR_INVALID_ARG.
+ */
+PP_API pp_status pp_meta_bounds(int32_t num_groups, int32_t num_segments, int64_t total_tokens, int32_t num_heads_q,
+                         int32_t num_heads_kv, int64_t *meta_bytes);
+
+/* ---------------------------------------------------------------------------------------------------------------
+ * pp_build_meta: group descriptors + segment boundaries -> grouped position ids and the tile schedule.
+ * ("prefix_grouper_utils.py" section 1 for the position ids; "PackInfer" abstract for building the attention work
+ * directly over the packed query-key regions and balancing it across thread blocks.)
+ *   groups_d      device pp_group_desc[num_groups]
+ *   cu_seqlens_d  device int32[num_segments + 1]: packed segment boundaries in the packed order (for each group its
+ *                 prefix, then each response); zero-length segments allowed. cu[0] must be 0, cu[nseg] must be T,
+ *                 and num_segments must equal sum_g (1 + k_g); a violation found on the device sets
+ *                 PP_ERR_DEVICE_INPUT (pp_get_status) and leaves the outputs undefined.
+ *   pos_ids_d     device int32[T] out: position ids (prefix 0..P-1, every response restarts at P).
+ *   meta_d        device buffer out, meta_bytes >= the pp_meta_bounds value, 256-byte aligned. Its content is
+ *                 private to the library (read it only through the calls below); it holds the per-token segment
+ *                 table, the forward query tiles (128 rows, aligned to each group's start) in cost order, and the
+ *                 backward key/value tiles (128 rows) split into work chunks in cost order.
+ * The buffers must stay alive and unchanged while attention calls that use them are in flight.
+ */
+PP_API pp_status pp_build_meta(const pp_group_desc *groups_d, int32_t num_groups, const int32_t *cu_seqlens_d,
+                        int32_t num_segments, int64_t total_tokens, int32_t num_heads_q, int32_t num_heads_kv,
+                        int32_t *pos_ids_d, void *meta_d, int64_t meta_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------------------------------------------
+ * pp_meta_tiles: expand the schedule in meta_d into explicit tiles, for checking and inspection.
+ *   which = PP_PASS_FWD: query tiles of 128 rows x key tiles of 128 rows; PP_PASS_BWD: key tiles of 128 rows x
+ *   query tiles of 64 rows. Both are aligned to each group's start. Writes one int32 triple
+ *   (q_row0, kv_row0, class) per non-empty tile into tiles_d (device int32[3 * capacity]), class 1 = every pair in
+ *   the tile allowed (FULL), 2 = some allowed (PARTIAL); fully masked tiles are never listed. *count_d (device
+ *   int32) receives the number of tiles (possibly > capacity; only the first `capacity` are written). The order is
+ *   unspecified. The classification is the same device code the attention kernels use.
+ */
+PP_API pp_status pp_meta_tiles(const void *meta_d, int32_t which, int32_t *tiles_d, int64_t capacity, int32_t *count_d,
+                        void *stream);
+
+/* ---------------------------------------------------------------------------------------------------------------
+ * pp_rope: rotary embedding at the grouped position ids, in place on q and k (v untouched).
+ * Rotate-half form with base theta: for m < d/2, w_m = theta^(-2m/d), a = pos * w_m,
+ *   y_m = x_m cos a - x_{m+d/2} sin a,  y_{m+d/2} = x_{m+d/2} cos a + x_m sin a
+ * (the pages give the positions, "prefix_grouper_utils.py" section 1, but not the variant; rotate-half is the
+ * reading taken). inverse != 0 rotates by -a, which maps gradients of the rotated tensors back.
+ *   q: [T, hq, d], k: [T, hkv, d] (either may be NULL to skip it), dt = PP_BF16 or PP_FP32 storage; the angle is
+ *   formed in fp64 and the rotation in fp32, rounded to nearest even on store. theta > 0 (0 means 10000).
+ */
+PP_API pp_status pp_rope(void *q, void *k, const int32_t *pos_ids_d, int64_t T, int32_t hq, int32_t hkv, int32_t d,
+                  float theta, pp_dtype dt, int32_t inverse, void *stream);
+
+/* ---------------------------------------------------------------------------------------------------------------
+ * pp_workspace_bytes (host only): scratch bytes pp_attn_fwd (which = PP_PASS_FWD) or pp_attn_bwd
+ * (PP_PASS_BWD) needs for these sizes. *bytes (host pointer) receives it.
+ */
+PP_API pp_status pp_workspace_bytes(int32_t which, int64_t T, int32_t hq, int32_t hkv, int32_t d, int64_t *bytes);
+
+/* ---------------------------------------------------------------------------------------------------------------
+ * pp_attn_fwd: O and the per-row log-sum-exp of exact packed attention.
+ *   s_ij = softmax_scale * q_i . k_j over the allowed keys j of row i (q head h reads kv head h / (hq/hkv));
+ *   lse_i = ln sum_j exp(s_ij) (natural log of the scaled scores); o_i = sum_j exp(s_ij - lse_i) v_j.
+ *   q, k, v: inputs as above in dtype dt (PP_BF16: tcgen05 tensor-core path, fp32 accumulation;
+ *   PP_FP32: fp32 CUDA-core path, meant for small checks). o: [T, hq, d] out in dt; lse: [hq, T] fp32 out.
+ *   softmax_scale 0 means 1/sqrt(d). meta_d from pp_build_meta with the same T, hq, hkv.
+ *   workspace: device scratch of ws_bytes >= pp_workspace_bytes(PP_PASS_FWD, ...), 256-byte aligned; contents
+ *   need not be initialised. Rows of fully masked positions do not exist (every row attends at least itself).
+ */
+PP_API pp_status pp_attn_fwd(const void *q, const void *k, const void *v, const void *meta_d, int64_t T, int32_t hq,
+                      int32_t hkv, int32_t d, float softmax_scale, pp_dtype dt, void *o, float *lse,
+                      void *workspace, int64_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------------------------------------------
+ * pp_attn_bwd: gradients of sum(O * dO) with respect to q, k and v (bf16 only).
+ *   D_i = dO_i . o_i; p_ij = exp(s_ij - lse_i); dS_ij = p_ij (dO_i . v_j - D_i);
+ *   dq_i = scale sum_j dS_ij k_j; dk_j = scale sum_h sum_i dS_ij q_i; dv_j = sum_h sum_i p_ij dO_i
+ *   (sums over the q heads h that share kv head j's head). q, k, v, o, lse: the forward's inputs and outputs;
+ *   dout: [T, hq, d]. dq, dk, dv: outputs in bf16 with the shapes of q, k, v (fully overwritten).
+ *   workspace: ws_bytes >= pp_workspace_bytes(PP_PASS_BWD, ...), 256-byte aligned, contents need not be
+ *   initialised. Prefix key tiles, attended by every response of their group, are split into chunks whose fp32
+ *   partial dK/dV are added tile by tile into the workspace (bounded: one bulk add per chunk and tile).
+ */
+PP_API pp_status pp_attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                      const void *dout, const void *meta_d, int64_t T, int32_t hq, int32_t hkv, int32_t d,
+                      float softmax_scale, void *dq, void *dk, void *dv, void *workspace, int64_t ws_bytes,
+                      void *stream);
+
+/* ---------------------------------------------------------------------------------------------------------------
+ * pp_get_status: synchronises `stream`, then reads and clears this device's error word. Returns PP_OK,
+ * PP_ERR_DEVICE_TIMEOUT, PP_ERR_DEVICE_INPUT or PP_ERR_CUDA (a sticky CUDA error is reported as such).
+ */
+PP_API pp_status pp_get_status(void *stream);
+
+/* Message describing the last failure seen by the calling thread ("" if none). Valid until its next call. */
+PP_API const char *pp_last_error(void);
+
+/* Library version string. */
+PP_API const char *pp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PP_H_ */

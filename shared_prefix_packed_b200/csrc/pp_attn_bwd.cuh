@@ -1,0 +1,542 @@
+// pp_attn_bwd.cuh - backward of exact attention over a preference-packed sequence (bf16, d = 128, sm_100a).
+//
+// What it computes (pp.h, pp_attn_bwd): with p_ij = exp(s_ij - lse_i) and D_i = dO_i . o_i,
+//   dS_ij = p_ij (dO_i . v_j - D_i),  dQ_i = scale sum_j dS_ij k_j,
+//   dK_j = scale sum_h sum_i dS_ij q_i,  dV_j = sum_h sum_i p_ij dO_i   (h over the q heads of j's kv head).
+//
+// Three kernels:
+//   k_bwd_pre     D = rowsum(dO * O) in fp32 (HBM-bound).
+//   k_bwd_tc      key/value-stationary tensor-core kernel. A work item is (key tile of 128 rows, kv head, chunk of
+//                 the query tiles that attend it). Seen from key y the attending queries are one interval
+//                 [y, e(y)) (pp_meta.cuh), so a key tile's query tiles are one contiguous range; prefix key tiles
+//                 (attended by every response of the group) get long ranges and are split into chunks so the
+//                 persistent grid stays balanced. Per step (query tile of 64 rows, one q head of the kv head):
+//                   S^T  = K Q^T         (M=128 keys, N=64 queries)     TMEM S[b]
+//                   dP^T = V dO^T                                       TMEM dP[b]
+//                   softmax warps: P^T = exp(S^T - lse), dS^T = P^T (dP^T - D)   -> TMEM (bf16) and smem (bf16)
+//                   dV  += P^T dO        (A from TMEM)                  TMEM dV
+//                   dK  += dS^T Q        (A from TMEM)                  TMEM dK
+//                   dQ^T = K^T dS^T      (M=128 = d, N=64 queries)      TMEM S[b] (reused once P^T is consumed)
+//                 dQ^T is read by a second warpgroup, scaled, staged in smem and added to an fp32 accumulator
+//                 with one bulk reduce-add per step. dK/dV stay in TMEM for the whole item; an unsplit key tile
+//                 writes them as bf16, a split one adds its fp32 partial into the workspace (one add per chunk).
+//   k_bwd_convert dQ (and the split tiles' dK/dV) from the fp32 accumulators to bf16.
+// TMEM (512 columns): S[0] [0,64), S[1] [64,128), dP[0] [128,192), dP[1] [192,256), dV [256,384), dK [384,512).
+// S/dP are double-buffered so the MMAs of step t+1 run while the softmax warps work on step t.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include "pp_meta.cuh"
+#include "pp_ptx.cuh"
+#include "pp_attn_fwd.cuh"   // bwait, globaltimer_ns
+
+namespace pp {
+
+constexpr int BWD_THREADS = 320;
+constexpr int BWD_D = 128;
+
+struct BwdWorkspace {
+    int64_t rows_pad;   // T + padding rows so tiles that stick out past T stay inside the buffers
+    int64_t off_delta;  // fp32 [hq][rows_pad]: D_i = dO_i . O_i
+    int64_t off_dq;     // fp32 [hq][rows_pad][d]: dQ accumulator
+    int64_t off_dk;     // fp32 [rows_pad][hkv][d]: dK accumulator of split key tiles
+    int64_t off_dv;     // fp32 [rows_pad][hkv][d]: dV accumulator of split key tiles
+    int64_t total;
+};
+
+inline BwdWorkspace bwd_workspace_layout(int64_t T, int hq, int hkv, int d) {
+    BwdWorkspace w{};
+    w.rows_pad = T + 256;
+    int64_t o = 0;
+    w.off_delta = o; o = align256(o + 4 * int64_t(hq) * w.rows_pad);
+    w.off_dq = o;    o = align256(o + 4 * int64_t(hq) * w.rows_pad * d);
+    w.off_dk = o;    o = align256(o + 4 * w.rows_pad * hkv * d);
+    w.off_dv = o;    o = align256(o + 4 * w.rows_pad * hkv * d);
+    w.total = o;
+    return w;
+}
+
+// ------------------------------------------------------------------------------------------------- preprocess
+// One warp per (row, head): D = sum_d dO * O in fp32; padding rows get 0.
+__global__ void k_bwd_pre(const __nv_bfloat16 *__restrict__ O, const __nv_bfloat16 *__restrict__ dO,
+                          float *__restrict__ delta, int64_t T, int64_t rows_pad, int hq) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = int64_t(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t w = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < rows_pad * hq; w += nwarps) {
+        const int64_t i = w / hq;
+        const int h = static_cast<int>(w % hq);
+        float acc = 0.f;
+        if (i < T) {
+            const uint2 a = reinterpret_cast<const uint2 *>(O + (i * hq + h) * BWD_D)[lane];
+            const uint2 b = reinterpret_cast<const uint2 *>(dO + (i * hq + h) * BWD_D)[lane];
+            const uint32_t av[2] = {a.x, a.y}, bv[2] = {b.x, b.y};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(bv[e] << 16), acc);
+                acc = fmaf(__uint_as_float(av[e] & 0xffff0000u), __uint_as_float(bv[e] & 0xffff0000u), acc);
+            }
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) delta[int64_t(h) * rows_pad + i] = acc;
+    }
+}
+
+// ------------------------------------------------------------------------------------------------- main kernel
+struct BwdSmem {
+    static constexpr int KV_BYTES = 128 * BWD_D * 2;     // 128 key rows x d, bf16
+    static constexpr int KV_CHUNK = 128 * 64 * 2;        // one 64-column swizzled chunk of it
+    static constexpr int QT_BYTES = 64 * BWD_D * 2;      // 64 query rows x d
+    static constexpr int QT_CHUNK = 64 * 64 * 2;
+    static constexpr int DS_BYTES = 128 * 64 * 2;        // dS^T: 128 key rows x 64 queries, bf16
+    alignas(1024) uint8_t k[KV_BYTES];
+    alignas(1024) uint8_t v[KV_BYTES];
+    alignas(1024) uint8_t q[2][QT_BYTES];
+    alignas(1024) uint8_t dout[2][QT_BYTES];
+    alignas(1024) uint8_t ds[2][DS_BYTES];
+    alignas(1024) float stage[64 * BWD_D];               // dQ tile [64 queries][d] for the bulk add
+    float lse2[2][64];                                   // lse * log2(e) of the step's query rows
+    float dl[2][64];                                     // D of the step's query rows
+    uint64_t kv_full, kv_empty, dkv_full, dkv_free;
+    uint64_t q_full[2], q_empty[2], sdp_full[2], ds_full[2], ds_free[2], dq_full[2], dq_free[2];
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+struct BwdItem {
+    KTile t;
+    int qa, qb, split, kh;
+};
+
+__device__ __forceinline__ BwdItem bwd_decode(const void *meta, const MetaHeader &hd, int item, int hkv) {
+    const BWork w = meta_ptr<BWork>(meta, hd.off_bw)[item / hkv];
+    BwdItem it;
+    it.kh = item % hkv;
+    it.t = meta_ptr<KTile>(meta, hd.off_kt)[w.kt];
+    it.qa = w.qa;
+    it.qb = w.qb;
+    it.split = w.split;
+    return it;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+         const void *__restrict__ meta, const float *__restrict__ LSE, const float *__restrict__ delta,
+         float *__restrict__ dq_acc, float *__restrict__ dk_acc, float *__restrict__ dv_acc,
+         __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV, int hq, int hkv, int64_t rows_pad,
+         float scale, float sl2) {
+    extern __shared__ uint8_t smem_raw[];
+    BwdSmem &sm = *reinterpret_cast<BwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const MetaHeader hd = *meta_ptr<MetaHeader>(meta, 0);
+    const int T = hd.T;
+    const int r = hq / hkv;
+    const int n_items = hd.n_bw * hkv;
+    volatile int *abort_flag = &sm.abort_flag;
+    constexpr float LOG2E = 1.4426950408889634f;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.kv_full, 1);
+        mbar_init(&sm.kv_empty, 1);
+        mbar_init(&sm.dkv_full, 1);
+        mbar_init(&sm.dkv_free, 128);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.q_full[b], 32);
+            mbar_init(&sm.q_empty[b], 1);
+            mbar_init(&sm.sdp_full[b], 1);
+            mbar_init(&sm.ds_full[b], 128);
+            mbar_init(&sm.ds_free[b], 1);
+            mbar_init(&sm.dq_full[b], 1);
+            mbar_init(&sm.dq_free[b], 128);
+        }
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmdO);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 384;
+
+    if (hd.dev_err != 0) {
+        // nothing to do: the metadata builder rejected its input
+    } else if (warp == 8) {
+        // ------------------------------------------------------------------ producer warp
+        uint32_t g = 0, it_n = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+            const BwdItem w = bwd_decode(meta, hd, item, hkv);
+            if (lane == 0) {
+                if (!bwait(&sm.kv_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
+                mbar_arrive_expect_tx(&sm.kv_full, 2 * BwdSmem::KV_BYTES);
+                for (int c = 0; c < BWD_D / 64; ++c) {
+                    tma_load_3d(sm.k + c * BwdSmem::KV_CHUNK, &tmK, c * 64, w.kh, w.t.row0, &sm.kv_full);
+                    tma_load_3d(sm.v + c * BwdSmem::KV_CHUNK, &tmV, c * 64, w.kh, w.t.row0, &sm.kv_full);
+                }
+            }
+            const int n = (w.qb - w.qa) * r;
+            for (int t = 0; t < n; ++t, ++g) {
+                const int b = g & 1;
+                const int h = w.kh * r + t % r;
+                const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
+                if (!bwait(&sm.q_empty[b], ((g >> 1) & 1) ^ 1, abort_flag)) goto done;
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int i = lane + 32 * e;
+                    const int row = x0 + i;
+                    sm.lse2[b][i] = row < T ? LSE[int64_t(h) * T + row] * LOG2E : 0.f;
+                    sm.dl[b][i] = delta[int64_t(h) * rows_pad + row];
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sm.q_full[b], 2 * BwdSmem::QT_BYTES);
+                    for (int c = 0; c < BWD_D / 64; ++c) {
+                        tma_load_3d(sm.q[b] + c * BwdSmem::QT_CHUNK, &tmQ, c * 64, h, x0, &sm.q_full[b]);
+                        tma_load_3d(sm.dout[b] + c * BwdSmem::QT_CHUNK, &tmdO, c * 64, h, x0, &sm.q_full[b]);
+                    }
+                } else {
+                    mbar_arrive(&sm.q_full[b]);
+                }
+            }
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------------------------ MMA issuer (one thread)
+        if (lane == 0) {
+            constexpr uint32_t ID_SDP = idesc_bf16(128, BWD_BM, 0, 0);     // S^T, dP^T
+            constexpr uint32_t ID_KV = idesc_bf16(128, BWD_D, 0, 1);       // dV, dK (B MN-major)
+            constexpr uint32_t ID_DQ = idesc_bf16(128, BWD_BM, 1, 1);      // dQ^T (A and B MN-major)
+            const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
+            uint32_t g = 0, it_n = 0;
+            auto issue_sdp = [&](int b) {
+                const uint32_t sq = smem_u32(sm.q[b]), sdo = smem_u32(sm.dout[b]);
+#pragma unroll
+                for (int kk = 0; kk < BWD_D / 16; ++kk) {
+                    const uint32_t ok = (kk >> 2) * BwdSmem::KV_CHUNK + (kk & 3) * 32;
+                    const uint32_t oq = (kk >> 2) * BwdSmem::QT_CHUNK + (kk & 3) * 32;
+                    umma_ss(tmem + COL_S + b * 64, smem_desc(sk + ok, 16, 1024), smem_desc(sq + oq, 16, 1024),
+                            ID_SDP, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < BWD_D / 16; ++kk) {
+                    const uint32_t ok = (kk >> 2) * BwdSmem::KV_CHUNK + (kk & 3) * 32;
+                    const uint32_t oq = (kk >> 2) * BwdSmem::QT_CHUNK + (kk & 3) * 32;
+                    umma_ss(tmem + COL_DP + b * 64, smem_desc(sv + ok, 16, 1024), smem_desc(sdo + oq, 16, 1024),
+                            ID_SDP, kk > 0);
+                }
+            };
+            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+                const BwdItem w = bwd_decode(meta, hd, item, hkv);
+                const int n = (w.qb - w.qa) * r;
+                if (!bwait(&sm.kv_full, it_n & 1, abort_flag)) goto done;
+                // S^T / dP^T of the item's first step
+                {
+                    const int b = g & 1;
+                    if (!bwait(&sm.q_full[b], (g >> 1) & 1, abort_flag)) goto done;
+                    if (!bwait(&sm.dq_free[b], ((g >> 1) & 1) ^ 1, abort_flag)) goto done;
+                    tc_fence_after();
+                    issue_sdp(b);
+                    umma_commit(&sm.sdp_full[b]);
+                }
+                if (!bwait(&sm.dkv_free, (it_n & 1) ^ 1, abort_flag)) goto done;
+                for (int t = 0; t < n; ++t, ++g) {
+                    const int b = g & 1, b1 = (g + 1) & 1;
+                    if (t + 1 < n) {
+                        const uint32_t g1 = g + 1;
+                        if (!bwait(&sm.q_full[b1], (g1 >> 1) & 1, abort_flag)) goto done;
+                        if (!bwait(&sm.dq_free[b1], ((g1 >> 1) & 1) ^ 1, abort_flag)) goto done;
+                        tc_fence_after();
+                        issue_sdp(b1);
+                        umma_commit(&sm.sdp_full[b1]);
+                    }
+                    if (!bwait(&sm.ds_full[b], (g >> 1) & 1, abort_flag)) goto done;
+                    tc_fence_after();
+                    const uint32_t sq = smem_u32(sm.q[b]), sdo = smem_u32(sm.dout[b]), sds = smem_u32(sm.ds[b]);
+#pragma unroll
+                    for (int kk = 0; kk < BWD_BM / 16; ++kk)       // dV += P^T dO
+                        umma_ts(tmem + COL_DV, tmem + COL_S + b * 64 + kk * 8,
+                                smem_desc(sdo + kk * 2048, BwdSmem::QT_CHUNK, 1024), ID_KV, (t > 0 || kk > 0));
+#pragma unroll
+                    for (int kk = 0; kk < BWD_BM / 16; ++kk)       // dK += dS^T Q
+                        umma_ts(tmem + COL_DK, tmem + COL_DP + b * 64 + kk * 8,
+                                smem_desc(sq + kk * 2048, BwdSmem::QT_CHUNK, 1024), ID_KV, (t > 0 || kk > 0));
+#pragma unroll
+                    for (int kk = 0; kk < 128 / 16; ++kk)          // dQ^T = K^T dS^T
+                        umma_ss(tmem + COL_S + b * 64, smem_desc(sk + kk * 2048, BwdSmem::KV_CHUNK, 1024),
+                                smem_desc(sds + kk * 2048, BwdSmem::DS_BYTES, 1024), ID_DQ, kk > 0);
+                    umma_commit(&sm.dq_full[b]);
+                    umma_commit(&sm.q_empty[b]);
+                    umma_commit(&sm.ds_free[b]);
+                }
+                umma_commit(&sm.dkv_full);
+                umma_commit(&sm.kv_empty);
+            }
+        }
+    } else if (warp < 4) {
+        // ------------------------------------------------------------------ softmax / gradient warpgroup
+        const int jr = warp * 32 + lane;                               // key row within the tile = TMEM lane
+        const uint32_t lane_off = uint32_t(warp * 32) << 16;
+        uint32_t g = 0, it_n = 0;
+        const int32_t *key_end = meta_ptr<int32_t>(meta, hd.off_key_end);
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+            const BwdItem w = bwd_decode(meta, hd, item, hkv);
+            const int n = (w.qb - w.qa) * r;
+            const int y = w.t.row0 + jr;
+            const int gend = w.t.gstart + w.t.glen;
+            const bool yin = y < gend;
+            const int ke = yin ? key_end[y] : y;                       // queries [y, ke) attend key y
+            for (int t = 0; t < n; ++t, ++g) {
+                const int b = g & 1;
+                const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
+                if (!bwait(&sm.ds_free[b], ((g >> 1) & 1) ^ 1, abort_flag)) goto done;
+                if (!bwait(&sm.sdp_full[b], (g >> 1) & 1, abort_flag)) goto done;
+                if (!bwait(&sm.q_full[b], (g >> 1) & 1, abort_flag)) goto done;
+                tc_fence_after();
+                uint32_t sr[64], pr[64];
+                {
+                    uint32_t tmp[32];
+                    tmem_ld32(tmem + lane_off + COL_S + b * 64, tmp);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) sr[e] = tmp[e];
+                    tmem_ld32(tmem + lane_off + COL_S + b * 64 + 32, tmp);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) sr[32 + e] = tmp[e];
+                    tmem_ld32(tmem + lane_off + COL_DP + b * 64, tmp);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) pr[e] = tmp[e];
+                    tmem_ld32(tmem + lane_off + COL_DP + b * 64 + 32, tmp);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) pr[32 + e] = tmp[e];
+                    tmem_wait_ld();
+                }
+                const int lo = y - x0, hi = ke - x0;                   // allowed query columns [lo, hi)
+                uint32_t pp[32], dd[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    float p2[2], d2[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int c = 2 * e + u;
+                        const bool ok = c >= lo && c < hi;
+                        const float p = ok ? ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -sm.lse2[b][c])) : 0.f;
+                        p2[u] = p;
+                        d2[u] = p * (__uint_as_float(pr[c]) - sm.dl[b][c]);
+                    }
+                    pp[e] = pack_bf16x2(p2[0], p2[1]);
+                    dd[e] = pack_bf16x2(d2[0], d2[1]);
+                }
+                {
+                    uint32_t tmp[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) tmp[e] = pp[e];
+                    tmem_st16(tmem + lane_off + COL_S + b * 64, tmp);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) tmp[e] = pp[16 + e];
+                    tmem_st16(tmem + lane_off + COL_S + b * 64 + 16, tmp);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) tmp[e] = dd[e];
+                    tmem_st16(tmem + lane_off + COL_DP + b * 64, tmp);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) tmp[e] = dd[16 + e];
+                    tmem_st16(tmem + lane_off + COL_DP + b * 64 + 16, tmp);
+                }
+                // dS^T row jr into the 128-byte-swizzled [key][query] tile read by the dQ MMA
+                uint8_t *dsrow = sm.ds[b] + jr * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(dsrow + ((c ^ (jr & 7)) << 4)) =
+                        make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&sm.ds_full[b]);
+            }
+            // item epilogue: dK (scaled) and dV from TMEM
+            if (!bwait(&sm.dkv_full, it_n & 1, abort_flag)) goto done;
+            tc_fence_after();
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t col = which == 0 ? COL_DK : COL_DV;
+                const float f = which == 0 ? scale : 1.f;
+                float *acc = which == 0 ? dk_acc : dv_acc;
+                __nv_bfloat16 *dst = which == 0 ? dK : dV;
+#pragma unroll
+                for (int c = 0; c < BWD_D / 32; ++c) {
+                    uint32_t rr[32];
+                    tmem_ld32(tmem + lane_off + col + c * 32, rr);
+                    tmem_wait_ld();
+                    if (!yin) continue;
+                    if (w.split) {
+                        float *a = acc + (int64_t(y) * hkv + w.kh) * BWD_D + c * 32;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            red_add_v4(a + 4 * e, __uint_as_float(rr[4 * e]) * f, __uint_as_float(rr[4 * e + 1]) * f,
+                                       __uint_as_float(rr[4 * e + 2]) * f, __uint_as_float(rr[4 * e + 3]) * f);
+                    } else {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            pk[e] = pack_bf16x2(__uint_as_float(rr[2 * e]) * f, __uint_as_float(rr[2 * e + 1]) * f);
+                        uint4 *o = reinterpret_cast<uint4 *>(dst + (int64_t(y) * hkv + w.kh) * BWD_D + c * 32);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) o[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.dkv_free);
+        }
+    } else {
+        // ------------------------------------------------------------------ dQ warpgroup (warps 4-7)
+        const int dcol = (warp - 4) * 32 + lane;                       // head-dim index = TMEM lane
+        const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
+        const bool leader = (warp == 4 && lane == 0);
+        uint32_t g = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+            const BwdItem w = bwd_decode(meta, hd, item, hkv);
+            const int n = (w.qb - w.qa) * r;
+            for (int t = 0; t < n; ++t, ++g) {
+                const int b = g & 1;
+                const int h = w.kh * r + t % r;
+                const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
+                if (!bwait(&sm.dq_full[b], (g >> 1) & 1, abort_flag)) goto done;
+                tc_fence_after();
+                uint32_t v[64];
+                {
+                    uint32_t tmp[32];
+                    tmem_ld32(tmem + lane_off + COL_S + b * 64, tmp);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = tmp[e];
+                    tmem_ld32(tmem + lane_off + COL_S + b * 64 + 32, tmp);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[32 + e] = tmp[e];
+                    tmem_wait_ld();
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.dq_free[b]);
+                if (leader) bulk_wait_read0();                         // the previous add has read the stage
+                named_bar_sync(1, 128);
+#pragma unroll
+                for (int c = 0; c < 64; ++c) sm.stage[c * BWD_D + dcol] = __uint_as_float(v[c]) * scale;
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (leader) {
+                    bulk_reduce_add_f32(dq_acc + (int64_t(h) * rows_pad + x0) * BWD_D, sm.stage,
+                                        64 * BWD_D * sizeof(float));
+                    bulk_commit();
+                }
+            }
+        }
+        if (leader) bulk_wait0();
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------------------------------------- convert
+// dQ[i][h][:] = bf16(dq_acc[h][i][:]); dK/dV rows of split key tiles = bf16(accumulators).
+__global__ void k_bwd_convert(const void *__restrict__ meta, const float *__restrict__ dq_acc,
+                              const float *__restrict__ dk_acc, const float *__restrict__ dv_acc,
+                              __nv_bfloat16 *__restrict__ dQ, __nv_bfloat16 *__restrict__ dK,
+                              __nv_bfloat16 *__restrict__ dV, int hq, int hkv, int64_t rows_pad) {
+    const MetaHeader hd = *meta_ptr<MetaHeader>(meta, 0);
+    if (hd.dev_err) return;
+    const int64_t T = hd.T;
+    const int64_t nvec_q = T * hq * (BWD_D / 4);
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < nvec_q; e += stride) {
+        const int64_t row = e / (int64_t(hq) * (BWD_D / 4));
+        const int64_t rem = e % (int64_t(hq) * (BWD_D / 4));
+        const int h = static_cast<int>(rem / (BWD_D / 4)), c = static_cast<int>(rem % (BWD_D / 4));
+        const float4 a = reinterpret_cast<const float4 *>(dq_acc + (int64_t(h) * rows_pad + row) * BWD_D)[c];
+        __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+        uint2 u;
+        u.x = *reinterpret_cast<uint32_t *>(&lo);
+        u.y = *reinterpret_cast<uint32_t *>(&hi);
+        reinterpret_cast<uint2 *>(dQ + (row * hq + h) * BWD_D)[c] = u;
+    }
+    const KTile *kts = meta_ptr<KTile>(meta, hd.off_kt);
+    const int64_t per_tile = int64_t(128) * hkv * (BWD_D / 4);
+    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < int64_t(hd.n_kt) * per_tile; e += stride) {
+        const KTile t = kts[e / per_tile];
+        if (t.nch <= 1) continue;
+        const int64_t rem = e % per_tile;
+        const int64_t row = t.row0 + rem / (hkv * (BWD_D / 4));
+        if (row >= t.gstart + t.glen) continue;
+        const int64_t off = row * hkv * BWD_D + (rem % (hkv * (BWD_D / 4))) * 4;
+        for (int which = 0; which < 2; ++which) {
+            const float4 a = *reinterpret_cast<const float4 *>((which ? dv_acc : dk_acc) + off);
+            __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+            uint2 u;
+            u.x = *reinterpret_cast<uint32_t *>(&lo);
+            u.y = *reinterpret_cast<uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>((which ? dV : dK) + off) = u;
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------------- launcher
+typedef pp_status (*MakeMapFn)(CUtensorMap *, const void *, int64_t, int, int, int);
+typedef pp_status (*FailFn)(pp_status, const char *, ...);
+
+inline pp_status launch_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                            const void *dout, const void *meta, int64_t T, int hq, int hkv, int d, float scale,
+                            void *dq, void *dk, void *dv, void *workspace, int sm_count, cudaStream_t s,
+                            MakeMapFn make_map, FailFn fail) {
+    if (d != BWD_D) return fail(PP_ERR_UNSUPPORTED, "backward supports head dim 128 only (got %d)", d);
+    const BwdWorkspace L = bwd_workspace_layout(T, hq, hkv, d);
+    char *ws = static_cast<char *>(workspace);
+    float *delta = reinterpret_cast<float *>(ws + L.off_delta);
+    float *dq_acc = reinterpret_cast<float *>(ws + L.off_dq);
+    float *dk_acc = reinterpret_cast<float *>(ws + L.off_dk);
+    float *dv_acc = reinterpret_cast<float *>(ws + L.off_dv);
+    const void *ptrs[8] = {q, k, v, o, dout, dq, dk, dv};
+    for (const void *p : ptrs)
+        if (reinterpret_cast<uintptr_t>(p) % 16) return fail(PP_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+    CUtensorMap mq, mk, mv, mdo;
+    pp_status st;
+    if ((st = make_map(&mq, q, T, hq, d, BWD_BM)) != PP_OK) return st;
+    if ((st = make_map(&mk, k, T, hkv, d, BWD_BN)) != PP_OK) return st;
+    if ((st = make_map(&mv, v, T, hkv, d, BWD_BN)) != PP_OK) return st;
+    if ((st = make_map(&mdo, dout, T, hq, d, BWD_BM)) != PP_OK) return st;
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(ws + L.off_dq, 0, L.total - L.off_dq, s)) != cudaSuccess)
+        return fail(PP_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    k_bwd_pre<<<sm_count * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(o),
+                                           static_cast<const __nv_bfloat16 *>(dout), delta, T, L.rows_pad, hq);
+    if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_pre: %s", cudaGetErrorString(e));
+    const size_t smem = sizeof(BwdSmem) + 1024;
+    if ((e = cudaFuncSetAttribute(k_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem))) != cudaSuccess)
+        return fail(PP_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    k_bwd_tc<<<sm_count, BWD_THREADS, smem, s>>>(mq, mk, mv, mdo, meta, lse, delta, dq_acc, dk_acc, dv_acc,
+                                                 static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv),
+                                                 hq, hkv, L.rows_pad, scale, scale * 1.4426950408889634f);
+    if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_tc: %s", cudaGetErrorString(e));
+    k_bwd_convert<<<sm_count * 8, 256, 0, s>>>(meta, dq_acc, dk_acc, dv_acc, static_cast<__nv_bfloat16 *>(dq),
+                                               static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv),
+                                               hq, hkv, L.rows_pad);
+    if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_convert: %s", cudaGetErrorString(e));
+    return PP_OK;
+}
+
+}  // namespace pp

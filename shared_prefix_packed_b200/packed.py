@@ -1,0 +1,78 @@
+"""PackedBatch: one packed batch's device buffers and the four library calls in order.
+
+Allocation (torch) and argument marshalling only; every step runs in libpp's kernels.
+"""
+from __future__ import annotations
+
+from typing import Sequence
+
+import torch
+
+from . import _lib
+
+
+class PackedBatch:
+    """Group descriptors on the device, the schedule built by ``pp_build_meta``, and reusable workspaces.
+
+    prefix_lens[g] = P_g, suffix_lens[g] = [S_g1, ..., S_gk]; the packed order is each group's prefix, then its
+    responses ("prefix_grouper_utils.py" section 2).
+    """
+
+    def __init__(self, prefix_lens: Sequence[int], suffix_lens: Sequence[Sequence[int]], hq: int, hkv: int, d: int,
+                 device="cuda", stream=None):
+        self.hq, self.hkv, self.d = hq, hkv, d
+        self.device = torch.device(device)
+        groups, lens = [], []
+        for p, ss in zip(prefix_lens, suffix_lens):
+            groups.append((int(p), len(ss)))
+            lens.append(int(p))
+            lens.extend(int(s) for s in ss)
+        self.T = int(sum(lens))
+        cu = [0]
+        for n in lens:
+            cu.append(cu[-1] + n)
+        self.groups = torch.tensor(groups, dtype=torch.int32).to(self.device)
+        self.cu_seqlens = torch.tensor(cu, dtype=torch.int32).to(self.device)
+        nbytes = _lib.pp_meta_bounds(len(groups), len(lens), self.T, hq, hkv)
+        self.meta = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.pos_ids = torch.empty(max(self.T, 1), dtype=torch.int32, device=self.device)
+        self.ws_fwd = torch.empty(_lib.pp_workspace_bytes(_lib.PP_PASS_FWD, self.T, hq, hkv, d), dtype=torch.uint8,
+                                  device=self.device)
+        self._ws_bwd = None
+        self.build(stream)
+
+    def build(self, stream=None):
+        _lib.pp_build_meta(self.groups, self.cu_seqlens, self.T, self.hq, self.hkv, self.pos_ids, self.meta, stream)
+
+    @property
+    def ws_bwd(self):
+        if self._ws_bwd is None:
+            n = _lib.pp_workspace_bytes(_lib.PP_PASS_BWD, self.T, self.hq, self.hkv, self.d)
+            self._ws_bwd = torch.empty(n, dtype=torch.uint8, device=self.device)
+        return self._ws_bwd
+
+    def rope(self, q, k, theta: float = 10000.0, inverse: bool = False, stream=None):
+        _lib.pp_rope(q, k, self.pos_ids, self.hq, self.hkv, self.d, theta, inverse, stream)
+
+    def forward(self, q, k, v, out=None, lse=None, softmax_scale: float = 0.0, stream=None):
+        o = torch.empty_like(q) if out is None else out
+        l = torch.empty(self.hq, self.T, dtype=torch.float32, device=q.device) if lse is None else lse
+        _lib.pp_attn_fwd(q, k, v, self.meta, o, l, self.ws_fwd, softmax_scale, stream)
+        return o, l
+
+    def backward(self, q, k, v, o, lse, dout, dq=None, dk=None, dv=None, softmax_scale: float = 0.0, stream=None):
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
+        _lib.pp_attn_bwd(q, k, v, o, lse, dout, self.meta, dq, dk, dv, self.ws_bwd, softmax_scale, stream)
+        return dq, dk, dv
+
+    def tiles(self, which: int, stream=None):
+        """Expanded schedule as a sorted list of (q_row0, kv_row0, class) (test and inspection helper)."""
+        count = torch.zeros(1, dtype=torch.int32, device=self.device)
+        _lib.pp_meta_tiles(self.meta, which, torch.empty(3, dtype=torch.int32, device=self.device), count, stream)
+        n = int(count.item())
+        buf = torch.empty(3 * max(n, 1), dtype=torch.int32, device=self.device)
+        _lib.pp_meta_tiles(self.meta, which, buf, count, stream)
+        rows = buf[: 3 * n].view(-1, 3).cpu().tolist()
+        return sorted(tuple(r) for r in rows)

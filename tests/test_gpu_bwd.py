@@ -1,0 +1,103 @@
+"""GPU parity of pp_attn_bwd against the fp64 oracle: dQ, dK, dV each within relative Frobenius error 1e-2.
+
+The GPU backward consumes the GPU forward's O (bf16) and LSE, as a training step would; the oracle recomputes
+everything in fp64 from the same bf16 inputs. At full workload sizes the oracle runs on whole groups (groups are
+independent, so a group's gradients are exact on their own) for a subset of kv heads.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests.gpu_util import random_case, to_np64
+
+pytestmark = pytest.mark.gpu
+
+REL_TOL = 1e-2
+
+
+def rel_fro(got, ref):
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(got - ref) / den) if den > 0 else float(np.linalg.norm(got))
+
+
+def _fwd_bwd(P, S, hq, hkv, d, seed, name="dpo"):
+    from shared_prefix_packed_b200 import PackedBatch, pp_get_status
+    inp = W.make_inputs(name, P, S, seed=seed, with_dout=True, heads=(hq, hkv, d))
+    b = PackedBatch(P, S, hq, hkv, d)
+    q, k, v, do = (inp[x].cuda() for x in ("q", "k", "v", "dout"))
+    o, lse = b.forward(q, k, v)
+    dq, dk, dv = b.backward(q, k, v, o, lse, do)
+    pp_get_status()
+    return inp, dq, dk, dv
+
+
+SMALL = [
+    ([3], [[2, 0, 3]]),
+    ([0], [[130, 77]]),
+    ([300], [[]]),
+    ([200], [[0, 0, 129]]),
+    ([1], [[1] * 40]),
+    ([128], [[128, 128]]),
+    ([127, 129, 1], [[1, 255], [3], [0]]),
+    ([513], [[200, 300, 64]]),
+    ([2100], [[700, 900]]),       # long prefix: its key tiles are split over several chunks
+]
+
+
+@pytest.mark.parametrize("case", range(len(SMALL)))
+@pytest.mark.parametrize("heads", [(4, 2), (7, 1)])
+def test_bwd_small(case, heads):
+    P, S = SMALL[case]
+    hq, hkv = heads
+    inp, dq, dk, dv = _fwd_bwd(P, S, hq, hkv, 128, 300 + case)
+    ref = oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["dout"], P, S)
+    for got, want in zip((dq, dk, dv), ref):
+        assert rel_fro(to_np64(got), want) <= REL_TOL
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_bwd_random(seed):
+    P, S = random_case(400 + seed, 1 + seed % 4, 1500, 800, 6)
+    inp, dq, dk, dv = _fwd_bwd(P, S, 8, 2, 128, seed)
+    ref = oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["dout"], P, S)
+    for got, want in zip((dq, dk, dv), ref):
+        assert rel_fro(to_np64(got), want) <= REL_TOL
+
+
+@pytest.mark.parametrize("name", ["dpo", "grpo", "longprefix"])
+def test_bwd_full_workload_sampled_groups(name):
+    """Full-size workload in the launch configuration the bench times; the oracle checks whole groups."""
+    from shared_prefix_packed_b200 import PackedBatch, pp_get_status
+    w = W.WORKLOADS[name]
+    P, S = W.group_lengths(name)
+    inp = W.make_inputs(name, P, S)
+    b = PackedBatch(P, S, w.num_heads_q, w.num_heads_kv, w.head_dim)
+    q, k, v, do = (inp[x].cuda() for x in ("q", "k", "v", "dout"))
+    o, lse = b.forward(q, k, v)
+    dq, dk, dv = b.backward(q, k, v, o, lse, do)
+    pp_get_status()
+    assert all(torch.isfinite(t.float()).all() for t in (dq, dk, dv))
+    lay = oracle.layout_of(P, S)
+    groups = [0, len(P) - 1]
+    kv_heads = [0, w.num_heads_kv - 1]
+    r = w.num_heads_q // w.num_heads_kv
+    qh = [h for kh in kv_heads for h in range(kh * r, (kh + 1) * r)]
+    dQ, dK, dV = oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["dout"], P, S, groups=groups,
+                                           kv_heads=kv_heads)
+    rows = np.concatenate([np.arange(lay.group_start[g], lay.group_start[g] + lay.group_len[g]) for g in groups])
+    assert rel_fro(to_np64(dq[rows][:, qh]), dQ[rows][:, qh]) <= REL_TOL
+    assert rel_fro(to_np64(dk[rows][:, kv_heads]), dK[rows][:, kv_heads]) <= REL_TOL
+    assert rel_fro(to_np64(dv[rows][:, kv_heads]), dV[rows][:, kv_heads]) <= REL_TOL
+
+
+def test_bwd_rejects_unsupported():
+    from shared_prefix_packed_b200 import PackedBatch, PPError
+    P, S = [10], [[5]]
+    b = PackedBatch(P, S, 4, 2, 64)
+    x = torch.zeros(15, 4, 64, dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros(15, 2, 64, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(4, 15, device="cuda")
+    with pytest.raises(PPError, match="UNSUPPORTED"):
+        b.backward(x, kv, kv, x, lse, x)

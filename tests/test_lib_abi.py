@@ -1,0 +1,52 @@
+"""CPU-only checks of the C-ABI boundary: libpp.so builds for sm_100a, loads, and exports every symbol that
+include/pp.h declares, with the signatures the binding uses. No compute call is made (there may be no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "pp.h")) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"PP_API\s+[\w\s\*]+?\b(pp_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("pp_build_meta", "pp_rope", "pp_attn_fwd", "pp_attn_bwd", "pp_meta_bounds", "pp_get_status",
+              "pp_last_error", "pp_workspace_bytes", "pp_meta_tiles"):
+        assert n in names
+
+
+def test_library_builds_loads_and_exports_every_declared_symbol():
+    from shared_prefix_packed_b200 import build as B
+    try:
+        B.build()
+    except RuntimeError as e:  # pragma: no cover - no toolchain
+        pytest.skip(f"nvcc unavailable: {e}")
+    L = ctypes.CDLL(B.LIB)
+    for name in _declared():
+        assert hasattr(L, name), name
+    from shared_prefix_packed_b200 import _lib
+    assert set(_declared()) == set(_lib.SIGNATURES), "binding and header disagree"
+    assert _lib.pp_version().startswith("libpp")
+
+
+def test_host_only_calls_and_validation():
+    """pp_meta_bounds / pp_workspace_bytes run on the host only; invalid sizes are rejected with a message."""
+    from shared_prefix_packed_b200 import _lib
+    n = _lib.pp_meta_bounds(8, 24, 17801, 32, 8)
+    assert n > 8 * 17801
+    assert _lib.pp_workspace_bytes(_lib.PP_PASS_BWD, 1000, 32, 8, 128) > 4 * 32 * 1000 * 128
+    with pytest.raises(_lib.PPError, match="INVALID_ARG"):
+        _lib.pp_meta_bounds(0, 1, 10, 32, 8)
+    with pytest.raises(_lib.PPError, match="INVALID_ARG"):
+        _lib.pp_workspace_bytes(_lib.PP_PASS_FWD, 100, 32, 6, 128)      # hq % hkv != 0
+    with pytest.raises(_lib.PPError, match="INVALID_ARG"):
+        _lib.pp_workspace_bytes(_lib.PP_PASS_FWD, 100, 32, 8, 96)       # unsupported head dim
+    with pytest.raises(_lib.PPError, match="INVALID_ARG"):
+        _lib.pp_workspace_bytes(_lib.PP_PASS_FWD, -1, 32, 8, 128)
