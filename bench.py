@@ -1,0 +1,392 @@
+"""Benchmark: packed-prefix attention fwd+bwd useful TFLOP/s on B200 (and its fraction of the bf16 tensor peak).
+
+One step = the whole hot path over one packed batch: pp_build_meta (position ids + tile schedule), pp_rope (Q, K),
+pp_attn_fwd (O, LSE) and pp_attn_bwd (dQ, dK, dV). Useful FLOPs count allowed (query, key) pairs only: 4*d per pair
+forward and 10*d per pair backward, per q head. Inputs are synthetic (workloads/), resident in HBM and larger than
+L2, so no flush is needed between steps. `e2e` times the same steps through the public API with pinned host buffers:
+the host->device copy of q, k, v, dout and the device->host copy of dq, dk, dv are inside its timed region.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dpo|grpo|longprefix|hetero|tiny]
+       python bench.py --impl reference ...   (the fp64 CPU oracle on a bounded sample of the same workload)
+Multi-GPU: launched by torch.distributed.run, one rank per GPU; each rank runs its own batch (weak scaling, no
+data-path collective); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = "dpo"
+L2_BYTES = 126 * 2 ** 20
+KERNEL_SOURCES = ("shared_prefix_packed_b200/csrc",)
+
+
+def pair_count(P, S):
+    tot = 0
+    for p, ss in zip(P, S):
+        tot += p * (p + 1) // 2 + sum(s * p + s * (s + 1) // 2 for s in ss)
+    return tot
+
+
+def unpacked_pairs(P, S):
+    return sum((p + s) * (p + s + 1) // 2 for p, ss in zip(P, S) for s in ss) + sum(
+        p * (p + 1) // 2 for p, ss in zip(P, S) if not ss)
+
+
+def flops_of(name, P, S):
+    w = W.WORKLOADS[name]
+    pairs = pair_count(P, S)
+    return pairs, 4 * w.head_dim * pairs * w.num_heads_q, (10 * w.head_dim * pairs * w.num_heads_q
+                                                          if w.backward else 0)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for d in KERNEL_SOURCES:
+        base = os.path.join(ROOT, d)
+        for fn in sorted(os.listdir(base)):
+            with open(os.path.join(base, fn), "rb") as f:
+                h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = kernel_source_hash()
+    with open(path) as f:
+        for ln in f:
+            parts = dict(p.split("=", 1) for p in ln.strip().split() if "=" in p)
+            if parts.get("kernel") == kernel and parts.get("sources") == src:
+                try:
+                    return float(parts["dram_bytes_per_launch"])
+                except (KeyError, ValueError):
+                    return None
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"pp_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for ln in f:
+                c = [x.strip() for x in ln.split(",")]
+                if len(c) < 9:
+                    continue
+                try:
+                    sm.append(float(c[1]))
+                    mx.append(float(c[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, c[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    from shared_prefix_packed_b200 import PackedBatch, _lib
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    name = args.workload
+    w = W.WORKLOADS[name]
+    P, S = W.group_lengths(name)
+    inp = W.make_inputs(name, P, S, seed=w.tensor_seed + 7919 * rank)   # each rank its own batch
+    hq, hkv, d = w.num_heads_q, w.num_heads_kv, w.head_dim
+    T = W.packed_total(P, S)
+    pairs, f_fwd, f_bwd = flops_of(name, P, S)
+    stream = torch.cuda.current_stream(dev)
+
+    q, k, v = (inp[x].to(dev) for x in "qkv")
+    dout = inp["dout"].to(dev) if w.backward else None
+    batch = PackedBatch(P, S, hq, hkv, d, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(hq, T, dtype=torch.float32, device=dev)
+    if w.backward:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    n_marks = 5
+
+    def step(marks=None):
+        if marks is not None:
+            marks[0].record(stream)
+        batch.build(stream)
+        if marks is not None:
+            marks[1].record(stream)
+        if w.rope:
+            batch.rope(q, k, stream=stream)
+        if marks is not None:
+            marks[2].record(stream)
+        batch.forward(q, k, v, out=o, lse=lse, stream=stream)
+        if marks is not None:
+            marks[3].record(stream)
+        if w.backward:
+            batch.backward(q, k, v, o, lse, dout, dq=dq, dk=dk, dv=dv, stream=stream)
+        if marks is not None:
+            marks[4].record(stream)
+
+    launches_per_step = 5 + (1 if w.rope else 0) + 1 + (3 if w.backward else 0)
+    for _ in range(args.warmup):
+        step()
+    _lib.pp_get_status(stream)
+
+    marks = [[ev() for _ in range(n_marks)] for _ in range(args.steps)]
+    t0, t1 = ev(), ev()
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    t0.record(stream)
+    for s in range(args.steps):
+        step(marks[s])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    _lib.pp_get_status(stream)
+    ms = t0.elapsed_time(t1)
+    parts = {"build_meta": 0.0, "rope": 0.0, "attn_fwd": 0.0, "attn_bwd": 0.0}
+    for m in marks:
+        for key, a, b in (("build_meta", 0, 1), ("rope", 1, 2), ("attn_fwd", 2, 3), ("attn_bwd", 3, 4)):
+            parts[key] += m[a].elapsed_time(m[b]) / args.steps
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    total_flops = (f_fwd + f_bwd) * world
+    value = total_flops / (ms_per_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {x: inp[x].pin_memory() for x in (("q", "k", "v", "dout") if w.backward else ("q", "k", "v"))}
+        outs = {"dq": torch.empty_like(inp["q"]).pin_memory(), "dk": torch.empty_like(inp["k"]).pin_memory(),
+                "dv": torch.empty_like(inp["v"]).pin_memory()} if w.backward else {
+            "o": torch.empty_like(inp["q"]).pin_memory(), "lse": torch.empty(hq, T).pin_memory()}
+        h2d = sum(t_.numel() * t_.element_size() for t_ in host.values())
+        d2h = sum(t_.numel() * t_.element_size() for t_ in outs.values())
+        e_steps = max(2, min(args.steps, 10))
+
+        def e2e_step():
+            q.copy_(host["q"], non_blocking=True)
+            k.copy_(host["k"], non_blocking=True)
+            v.copy_(host["v"], non_blocking=True)
+            if w.backward:
+                dout.copy_(host["dout"], non_blocking=True)
+            step()
+            if w.backward:
+                outs["dq"].copy_(dq, non_blocking=True)
+                outs["dk"].copy_(dk, non_blocking=True)
+                outs["dv"].copy_(dv, non_blocking=True)
+            else:
+                outs["o"].copy_(o, non_blocking=True)
+                outs["lse"].copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        te = torch.tensor([a.elapsed_time(b) / e_steps], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": round(total_flops / (float(te.item()) * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "ms_per_step": round(float(te.item()), 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks = load_peaks()
+    dom = "attn_bwd" if w.backward and parts["attn_bwd"] >= parts["attn_fwd"] else "attn_fwd"
+    dom_flops = f_bwd if dom == "attn_bwd" else f_fwd
+    achieved = dom_flops / (parts[dom] * 1e-3) / 1e12
+    kernel_name = "k_bwd_tc" if dom == "attn_bwd" else "k_attn_fwd_tc"
+    roofline = {"bound": "tensor", "kernel": f"pp_{dom} ({kernel_name} + its helper kernels)",
+                "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": recorded_traffic(kernel_name),
+                "peak_source": peaks["source"] + " bf16_tflops (burst)",
+                "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4)
+                if peaks.get("bf16_tflops_sustained") else None,
+                "flops_per_launch": dom_flops, "ms_per_launch": round(parts[dom], 4)}
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu = cpu_baseline(name, P, S, seconds=args.cpu_seconds)
+    line = {
+        "metric": "packed-prefix attn fwd+bwd useful TFLOP/s", "value": round(value, 2), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16"
+        else "fp32", "data": "synthetic",
+        "config": {"workload": f"{name}: {w.description}", "T": T, "groups": len(P), "allowed_pairs_per_head": pairs,
+                   "unpacked_pairs_per_head": unpacked_pairs(P, S), "useful_gflop_per_rank": (f_fwd + f_bwd) / 1e9,
+                   "l2": f"inputs larger than L2 ({(q.numel() + k.numel() + v.numel()) * 2 / 2**20:.0f} MiB of Q/K/V "
+                         f"per rank vs 126 MiB), no flush", "parallelism": f"weak-scaled replicas x{world}"},
+        "frac_of_peak": round(value / world / peaks["bf16_tflops"], 4),
+        "ms_per_call": {k_: round(v_, 4) for k_, v_ in parts.items()},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------------- CPU oracle
+def cpu_baseline(name, P, S, seconds=15.0, steps=1):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the workload: whole groups, fwd (+bwd)."""
+    import oracle
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(name, P, S)
+    lay = oracle.layout_of(P, S)
+    hq, hkv = w.num_heads_q, w.num_heads_kv
+    r = hq // hkv
+    # take one kv head (and its r q heads) of as many groups as fit roughly in the budget, smallest first
+    order = sorted(range(len(P)), key=lambda g: int(lay.group_len[g]))
+    chosen, flops, t_used = [], 0, 0.0
+    t_start = time.perf_counter()
+    for g in order:
+        if chosen and time.perf_counter() - t_start > seconds:
+            break
+        gp = pair_count([P[g]], [S[g]])
+        t0 = time.perf_counter()
+        oracle.attention_forward(inp["q"], inp["k"], inp["v"], P, S, heads=list(range(r)), groups=[g])
+        if w.backward:
+            oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["dout"], P, S, groups=[g], kv_heads=[0])
+        t_used += time.perf_counter() - t0
+        flops += (4 + (10 if w.backward else 0)) * w.head_dim * gp * r
+        chosen.append(g)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # pragma: no cover
+        cores = 1
+    return {"value": round(flops / t_used / 1e12, 6), "unit": "TFLOP/s", "cores": int(cores), "kind": "oracle",
+            "sample": f"{len(chosen)} whole group(s) of {len(P)}, kv head 0 with its {r} q heads, "
+                      f"fwd{'+bwd' if w.backward else ''}, fp64 numpy ({flops / 1e9:.1f} useful GFLOP in "
+                      f"{t_used:.1f} s)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    name = args.workload
+    P, S = W.group_lengths(name)
+    per = []
+    info = None
+    for _ in range(args.warmup + args.steps):
+        info = cpu_baseline(name, P, S, seconds=args.cpu_seconds / max(1, args.steps))
+        per.append(info)
+    vals = [x["value"] for x in per[args.warmup:]]
+    value = statistics.median(vals)
+    w = W.WORKLOADS[name]
+    line = {"impl": "reference", "metric": "packed-prefix attn fwd+bwd useful TFLOP/s", "value": value,
+            "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{name}: {w.description}", "T": W.packed_total(P, S)},
+            "cpu_baseline": {"kind": "oracle", "cores": info["cores"], "sample": info["sample"], "value": value},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()
