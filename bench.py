@@ -54,6 +54,25 @@ def flops_of(name, P, S):
                                                           if w.backward else 0)
 
 
+def rank_tensor_seed(name, rank):
+    """Each rank draws its own batch of the same shape (weak scaling: per-GPU work fixed as N grows)."""
+    return W.WORKLOADS[name].tensor_seed + 7919 * rank
+
+
+def max_over_ranks(value, device, dist=None):
+    """Max of a per-rank float over all ranks (the step time the job is charged with)."""
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(flops_per_rank, world, ms_per_step):
+    """Whole-job throughput: the useful FLOPs of all ranks over the slowest rank's step time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -163,7 +182,7 @@ def run_gpu(args):
     name = args.workload
     w = W.WORKLOADS[name]
     P, S = W.group_lengths(name)
-    inp = W.make_inputs(name, P, S, seed=w.tensor_seed + 7919 * rank)   # each rank its own batch
+    inp = W.make_inputs(name, P, S, seed=rank_tensor_seed(name, rank))
     hq, hkv, d = w.num_heads_q, w.num_heads_kv, w.head_dim
     T = W.packed_total(P, S)
     pairs, f_fwd, f_bwd = flops_of(name, P, S)
@@ -223,13 +242,9 @@ def run_gpu(args):
     for m in marks:
         for key, a, b in (("build_meta", 0, 1), ("rope", 1, 2), ("attn_fwd", 2, 3), ("attn_bwd", 3, 4)):
             parts[key] += m[a].elapsed_time(m[b]) / args.steps
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    ms_per_step = ms_max / args.steps
+    ms_per_step = max_over_ranks(ms, dev, dist) / args.steps
     total_flops = (f_fwd + f_bwd) * world
-    value = total_flops / (ms_per_step * 1e-3) / 1e12
+    value = aggregate_tflops(f_fwd + f_bwd, world, ms_per_step)
 
     # ---- end to end through the public API with pinned host buffers
     e2e = None
@@ -267,11 +282,9 @@ def run_gpu(args):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize(dev)
-        te = torch.tensor([a.elapsed_time(b) / e_steps], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": round(total_flops / (float(te.item()) * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-               "ms_per_step": round(float(te.item()), 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        te = max_over_ranks(a.elapsed_time(b) / e_steps, dev, dist)
+        e2e = {"value": round(aggregate_tflops(f_fwd + f_bwd, world, te), 2), "unit": "TFLOP/s",
+               "ms_per_step": round(te, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if world > 1:
         dist.barrier()
