@@ -150,6 +150,28 @@ PP_API pp_status pp_attn_bwd(const void *q, const void *k, const void *v, const 
                       void *stream);
 
 /* ---------------------------------------------------------------------------------------------------------------
+ * pp_attn_bwd_noalloc: pp_attn_bwd for callers that cannot allocate device memory.
+ * (The paper has no counterpart; this is a convenience of the library.)
+ * Some callers cannot call cudaMalloc or ask anyone for a scratch buffer: a plugin or custom op handed only its
+ * input and output pointers by a host framework whose caching allocator owns the device memory, or code that must
+ * not allocate at that point. This entry point takes the same arguments as pp_attn_bwd minus the workspace, and
+ * uses instead a scratch array compiled into the library (a file-scope __device__ array of
+ * PP_NOALLOC_SCRATCH_BYTES = 64 MiB; every GPU that loads libpp holds it until the process exits). It calls no
+ * allocator at all.
+ *   Limit: the scratch a call needs (pp_workspace_bytes(PP_PASS_BWD, T, hq, hkv, d)) must fit in 64 MiB, e.g.
+ *   T <= about 2,400 tokens at 32/8 heads and d = 128; a larger call returns PP_ERR_WORKSPACE and enqueues nothing.
+ *   Set-up: the first call on each device looks up the array's device address (cudaGetSymbolAddress) with that
+ *   device current; make that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last call's contents; the call clears the
+ *   parts that must start at zero itself. Calls that overlap on the GPU (other streams, other host threads) race
+ *   on the array: serialise them.
+ */
+#define PP_NOALLOC_SCRATCH_BYTES (64ll << 20)
+PP_API pp_status pp_attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                              const void *dout, const void *meta_d, int64_t T, int32_t hq, int32_t hkv, int32_t d,
+                              float softmax_scale, void *dq, void *dk, void *dv, void *stream);
+
+/* ---------------------------------------------------------------------------------------------------------------
  * pp_get_status: synchronises `stream`, then reads and clears this device's error word. Returns PP_OK,
  * PP_ERR_DEVICE_TIMEOUT, PP_ERR_DEVICE_INPUT or PP_ERR_CUDA (a sticky CUDA error is reported as such).
  */

@@ -40,6 +40,8 @@ SIGNATURES = {
     "pp_attn_fwd": (_I32, [_VP, _VP, _VP, _VP, _I64, _I32, _I32, _I32, _F32, _I32, _VP, _VP, _VP, _I64, _VP]),
     "pp_attn_bwd": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _I32, _I32, _I32, _F32, _VP, _VP, _VP, _VP,
                            _I64, _VP]),
+    "pp_attn_bwd_noalloc": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _I32, _I32, _I32, _F32, _VP, _VP, _VP,
+                                   _VP]),
     "pp_get_status": (_I32, [_VP]),
     "pp_last_error": (ctypes.c_char_p, []),
     "pp_version": (ctypes.c_char_p, []),
@@ -152,6 +154,17 @@ def pp_attn_bwd(q, k, v, o, lse, dout, meta_d, dq, dk, dv, workspace, softmax_sc
     _call("pp_attn_bwd", _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(meta_d), T, hq, hkv, d,
           float(softmax_scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
           workspace.numel() * workspace.element_size(), _stream(stream))
+
+
+def pp_attn_bwd_noalloc(q, k, v, o, lse, dout, meta_d, dq, dk, dv, softmax_scale: float = 0.0, stream=None):
+    """pp_attn_bwd without a workspace argument: the library's built-in 64 MiB scratch is used instead."""
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    _call("pp_attn_bwd_noalloc", _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(meta_d), T, hq,
+          hkv, d, float(softmax_scale), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream))
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 def pp_get_status(stream=None) -> int:

@@ -124,6 +124,28 @@ int grid_for(int sm_count, int per_sm, int64_t work) {
     return int(g < 1 ? 1 : g);
 }
 
+// Scratch of pp_attn_bwd_noalloc (see include/pp.h): compiled into the library so that callers who cannot
+// allocate still get a backward. Host code must not use the symbol's host-side name as a device address; the
+// device address is looked up once per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PP_NOALLOC_SCRATCH_BYTES];
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+pp_status noalloc_scratch(void **out) {
+    int dev = 0;
+    PP_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(PP_ERR_CUDA, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // with `dev` current
+        if (e != cudaSuccess || !p)
+            return fail(PP_ERR_CUDA, "cudaGetSymbolAddress(noalloc scratch): %s", cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return PP_OK;
+}
+
 }  // namespace
 
 // =====================================================================================================================
@@ -312,6 +334,25 @@ pp_status pp_attn_bwd(const void *q, const void *k, const void *v, const void *o
     if ((st = device_info(&di)) != PP_OK) return st;
     return pp::launch_bwd(q, k, v, o, lse, dout, meta_d, T, hq, hkv, d, scale, dq, dk, dv, workspace, di->sm_count,
                           as_stream(stream), make_map_3d, fail);
+}
+
+pp_status pp_attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                              const void *dout, const void *meta_d, int64_t T, int32_t hq, int32_t hkv, int32_t d,
+                              float softmax_scale, void *dq, void *dk, void *dv, void *stream) {
+    pp_status st = check_heads(T, hq, hkv, d);
+    if (st != PP_OK) return st;
+    int64_t need = 0;
+    if ((st = pp_workspace_bytes(PP_PASS_BWD, T, hq, hkv, d, &need)) != PP_OK) return st;
+    if (need > PP_NOALLOC_SCRATCH_BYTES)
+        return fail(PP_ERR_WORKSPACE,
+                    "pp_attn_bwd_noalloc: these sizes need %lld bytes of scratch but the built-in array holds %lld; "
+                    "call pp_attn_bwd with a caller workspace instead",
+                    (long long)need, (long long)PP_NOALLOC_SCRATCH_BYTES);
+    if (T == 0) return PP_OK;
+    void *scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != PP_OK) return st;
+    return pp_attn_bwd(q, k, v, o, lse, dout, meta_d, T, hq, hkv, d, softmax_scale, dq, dk, dv, scratch,
+                       PP_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 pp_status pp_get_status(void *stream) {
