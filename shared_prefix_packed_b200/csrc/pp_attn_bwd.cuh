@@ -16,13 +16,18 @@
 //                   softmax warps: P^T = exp(S^T - lse), dS^T = P^T (dP^T - D)   -> TMEM (bf16) and smem (bf16)
 //                   dV  += P^T dO        (A from TMEM)                  TMEM dV
 //                   dK  += dS^T Q        (A from TMEM)                  TMEM dK
-//                   dQ^T = K^T dS^T      (M=128 = d, N=64 queries)      TMEM S[b] (reused once P^T is consumed)
+//                   dQ^T = K^T dS^T      (M=128 = d, N=64 queries)      TMEM dP[b] (free once dS^T is consumed)
 //                 dQ^T is read by a second warpgroup, scaled, staged in smem and added to an fp32 accumulator
-//                 with one bulk reduce-add per step. dK/dV stay in TMEM for the whole item; an unsplit key tile
+//                 with bulk reduce-adds (two 16 KiB halves per step, so staging overlaps the previous add). dK/dV stay in TMEM for the whole item; an unsplit key tile
 //                 writes them as bf16, a split one adds its fp32 partial into the workspace (one add per chunk).
 //   k_bwd_convert dQ (and the split tiles' dK/dV) from the fp32 accumulators to bf16.
 // TMEM (512 columns): S[0] [0,64), S[1] [64,128), dP[0] [128,192), dP[1] [192,256), dV [256,384), dK [384,512).
-// S/dP are double-buffered so the MMAs of step t+1 run while the softmax warps work on step t.
+// S/dP are double-buffered so the MMAs of step t+1 run while the softmax warps work on step t. dQ^T(t) lands in
+// dP[b]; the only MMA that must wait for the dQ warps to read it is dP^T(t+2), and S^T(t+2) is issued first.
+// The producer fetches each step's (lse * log2 e, D) pairs with one bulk copy: the preprocess kernel packs them
+// into the workspace with padding, so the copy can start at a 16-byte boundary below the tile's first row.
+// Work items run kv-head-major: concurrently running CTAs share a kv head, so a group's Q/dO rows and dQ
+// accumulator rows are reused from L2 across its key tiles.
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -37,7 +42,7 @@ constexpr int BWD_D = 128;
 
 struct BwdWorkspace {
     int64_t rows_pad;   // T + padding rows so tiles that stick out past T stay inside the buffers
-    int64_t off_delta;  // fp32 [hq][rows_pad]: D_i = dO_i . O_i
+    int64_t off_delta;  // float2 [hq][rows_pad]: (lse_i * log2 e, D_i = dO_i . O_i)
     int64_t off_dq;     // fp32 [hq][rows_pad][d]: dQ accumulator
     int64_t off_dk;     // fp32 [rows_pad][hkv][d]: dK accumulator of split key tiles
     int64_t off_dv;     // fp32 [rows_pad][hkv][d]: dV accumulator of split key tiles
@@ -46,9 +51,9 @@ struct BwdWorkspace {
 
 inline BwdWorkspace bwd_workspace_layout(int64_t T, int hq, int hkv, int d) {
     BwdWorkspace w{};
-    w.rows_pad = T + 256;
+    w.rows_pad = (T + 256 + 7) & ~int64_t(7);
     int64_t o = 0;
-    w.off_delta = o; o = align256(o + 4 * int64_t(hq) * w.rows_pad);
+    w.off_delta = o; o = align256(o + 8 * int64_t(hq) * w.rows_pad);
     w.off_dq = o;    o = align256(o + 4 * int64_t(hq) * w.rows_pad * d);
     w.off_dk = o;    o = align256(o + 4 * w.rows_pad * hkv * d);
     w.off_dv = o;    o = align256(o + 4 * w.rows_pad * hkv * d);
@@ -57,9 +62,10 @@ inline BwdWorkspace bwd_workspace_layout(int64_t T, int hq, int hkv, int d) {
 }
 
 // ------------------------------------------------------------------------------------------------- preprocess
-// One warp per (row, head): D = sum_d dO * O in fp32; padding rows get 0.
+// One warp per (row, head): (lse * log2 e, D = sum_d dO * O) in fp32; padding rows get (0, 0).
 __global__ void k_bwd_pre(const __nv_bfloat16 *__restrict__ O, const __nv_bfloat16 *__restrict__ dO,
-                          float *__restrict__ delta, int64_t T, int64_t rows_pad, int hq) {
+                          const float *__restrict__ lse, float2 *__restrict__ ld, int64_t T, int64_t rows_pad,
+                          int hq) {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = int64_t(gridDim.x) * (blockDim.x >> 5);
     for (int64_t w = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < rows_pad * hq; w += nwarps) {
@@ -78,7 +84,9 @@ __global__ void k_bwd_pre(const __nv_bfloat16 *__restrict__ O, const __nv_bfloat
         }
 #pragma unroll
         for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) delta[int64_t(h) * rows_pad + i] = acc;
+        if (lane == 0)
+            ld[int64_t(h) * rows_pad + i] = make_float2(i < T ? lse[int64_t(h) * T + i] * 1.4426950408889634f : 0.f,
+                                                        acc);
     }
 }
 
@@ -89,14 +97,14 @@ struct BwdSmem {
     static constexpr int QT_BYTES = 64 * BWD_D * 2;      // 64 query rows x d
     static constexpr int QT_CHUNK = 64 * 64 * 2;
     static constexpr int DS_BYTES = 128 * 64 * 2;        // dS^T: 128 key rows x 64 queries, bf16
+    static constexpr int LD_PAIRS = 66;                  // 64 rows + 1 alignment slack, rounded to 16 bytes
     alignas(1024) uint8_t k[KV_BYTES];
     alignas(1024) uint8_t v[KV_BYTES];
     alignas(1024) uint8_t q[2][QT_BYTES];
     alignas(1024) uint8_t dout[2][QT_BYTES];
     alignas(1024) uint8_t ds[2][DS_BYTES];
-    alignas(1024) float stage[64 * BWD_D];               // dQ tile [64 queries][d] for the bulk add
-    float lse2[2][64];                                   // lse * log2(e) of the step's query rows
-    float dl[2][64];                                     // D of the step's query rows
+    alignas(1024) float stage[64 * BWD_D];               // dQ tile [64 queries][d] for the bulk adds (2 halves)
+    alignas(16) float2 ld[2][LD_PAIRS];                  // (lse * log2 e, D) of the step's rows, from 16-B boundary
     uint64_t kv_full, kv_empty, dkv_full, dkv_free;
     uint64_t q_full[2], q_empty[2], sdp_full[2], ds_full[2], ds_free[2], dq_full[2], dq_free[2];
     uint32_t tmem_base;
@@ -109,9 +117,9 @@ struct BwdItem {
 };
 
 __device__ __forceinline__ BwdItem bwd_decode(const void *meta, const MetaHeader &hd, int item, int hkv) {
-    const BWork w = meta_ptr<BWork>(meta, hd.off_bw)[item / hkv];
+    const BWork w = meta_ptr<BWork>(meta, hd.off_bw)[item % hd.n_bw];
     BwdItem it;
-    it.kh = item % hkv;
+    it.kh = item / hd.n_bw;
     it.t = meta_ptr<KTile>(meta, hd.off_kt)[w.kt];
     it.qa = w.qa;
     it.qb = w.qb;
@@ -130,7 +138,7 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-         const void *__restrict__ meta, const float *__restrict__ LSE, const float *__restrict__ delta,
+         const void *__restrict__ meta, const float2 *__restrict__ ldg,
          float *__restrict__ dq_acc, float *__restrict__ dk_acc, float *__restrict__ dv_acc,
          __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV, int hq, int hkv, int64_t rows_pad,
          float scale, float sl2) {
@@ -142,7 +150,6 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     const int r = hq / hkv;
     const int n_items = hd.n_bw * hkv;
     volatile int *abort_flag = &sm.abort_flag;
-    constexpr float LOG2E = 1.4426950408889634f;
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.kv_full, 1);
@@ -150,7 +157,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         mbar_init(&sm.dkv_full, 1);
         mbar_init(&sm.dkv_free, 128);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm.q_full[b], 32);
+            mbar_init(&sm.q_full[b], 1);
             mbar_init(&sm.q_empty[b], 1);
             mbar_init(&sm.sdp_full[b], 1);
             mbar_init(&sm.ds_full[b], 128);
@@ -180,39 +187,31 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     if (hd.dev_err != 0) {
         // nothing to do: the metadata builder rejected its input
     } else if (warp == 8) {
-        // ------------------------------------------------------------------ producer warp
-        uint32_t g = 0, it_n = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
-            const BwdItem w = bwd_decode(meta, hd, item, hkv);
-            if (lane == 0) {
+        // ------------------------------------------------------------------ producer (one thread)
+        if (lane == 0) {
+            uint32_t g = 0, it_n = 0;
+            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+                const BwdItem w = bwd_decode(meta, hd, item, hkv);
                 if (!bwait(&sm.kv_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
                 mbar_arrive_expect_tx(&sm.kv_full, 2 * BwdSmem::KV_BYTES);
                 for (int c = 0; c < BWD_D / 64; ++c) {
                     tma_load_3d(sm.k + c * BwdSmem::KV_CHUNK, &tmK, c * 64, w.kh, w.t.row0, &sm.kv_full);
                     tma_load_3d(sm.v + c * BwdSmem::KV_CHUNK, &tmV, c * 64, w.kh, w.t.row0, &sm.kv_full);
                 }
-            }
-            const int n = (w.qb - w.qa) * r;
-            for (int t = 0; t < n; ++t, ++g) {
-                const int b = g & 1;
-                const int h = w.kh * r + t % r;
-                const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
-                if (!bwait(&sm.q_empty[b], ((g >> 1) & 1) ^ 1, abort_flag)) goto done;
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int i = lane + 32 * e;
-                    const int row = x0 + i;
-                    sm.lse2[b][i] = row < T ? LSE[int64_t(h) * T + row] * LOG2E : 0.f;
-                    sm.dl[b][i] = delta[int64_t(h) * rows_pad + row];
-                }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&sm.q_full[b], 2 * BwdSmem::QT_BYTES);
+                const int n = (w.qb - w.qa) * r;
+                for (int t = 0; t < n; ++t, ++g) {
+                    const int b = g & 1;
+                    const int h = w.kh * r + t % r;
+                    const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
+                    if (!bwait(&sm.q_empty[b], ((g >> 1) & 1) ^ 1, abort_flag)) goto done;
+                    mbar_arrive_expect_tx(&sm.q_full[b], 2 * BwdSmem::QT_BYTES + BwdSmem::LD_PAIRS * 8);
                     for (int c = 0; c < BWD_D / 64; ++c) {
                         tma_load_3d(sm.q[b] + c * BwdSmem::QT_CHUNK, &tmQ, c * 64, h, x0, &sm.q_full[b]);
                         tma_load_3d(sm.dout[b] + c * BwdSmem::QT_CHUNK, &tmdO, c * 64, h, x0, &sm.q_full[b]);
                     }
-                } else {
-                    mbar_arrive(&sm.q_full[b]);
+                    // (lse, D) pairs of rows [x0 & ~1, +66): a 16-byte aligned, padded slice of the workspace
+                    bulk_load(sm.ld[b], ldg + int64_t(h) * rows_pad + (x0 & ~1), BwdSmem::LD_PAIRS * 8,
+                              &sm.q_full[b]);
                 }
             }
         }
@@ -224,8 +223,8 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             constexpr uint32_t ID_DQ = idesc_bf16(128, BWD_BM, 1, 1);      // dQ^T (A and B MN-major)
             const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
             uint32_t g = 0, it_n = 0;
-            auto issue_sdp = [&](int b) {
-                const uint32_t sq = smem_u32(sm.q[b]), sdo = smem_u32(sm.dout[b]);
+            auto issue_s = [&](int b) {
+                const uint32_t sq = smem_u32(sm.q[b]);
 #pragma unroll
                 for (int kk = 0; kk < BWD_D / 16; ++kk) {
                     const uint32_t ok = (kk >> 2) * BwdSmem::KV_CHUNK + (kk & 3) * 32;
@@ -233,6 +232,9 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     umma_ss(tmem + COL_S + b * 64, smem_desc(sk + ok, 16, 1024), smem_desc(sq + oq, 16, 1024),
                             ID_SDP, kk > 0);
                 }
+            };
+            auto issue_dp = [&](int b) {
+                const uint32_t sdo = smem_u32(sm.dout[b]);
 #pragma unroll
                 for (int kk = 0; kk < BWD_D / 16; ++kk) {
                     const uint32_t ok = (kk >> 2) * BwdSmem::KV_CHUNK + (kk & 3) * 32;
@@ -241,30 +243,27 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                             ID_SDP, kk > 0);
                 }
             };
+            // S^T/dP^T of step g1 into buffers g1 & 1: S at once, dP once the dQ warps have read dQ^T(g1 - 2)
+            auto issue_sdp = [&](uint32_t g1) -> bool {
+                const int b = g1 & 1;
+                if (!bwait(&sm.q_full[b], (g1 >> 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                issue_s(b);
+                if (!bwait(&sm.dq_free[b], ((g1 >> 1) & 1) ^ 1, abort_flag)) return false;
+                tc_fence_after();
+                issue_dp(b);
+                umma_commit(&sm.sdp_full[b]);
+                return true;
+            };
             for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
                 const BwdItem w = bwd_decode(meta, hd, item, hkv);
                 const int n = (w.qb - w.qa) * r;
                 if (!bwait(&sm.kv_full, it_n & 1, abort_flag)) goto done;
-                // S^T / dP^T of the item's first step
-                {
-                    const int b = g & 1;
-                    if (!bwait(&sm.q_full[b], (g >> 1) & 1, abort_flag)) goto done;
-                    if (!bwait(&sm.dq_free[b], ((g >> 1) & 1) ^ 1, abort_flag)) goto done;
-                    tc_fence_after();
-                    issue_sdp(b);
-                    umma_commit(&sm.sdp_full[b]);
-                }
+                if (!issue_sdp(g)) goto done;
                 if (!bwait(&sm.dkv_free, (it_n & 1) ^ 1, abort_flag)) goto done;
                 for (int t = 0; t < n; ++t, ++g) {
-                    const int b = g & 1, b1 = (g + 1) & 1;
-                    if (t + 1 < n) {
-                        const uint32_t g1 = g + 1;
-                        if (!bwait(&sm.q_full[b1], (g1 >> 1) & 1, abort_flag)) goto done;
-                        if (!bwait(&sm.dq_free[b1], ((g1 >> 1) & 1) ^ 1, abort_flag)) goto done;
-                        tc_fence_after();
-                        issue_sdp(b1);
-                        umma_commit(&sm.sdp_full[b1]);
-                    }
+                    const int b = g & 1;
+                    if (t + 1 < n && !issue_sdp(g + 1)) goto done;
                     if (!bwait(&sm.ds_full[b], (g >> 1) & 1, abort_flag)) goto done;
                     tc_fence_after();
                     const uint32_t sq = smem_u32(sm.q[b]), sdo = smem_u32(sm.dout[b]), sds = smem_u32(sm.ds[b]);
@@ -276,12 +275,12 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     for (int kk = 0; kk < BWD_BM / 16; ++kk)       // dK += dS^T Q
                         umma_ts(tmem + COL_DK, tmem + COL_DP + b * 64 + kk * 8,
                                 smem_desc(sq + kk * 2048, BwdSmem::QT_CHUNK, 1024), ID_KV, (t > 0 || kk > 0));
+                    umma_commit(&sm.q_empty[b]);
 #pragma unroll
-                    for (int kk = 0; kk < 128 / 16; ++kk)          // dQ^T = K^T dS^T
-                        umma_ss(tmem + COL_S + b * 64, smem_desc(sk + kk * 2048, BwdSmem::KV_CHUNK, 1024),
+                    for (int kk = 0; kk < 128 / 16; ++kk)          // dQ^T = K^T dS^T, into dP[b]
+                        umma_ss(tmem + COL_DP + b * 64, smem_desc(sk + kk * 2048, BwdSmem::KV_CHUNK, 1024),
                                 smem_desc(sds + kk * 2048, BwdSmem::DS_BYTES, 1024), ID_DQ, kk > 0);
                     umma_commit(&sm.dq_full[b]);
-                    umma_commit(&sm.q_empty[b]);
                     umma_commit(&sm.ds_free[b]);
                 }
                 umma_commit(&sm.dkv_full);
@@ -304,64 +303,45 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             for (int t = 0; t < n; ++t, ++g) {
                 const int b = g & 1;
                 const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
+                const float2 *ldp = sm.ld[b] + (x0 & 1);
                 if (!bwait(&sm.ds_free[b], ((g >> 1) & 1) ^ 1, abort_flag)) goto done;
                 if (!bwait(&sm.sdp_full[b], (g >> 1) & 1, abort_flag)) goto done;
                 if (!bwait(&sm.q_full[b], (g >> 1) & 1, abort_flag)) goto done;
                 tc_fence_after();
-                uint32_t sr[64], pr[64];
-                {
-                    uint32_t tmp[32];
-                    tmem_ld32(tmem + lane_off + COL_S + b * 64, tmp);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) sr[e] = tmp[e];
-                    tmem_ld32(tmem + lane_off + COL_S + b * 64 + 32, tmp);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) sr[32 + e] = tmp[e];
-                    tmem_ld32(tmem + lane_off + COL_DP + b * 64, tmp);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) pr[e] = tmp[e];
-                    tmem_ld32(tmem + lane_off + COL_DP + b * 64 + 32, tmp);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) pr[32 + e] = tmp[e];
-                    tmem_wait_ld();
-                }
                 const int lo = y - x0, hi = ke - x0;                   // allowed query columns [lo, hi)
-                uint32_t pp[32], dd[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float p2[2], d2[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int c = 2 * e + u;
-                        const bool ok = c >= lo && c < hi;
-                        const float p = ok ? ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -sm.lse2[b][c])) : 0.f;
-                        p2[u] = p;
-                        d2[u] = p * (__uint_as_float(pr[c]) - sm.dl[b][c]);
-                    }
-                    pp[e] = pack_bf16x2(p2[0], p2[1]);
-                    dd[e] = pack_bf16x2(d2[0], d2[1]);
-                }
-                {
-                    uint32_t tmp[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) tmp[e] = pp[e];
-                    tmem_st16(tmem + lane_off + COL_S + b * 64, tmp);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) tmp[e] = pp[16 + e];
-                    tmem_st16(tmem + lane_off + COL_S + b * 64 + 16, tmp);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) tmp[e] = dd[e];
-                    tmem_st16(tmem + lane_off + COL_DP + b * 64, tmp);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) tmp[e] = dd[16 + e];
-                    tmem_st16(tmem + lane_off + COL_DP + b * 64 + 16, tmp);
-                }
-                // dS^T row jr into the 128-byte-swizzled [key][query] tile read by the dQ MMA
                 uint8_t *dsrow = sm.ds[b] + jr * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4 *>(dsrow + ((c ^ (jr & 7)) << 4)) =
-                        make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t sr[32], pr[32];
+                    tmem_ld32(tmem + lane_off + COL_S + b * 64 + half * 32, sr);
+                    tmem_ld32(tmem + lane_off + COL_DP + b * 64 + half * 32, pr);
+                    tmem_wait_ld();
+                    uint32_t pp[16], dd[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float p2[2], d2[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int cl = 2 * e + u, c = half * 32 + cl;
+                            const float2 l2 = ldp[c];
+                            const bool ok = c >= lo && c < hi;
+                            const float p = ok ? ex2_approx(fmaf(__uint_as_float(sr[cl]), sl2, -l2.x)) : 0.f;
+                            p2[u] = p;
+                            d2[u] = p * (__uint_as_float(pr[cl]) - l2.y);
+                        }
+                        pp[e] = pack_bf16x2(p2[0], p2[1]);
+                        dd[e] = pack_bf16x2(d2[0], d2[1]);
+                    }
+                    tmem_st16(tmem + lane_off + COL_S + b * 64 + half * 16, pp);
+                    tmem_st16(tmem + lane_off + COL_DP + b * 64 + half * 16, dd);
+                    // dS^T row jr, queries [32 half, +32), into the 128-byte-swizzled [key][query] tile
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int ch = half * 4 + c;
+                        *reinterpret_cast<uint4 *>(dsrow + ((ch ^ (jr & 7)) << 4)) =
+                            make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+                    }
+                }
                 tmem_wait_st();
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -419,32 +399,36 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 uint32_t v[64];
                 {
                     uint32_t tmp[32];
-                    tmem_ld32(tmem + lane_off + COL_S + b * 64, tmp);
+                    tmem_ld32(tmem + lane_off + COL_DP + b * 64, tmp);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) v[e] = tmp[e];
-                    tmem_ld32(tmem + lane_off + COL_S + b * 64 + 32, tmp);
+                    tmem_ld32(tmem + lane_off + COL_DP + b * 64 + 32, tmp);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) v[32 + e] = tmp[e];
                     tmem_wait_ld();
                 }
                 tc_fence_before();
                 mbar_arrive(&sm.dq_free[b]);
-                if (leader) bulk_wait_read0();                         // the previous add has read the stage
-                named_bar_sync(1, 128);
+                float *gdst = dq_acc + (int64_t(h) * rows_pad + x0) * BWD_D;
 #pragma unroll
-                for (int c = 0; c < 64; ++c) sm.stage[c * BWD_D + dcol] = __uint_as_float(v[c]) * scale;
-                fence_proxy_async_smem();
-                named_bar_sync(1, 128);
-                if (leader) {
-                    bulk_reduce_add_f32(dq_acc + (int64_t(h) * rows_pad + x0) * BWD_D, sm.stage,
-                                        64 * BWD_D * sizeof(float));
-                    bulk_commit();
+                for (int half = 0; half < 2; ++half) {
+                    float *stg = sm.stage + half * 32 * BWD_D;
+                    if (leader) bulk_wait_read1();                     // this half's previous add has read it
+                    named_bar_sync(1, 128);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) stg[c * BWD_D + dcol] = __uint_as_float(v[half * 32 + c]) * scale;
+                    fence_proxy_async_smem();
+                    named_bar_sync(1, 128);
+                    if (leader) {
+                        bulk_reduce_add_f32(gdst + half * 32 * BWD_D, stg, 32 * BWD_D * sizeof(float));
+                        bulk_commit();
+                    }
                 }
             }
         }
-        if (leader) bulk_wait0();
     }
 done:
+    if (warp == 4 && lane == 0) bulk_wait0();   // no bulk add may still read shared memory when the CTA exits
     tc_fence_before();
     __syncthreads();
     if (warp == 9) {
@@ -506,7 +490,7 @@ inline pp_status launch_bwd(const void *q, const void *k, const void *v, const v
     if (d != BWD_D) return fail(PP_ERR_UNSUPPORTED, "backward supports head dim 128 only (got %d)", d);
     const BwdWorkspace L = bwd_workspace_layout(T, hq, hkv, d);
     char *ws = static_cast<char *>(workspace);
-    float *delta = reinterpret_cast<float *>(ws + L.off_delta);
+    float2 *ldg = reinterpret_cast<float2 *>(ws + L.off_delta);
     float *dq_acc = reinterpret_cast<float *>(ws + L.off_dq);
     float *dk_acc = reinterpret_cast<float *>(ws + L.off_dk);
     float *dv_acc = reinterpret_cast<float *>(ws + L.off_dv);
@@ -523,12 +507,12 @@ inline pp_status launch_bwd(const void *q, const void *k, const void *v, const v
     if ((e = cudaMemsetAsync(ws + L.off_dq, 0, L.total - L.off_dq, s)) != cudaSuccess)
         return fail(PP_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
     k_bwd_pre<<<sm_count * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(o),
-                                           static_cast<const __nv_bfloat16 *>(dout), delta, T, L.rows_pad, hq);
+                                           static_cast<const __nv_bfloat16 *>(dout), lse, ldg, T, L.rows_pad, hq);
     if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_pre: %s", cudaGetErrorString(e));
     const size_t smem = sizeof(BwdSmem) + 1024;
     if ((e = cudaFuncSetAttribute(k_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem))) != cudaSuccess)
         return fail(PP_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    k_bwd_tc<<<sm_count, BWD_THREADS, smem, s>>>(mq, mk, mv, mdo, meta, lse, delta, dq_acc, dk_acc, dv_acc,
+    k_bwd_tc<<<sm_count, BWD_THREADS, smem, s>>>(mq, mk, mv, mdo, meta, ldg, dq_acc, dk_acc, dv_acc,
                                                  static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv),
                                                  hq, hkv, L.rows_pad, scale, scale * 1.4426950408889634f);
     if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_tc: %s", cudaGetErrorString(e));
