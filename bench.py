@@ -217,17 +217,18 @@ def run_gpu(args):
             marks[4].record(stream)
 
     launches_per_step = 5 + (1 if w.rope else 0) + 1 + (3 if w.backward else 0)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)                      # nvidia-smi needs a moment before its first sample
     for _ in range(args.warmup):
         step()
     _lib.pp_get_status(stream)
 
     marks = [[ev() for _ in range(n_marks)] for _ in range(args.steps)]
     t0, t1 = ev(), ev()
-    sampler = ClockSampler(local)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    sampler.start()
     t0.record(stream)
     for s in range(args.steps):
         step(marks[s])
@@ -385,7 +386,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])

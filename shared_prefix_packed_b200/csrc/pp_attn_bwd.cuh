@@ -18,7 +18,7 @@
 //                   dK  += dS^T Q        (A from TMEM)                  TMEM dK
 //                   dQ^T = K^T dS^T      (M=128 = d, N=64 queries)      TMEM dP[b] (free once dS^T is consumed)
 //                 dQ^T is read by a second warpgroup, scaled, staged in smem and added to an fp32 accumulator
-//                 with bulk reduce-adds (two 16 KiB halves per step, so staging overlaps the previous add). dK/dV stay in TMEM for the whole item; an unsplit key tile
+//                 with bulk reduce-adds (two 16 KiB halves per step through one staging buffer). dK/dV stay in TMEM for the whole item; an unsplit key tile
 //                 writes them as bf16, a split one adds its fp32 partial into the workspace (one add per chunk).
 //   k_bwd_convert dQ (and the split tiles' dK/dV) from the fp32 accumulators to bf16.
 // TMEM (512 columns): S[0] [0,64), S[1] [64,128), dP[0] [128,192), dP[1] [192,256), dV [256,384), dK [384,512).
@@ -98,15 +98,17 @@ struct BwdSmem {
     static constexpr int QT_CHUNK = 64 * 64 * 2;
     static constexpr int DS_BYTES = 128 * 64 * 2;        // dS^T: 128 key rows x 64 queries, bf16
     static constexpr int LD_PAIRS = 66;                  // 64 rows + 1 alignment slack, rounded to 16 bytes
+    static constexpr int QSTAGES = 3;                    // Q/dO ring depth: hides the L2 latency of a step's loads
     alignas(1024) uint8_t k[KV_BYTES];
     alignas(1024) uint8_t v[KV_BYTES];
-    alignas(1024) uint8_t q[2][QT_BYTES];
-    alignas(1024) uint8_t dout[2][QT_BYTES];
+    alignas(1024) uint8_t q[QSTAGES][QT_BYTES];
+    alignas(1024) uint8_t dout[QSTAGES][QT_BYTES];
     alignas(1024) uint8_t ds[2][DS_BYTES];
-    alignas(1024) float stage[64 * BWD_D];               // dQ tile [64 queries][d] for the bulk adds (2 halves)
-    alignas(16) float2 ld[2][LD_PAIRS];                  // (lse * log2 e, D) of the step's rows, from 16-B boundary
+    alignas(1024) float stage[32 * BWD_D];               // half a dQ tile [32 queries][d] for one bulk add
+    alignas(16) float2 ld[QSTAGES][LD_PAIRS];            // (lse * log2 e, D) of the step's rows, from 16-B boundary
     uint64_t kv_full, kv_empty, dkv_full, dkv_free;
-    uint64_t q_full[2], q_empty[2], sdp_full[2], ds_full[2], ds_free[2], dq_full[2], dq_free[2];
+    uint64_t q_full[QSTAGES], q_empty[QSTAGES];
+    uint64_t sdp_full[2], ds_full[2], ds_free[2], dq_full[2], dq_free[2];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -156,9 +158,11 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         mbar_init(&sm.kv_empty, 1);
         mbar_init(&sm.dkv_full, 1);
         mbar_init(&sm.dkv_free, 128);
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < BwdSmem::QSTAGES; ++b) {
             mbar_init(&sm.q_full[b], 1);
             mbar_init(&sm.q_empty[b], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.sdp_full[b], 1);
             mbar_init(&sm.ds_full[b], 128);
             mbar_init(&sm.ds_free[b], 1);
@@ -200,10 +204,10 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 }
                 const int n = (w.qb - w.qa) * r;
                 for (int t = 0; t < n; ++t, ++g) {
-                    const int b = g & 1;
+                    const int b = g % BwdSmem::QSTAGES;
                     const int h = w.kh * r + t % r;
                     const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
-                    if (!bwait(&sm.q_empty[b], ((g >> 1) & 1) ^ 1, abort_flag)) goto done;
+                    if (!bwait(&sm.q_empty[b], ((g / BwdSmem::QSTAGES) & 1) ^ 1, abort_flag)) goto done;
                     mbar_arrive_expect_tx(&sm.q_full[b], 2 * BwdSmem::QT_BYTES + BwdSmem::LD_PAIRS * 8);
                     for (int c = 0; c < BWD_D / 64; ++c) {
                         tma_load_3d(sm.q[b] + c * BwdSmem::QT_CHUNK, &tmQ, c * 64, h, x0, &sm.q_full[b]);
@@ -223,8 +227,8 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             constexpr uint32_t ID_DQ = idesc_bf16(128, BWD_BM, 1, 1);      // dQ^T (A and B MN-major)
             const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
             uint32_t g = 0, it_n = 0;
-            auto issue_s = [&](int b) {
-                const uint32_t sq = smem_u32(sm.q[b]);
+            auto issue_s = [&](int b, int qs) {
+                const uint32_t sq = smem_u32(sm.q[qs]);
 #pragma unroll
                 for (int kk = 0; kk < BWD_D / 16; ++kk) {
                     const uint32_t ok = (kk >> 2) * BwdSmem::KV_CHUNK + (kk & 3) * 32;
@@ -233,8 +237,8 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                             ID_SDP, kk > 0);
                 }
             };
-            auto issue_dp = [&](int b) {
-                const uint32_t sdo = smem_u32(sm.dout[b]);
+            auto issue_dp = [&](int b, int qs) {
+                const uint32_t sdo = smem_u32(sm.dout[qs]);
 #pragma unroll
                 for (int kk = 0; kk < BWD_D / 16; ++kk) {
                     const uint32_t ok = (kk >> 2) * BwdSmem::KV_CHUNK + (kk & 3) * 32;
@@ -245,13 +249,13 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             };
             // S^T/dP^T of step g1 into buffers g1 & 1: S at once, dP once the dQ warps have read dQ^T(g1 - 2)
             auto issue_sdp = [&](uint32_t g1) -> bool {
-                const int b = g1 & 1;
-                if (!bwait(&sm.q_full[b], (g1 >> 1) & 1, abort_flag)) return false;
+                const int b = g1 & 1, qs = g1 % BwdSmem::QSTAGES;
+                if (!bwait(&sm.q_full[qs], (g1 / BwdSmem::QSTAGES) & 1, abort_flag)) return false;
                 tc_fence_after();
-                issue_s(b);
+                issue_s(b, qs);
                 if (!bwait(&sm.dq_free[b], ((g1 >> 1) & 1) ^ 1, abort_flag)) return false;
                 tc_fence_after();
-                issue_dp(b);
+                issue_dp(b, qs);
                 umma_commit(&sm.sdp_full[b]);
                 return true;
             };
@@ -262,11 +266,11 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 if (!issue_sdp(g)) goto done;
                 if (!bwait(&sm.dkv_free, (it_n & 1) ^ 1, abort_flag)) goto done;
                 for (int t = 0; t < n; ++t, ++g) {
-                    const int b = g & 1;
+                    const int b = g & 1, qs = g % BwdSmem::QSTAGES;
                     if (t + 1 < n && !issue_sdp(g + 1)) goto done;
                     if (!bwait(&sm.ds_full[b], (g >> 1) & 1, abort_flag)) goto done;
                     tc_fence_after();
-                    const uint32_t sq = smem_u32(sm.q[b]), sdo = smem_u32(sm.dout[b]), sds = smem_u32(sm.ds[b]);
+                    const uint32_t sq = smem_u32(sm.q[qs]), sdo = smem_u32(sm.dout[qs]), sds = smem_u32(sm.ds[b]);
 #pragma unroll
                     for (int kk = 0; kk < BWD_BM / 16; ++kk)       // dV += P^T dO
                         umma_ts(tmem + COL_DV, tmem + COL_S + b * 64 + kk * 8,
@@ -275,7 +279,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     for (int kk = 0; kk < BWD_BM / 16; ++kk)       // dK += dS^T Q
                         umma_ts(tmem + COL_DK, tmem + COL_DP + b * 64 + kk * 8,
                                 smem_desc(sq + kk * 2048, BwdSmem::QT_CHUNK, 1024), ID_KV, (t > 0 || kk > 0));
-                    umma_commit(&sm.q_empty[b]);
+                    umma_commit(&sm.q_empty[qs]);
 #pragma unroll
                     for (int kk = 0; kk < 128 / 16; ++kk)          // dQ^T = K^T dS^T, into dP[b]
                         umma_ss(tmem + COL_DP + b * 64, smem_desc(sk + kk * 2048, BwdSmem::KV_CHUNK, 1024),
@@ -301,12 +305,12 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             const bool yin = y < gend;
             const int ke = yin ? key_end[y] : y;                       // queries [y, ke) attend key y
             for (int t = 0; t < n; ++t, ++g) {
-                const int b = g & 1;
+                const int b = g & 1, qs = g % BwdSmem::QSTAGES;
                 const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
-                const float2 *ldp = sm.ld[b] + (x0 & 1);
+                const float2 *ldp = sm.ld[qs] + (x0 & 1);
                 if (!bwait(&sm.ds_free[b], ((g >> 1) & 1) ^ 1, abort_flag)) goto done;
                 if (!bwait(&sm.sdp_full[b], (g >> 1) & 1, abort_flag)) goto done;
-                if (!bwait(&sm.q_full[b], (g >> 1) & 1, abort_flag)) goto done;
+                if (!bwait(&sm.q_full[qs], (g / BwdSmem::QSTAGES) & 1, abort_flag)) goto done;
                 tc_fence_after();
                 const int lo = y - x0, hi = ke - x0;                   // allowed query columns [lo, hi)
                 uint8_t *dsrow = sm.ds[b] + jr * 128;
@@ -412,8 +416,8 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 float *gdst = dq_acc + (int64_t(h) * rows_pad + x0) * BWD_D;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    float *stg = sm.stage + half * 32 * BWD_D;
-                    if (leader) bulk_wait_read1();                     // this half's previous add has read it
+                    float *stg = sm.stage;
+                    if (leader) bulk_wait_read0();                     // the previous add has read the stage
                     named_bar_sync(1, 128);
 #pragma unroll
                     for (int c = 0; c < 32; ++c) stg[c * BWD_D + dcol] = __uint_as_float(v[half * 32 + c]) * scale;
