@@ -17,8 +17,9 @@
 //                   dV  += P^T dO        (A from TMEM)                  TMEM dV
 //                   dK  += dS^T Q        (A from TMEM)                  TMEM dK
 //                   dQ^T = K^T dS^T      (M=128 = d, N=64 queries)      TMEM dP[b] (free once dS^T is consumed)
-//                 dQ^T is read by a second warpgroup, scaled, staged in smem and added to an fp32 accumulator
-//                 with bulk reduce-adds (two 16 KiB halves per step through one staging buffer). dK/dV stay in TMEM for the whole item; an unsplit key tile
+//                 dQ^T is read by a second warpgroup (TMEM lane = head-dim index), scaled and added to an fp32
+//                 accumulator straight from registers: per row one coalesced 128-byte red.global.add per warp,
+//                 so dQ costs no shared-memory bandwidth (the MMAs' operand reads already nearly fill it). dK/dV stay in TMEM for the whole item; an unsplit key tile
 //                 writes them as bf16, a split one adds its fp32 partial into the workspace (one add per chunk).
 //   k_bwd_convert dQ (and the split tiles' dK/dV) from the fp32 accumulators to bf16.
 // TMEM (512 columns): S[0] [0,64), S[1] [64,128), dP[0] [128,192), dP[1] [192,256), dV [256,384), dK [384,512).
@@ -104,7 +105,6 @@ struct BwdSmem {
     alignas(1024) uint8_t q[QSTAGES][QT_BYTES];
     alignas(1024) uint8_t dout[QSTAGES][QT_BYTES];
     alignas(1024) uint8_t ds[2][DS_BYTES];
-    alignas(1024) float stage[32 * BWD_D];               // half a dQ tile [32 queries][d] for one bulk add
     alignas(16) float2 ld[QSTAGES][LD_PAIRS];            // (lse * log2 e, D) of the step's rows, from 16-B boundary
     uint64_t kv_full, kv_empty, dkv_full, dkv_free;
     uint64_t q_full[QSTAGES], q_empty[QSTAGES];
@@ -131,6 +131,9 @@ __device__ __forceinline__ BwdItem bwd_decode(const void *meta, const MetaHeader
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void red_add_f32(float *addr, float a) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
 }
 __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
@@ -389,7 +392,6 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         // ------------------------------------------------------------------ dQ warpgroup (warps 4-7)
         const int dcol = (warp - 4) * 32 + lane;                       // head-dim index = TMEM lane
         const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
-        const bool leader = (warp == 4 && lane == 0);
         uint32_t g = 0;
         for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
             const BwdItem w = bwd_decode(meta, hd, item, hkv);
@@ -413,26 +415,14 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 }
                 tc_fence_before();
                 mbar_arrive(&sm.dq_free[b]);
-                float *gdst = dq_acc + (int64_t(h) * rows_pad + x0) * BWD_D;
+                // dQ rows x0..x0+63, column dcol: one coalesced 128-byte add per warp and row
+                float *gdst = dq_acc + (int64_t(h) * rows_pad + x0) * BWD_D + dcol;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float *stg = sm.stage;
-                    if (leader) bulk_wait_read0();                     // the previous add has read the stage
-                    named_bar_sync(1, 128);
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) stg[c * BWD_D + dcol] = __uint_as_float(v[half * 32 + c]) * scale;
-                    fence_proxy_async_smem();
-                    named_bar_sync(1, 128);
-                    if (leader) {
-                        bulk_reduce_add_f32(gdst + half * 32 * BWD_D, stg, 32 * BWD_D * sizeof(float));
-                        bulk_commit();
-                    }
-                }
+                for (int c = 0; c < 64; ++c) red_add_f32(gdst + c * BWD_D, __uint_as_float(v[c]) * scale);
             }
         }
     }
 done:
-    if (warp == 4 && lane == 0) bulk_wait0();   // no bulk add may still read shared memory when the CTA exits
     tc_fence_before();
     __syncthreads();
     if (warp == 9) {
