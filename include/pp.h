@@ -93,7 +93,7 @@ PP_API pp_status pp_build_meta(const pp_group_desc *groups_d, int32_t num_groups
 /* ---------------------------------------------------------------------------------------------------------------
  * pp_meta_tiles: expand the schedule in meta_d into explicit tiles, for checking and inspection.
  *   which = PP_PASS_FWD: query tiles of 128 rows x key tiles of 128 rows; PP_PASS_BWD: key tiles of 128 rows x
- *   query tiles of 64 rows. Both are aligned to each group's start. Writes one int32 triple
+ *   query tiles of 128 rows. Both are aligned to each group's start. Writes one int32 triple
  *   (q_row0, kv_row0, class) per non-empty tile into tiles_d (device int32[3 * capacity]), class 1 = every pair in
  *   the tile allowed (FULL), 2 = some allowed (PARTIAL); fully masked tiles are never listed. *count_d (device
  *   int32) receives the number of tiles (possibly > capacity; only the first `capacity` are written). The order is

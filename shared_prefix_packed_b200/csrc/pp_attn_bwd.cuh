@@ -5,28 +5,29 @@
 //   dK_j = scale sum_h sum_i dS_ij q_i,  dV_j = sum_h sum_i p_ij dO_i   (h over the q heads of j's kv head).
 //
 // Three kernels:
-//   k_bwd_pre     D = rowsum(dO * O) in fp32 (HBM-bound).
+//   k_bwd_pre     (lse * log2 e, D = rowsum(dO * O)) per row and head, fp32 (HBM-bound).
 //   k_bwd_tc      key/value-stationary tensor-core kernel. A work item is (key tile of 128 rows, kv head, chunk of
 //                 the query tiles that attend it). Seen from key y the attending queries are one interval
 //                 [y, e(y)) (pp_meta.cuh), so a key tile's query tiles are one contiguous range; prefix key tiles
 //                 (attended by every response of the group) get long ranges and are split into chunks so the
-//                 persistent grid stays balanced. Per step (query tile of 64 rows, one q head of the kv head):
-//                   S^T  = K Q^T         (M=128 keys, N=64 queries)     TMEM S[b]
-//                   dP^T = V dO^T                                       TMEM dP[b]
-//                   softmax warps: P^T = exp(S^T - lse), dS^T = P^T (dP^T - D)   -> TMEM (bf16) and smem (bf16)
-//                   dV  += P^T dO        (A from TMEM)                  TMEM dV
-//                   dK  += dS^T Q        (A from TMEM)                  TMEM dK
-//                   dQ^T = K^T dS^T      (M=128 = d, N=64 queries)      TMEM dP[b] (free once dS^T is consumed)
+//                 persistent grid stays balanced. Per step (query tile of 128 rows, one q head of the kv head),
+//                 five MMAs, all with N = 128 (an N = 64 MMA costs as long as an N = 128 one on this part):
+//                   S^T  = K Q^T                          TMEM S
+//                   dP^T = V dO^T                         TMEM dP
+//                   softmax warps, phase 1: P^T = exp(S^T - lse) -> TMEM S (bf16)      -> dV may start
+//                   dV  += P^T dO        (A from TMEM)    TMEM dV
+//                   softmax warps, phase 2: dS^T = P^T (dP^T - D) -> smem, into the dO tile's buffer once
+//                                                          dV has read it
+//                   dK  += dS^T Q        (A from smem)    TMEM dK
+//                   dQ^T = K^T dS^T      (M = d)          TMEM dP (free once dS^T is computed)
 //                 dQ^T is read by a second warpgroup (TMEM lane = head-dim index), scaled and added to an fp32
-//                 accumulator straight from registers: per row one coalesced 128-byte red.global.add per warp,
-//                 so dQ costs no shared-memory bandwidth (the MMAs' operand reads already nearly fill it). dK/dV stay in TMEM for the whole item; an unsplit key tile
-//                 writes them as bf16, a split one adds its fp32 partial into the workspace (one add per chunk).
+//                 accumulator from registers: per row one coalesced 128-byte red.global.add per warp. dK/dV stay
+//                 in TMEM for the whole item; an unsplit key tile writes them as bf16, a split one adds its fp32
+//                 partial into the workspace (one add per element and chunk).
 //   k_bwd_convert dQ (and the split tiles' dK/dV) from the fp32 accumulators to bf16.
-// TMEM (512 columns): S[0] [0,64), S[1] [64,128), dP[0] [128,192), dP[1] [192,256), dV [256,384), dK [384,512).
-// S/dP are double-buffered so the MMAs of step t+1 run while the softmax warps work on step t. dQ^T(t) lands in
-// dP[b]; the only MMA that must wait for the dQ warps to read it is dP^T(t+2), and S^T(t+2) is issued first.
-// The producer fetches each step's (lse * log2 e, D) pairs with one bulk copy: the preprocess kernel packs them
-// into the workspace with padding, so the copy can start at a 16-byte boundary below the tile's first row.
+// TMEM (512 columns): S/P [0,128), dP/dQ [128,256), dV [256,384), dK [384,512).
+// Q/dO tiles come through a 2-stage ring; each step's (lse, D) values come with them in one bulk copy of a padded
+// float4 table ((lse_i, D_i, lse_i+1, D_i+1) at index i) so any first row starts on a 16-byte boundary.
 // Work items run kv-head-major: concurrently running CTAs share a kv head, so a group's Q/dO rows and dQ
 // accumulator rows are reused from L2 across its key tiles.
 #pragma once
@@ -43,7 +44,7 @@ constexpr int BWD_D = 128;
 
 struct BwdWorkspace {
     int64_t rows_pad;   // T + padding rows so tiles that stick out past T stay inside the buffers
-    int64_t off_delta;  // float2 [hq][rows_pad]: (lse_i * log2 e, D_i = dO_i . O_i)
+    int64_t off_delta;  // float4 [hq][rows_pad]: (lse_i * log2 e, D_i, lse_{i+1} * log2 e, D_{i+1})
     int64_t off_dq;     // fp32 [hq][rows_pad][d]: dQ accumulator
     int64_t off_dk;     // fp32 [rows_pad][hkv][d]: dK accumulator of split key tiles
     int64_t off_dv;     // fp32 [rows_pad][hkv][d]: dV accumulator of split key tiles
@@ -54,7 +55,7 @@ inline BwdWorkspace bwd_workspace_layout(int64_t T, int hq, int hkv, int d) {
     BwdWorkspace w{};
     w.rows_pad = (T + 256 + 7) & ~int64_t(7);
     int64_t o = 0;
-    w.off_delta = o; o = align256(o + 8 * int64_t(hq) * w.rows_pad);
+    w.off_delta = o; o = align256(o + 16 * int64_t(hq) * w.rows_pad);
     w.off_dq = o;    o = align256(o + 4 * int64_t(hq) * w.rows_pad * d);
     w.off_dk = o;    o = align256(o + 4 * w.rows_pad * hkv * d);
     w.off_dv = o;    o = align256(o + 4 * w.rows_pad * hkv * d);
@@ -63,9 +64,10 @@ inline BwdWorkspace bwd_workspace_layout(int64_t T, int hq, int hkv, int d) {
 }
 
 // ------------------------------------------------------------------------------------------------- preprocess
-// One warp per (row, head): (lse * log2 e, D = sum_d dO * O) in fp32; padding rows get (0, 0).
+// One warp per (row, head): D = sum_d dO * O in fp32. Writes (lse * log2 e, D) into the .xy of entry i and the .zw
+// of entry i - 1 of the float4 table; padding rows get zeros.
 __global__ void k_bwd_pre(const __nv_bfloat16 *__restrict__ O, const __nv_bfloat16 *__restrict__ dO,
-                          const float *__restrict__ lse, float2 *__restrict__ ld, int64_t T, int64_t rows_pad,
+                          const float *__restrict__ lse, float4 *__restrict__ ld, int64_t T, int64_t rows_pad,
                           int hq) {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = int64_t(gridDim.x) * (blockDim.x >> 5);
@@ -85,30 +87,37 @@ __global__ void k_bwd_pre(const __nv_bfloat16 *__restrict__ O, const __nv_bfloat
         }
 #pragma unroll
         for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0)
-            ld[int64_t(h) * rows_pad + i] = make_float2(i < T ? lse[int64_t(h) * T + i] * 1.4426950408889634f : 0.f,
-                                                        acc);
+        if (lane == 0) {
+            const float l2 = i < T ? lse[int64_t(h) * T + i] * 1.4426950408889634f : 0.f;
+            float *row = reinterpret_cast<float *>(ld + int64_t(h) * rows_pad);
+            row[4 * i] = l2;
+            row[4 * i + 1] = acc;
+            if (i > 0) {
+                row[4 * (i - 1) + 2] = l2;
+                row[4 * (i - 1) + 3] = acc;
+            }
+            if (i == rows_pad - 1) {
+                row[4 * i + 2] = 0.f;
+                row[4 * i + 3] = 0.f;
+            }
+        }
     }
 }
 
 // ------------------------------------------------------------------------------------------------- main kernel
 struct BwdSmem {
-    static constexpr int KV_BYTES = 128 * BWD_D * 2;     // 128 key rows x d, bf16
-    static constexpr int KV_CHUNK = 128 * 64 * 2;        // one 64-column swizzled chunk of it
-    static constexpr int QT_BYTES = 64 * BWD_D * 2;      // 64 query rows x d
-    static constexpr int QT_CHUNK = 64 * 64 * 2;
-    static constexpr int DS_BYTES = 128 * 64 * 2;        // dS^T: 128 key rows x 64 queries, bf16
-    static constexpr int LD_PAIRS = 66;                  // 64 rows + 1 alignment slack, rounded to 16 bytes
-    static constexpr int QSTAGES = 3;                    // Q/dO ring depth: hides the L2 latency of a step's loads
-    alignas(1024) uint8_t k[KV_BYTES];
-    alignas(1024) uint8_t v[KV_BYTES];
-    alignas(1024) uint8_t q[QSTAGES][QT_BYTES];
-    alignas(1024) uint8_t dout[QSTAGES][QT_BYTES];
-    alignas(1024) uint8_t ds[2][DS_BYTES];
-    alignas(16) float2 ld[QSTAGES][LD_PAIRS];            // (lse * log2 e, D) of the step's rows, from 16-B boundary
+    static constexpr int TILE = 128 * BWD_D * 2;         // 128 rows x d, bf16 (K, V, Q, dO; dS^T has the same size)
+    static constexpr int CHUNK = 128 * 64 * 2;           // one 64-column 128-byte-swizzled chunk of such a tile
+    static constexpr int QSTAGES = 2;
+    static constexpr int LD_BYTES = BWD_BM * 16;         // the step's (lse, D) float4 entries
+    alignas(1024) uint8_t k[TILE];
+    alignas(1024) uint8_t v[TILE];
+    alignas(1024) uint8_t q[QSTAGES][TILE];
+    alignas(1024) uint8_t dout[QSTAGES][TILE];          // dO(t), then dS^T(t) once dV(t) has read dO(t)
+    alignas(16) float4 ld[QSTAGES][BWD_BM];
     uint64_t kv_full, kv_empty, dkv_full, dkv_free;
     uint64_t q_full[QSTAGES], q_empty[QSTAGES];
-    uint64_t sdp_full[2], ds_full[2], ds_free[2], dq_full[2], dq_free[2];
+    uint64_t s_full, dp_full, p_ready, dv_done, ds_ready, dq_full, dq_free;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -118,7 +127,7 @@ struct BwdItem {
     int qa, qb, split, kh;
 };
 
-__device__ __forceinline__ BwdItem bwd_decode(const void *meta, const MetaHeader &hd, int item, int hkv) {
+__device__ __forceinline__ BwdItem bwd_decode(const void *meta, const MetaHeader &hd, int item) {
     const BWork w = meta_ptr<BWork>(meta, hd.off_bw)[item % hd.n_bw];
     BwdItem it;
     it.kh = item / hd.n_bw;
@@ -129,9 +138,6 @@ __device__ __forceinline__ BwdItem bwd_decode(const void *meta, const MetaHeader
     return it;
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 __device__ __forceinline__ void red_add_f32(float *addr, float a) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
 }
@@ -139,11 +145,40 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
 }
+__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+// dK (scaled) or dV of the item from TMEM: bf16 rows for an unsplit tile, fp32 adds into the workspace otherwise.
+__device__ __forceinline__ void bwd_store_kv(uint32_t taddr, bool yin, bool split, float f, float *acc,
+                                             __nv_bfloat16 *dst, int64_t rowoff) {
+#pragma unroll
+    for (int c = 0; c < BWD_D / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(taddr + c * 32, rr);
+        tmem_wait_ld();
+        if (!yin) continue;
+        if (split) {
+            float *a = acc + rowoff + c * 32;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                red_add_v4(a + 4 * e, __uint_as_float(rr[4 * e]) * f, __uint_as_float(rr[4 * e + 1]) * f,
+                           __uint_as_float(rr[4 * e + 2]) * f, __uint_as_float(rr[4 * e + 3]) * f);
+        } else {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                pk[e] = pack_bf16x2(__uint_as_float(rr[2 * e]) * f, __uint_as_float(rr[2 * e + 1]) * f);
+            uint4 *o = reinterpret_cast<uint4 *>(dst + rowoff + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+    }
+}
 
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-         const void *__restrict__ meta, const float2 *__restrict__ ldg,
+         const void *__restrict__ meta, const float4 *__restrict__ ldg,
          float *__restrict__ dq_acc, float *__restrict__ dk_acc, float *__restrict__ dv_acc,
          __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV, int hq, int hkv, int64_t rows_pad,
          float scale, float sl2) {
@@ -151,7 +186,6 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     BwdSmem &sm = *reinterpret_cast<BwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const MetaHeader hd = *meta_ptr<MetaHeader>(meta, 0);
-    const int T = hd.T;
     const int r = hq / hkv;
     const int n_items = hd.n_bw * hkv;
     volatile int *abort_flag = &sm.abort_flag;
@@ -160,18 +194,18 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         mbar_init(&sm.kv_full, 1);
         mbar_init(&sm.kv_empty, 1);
         mbar_init(&sm.dkv_full, 1);
-        mbar_init(&sm.dkv_free, 128);
+        mbar_init(&sm.dkv_free, 256);
         for (int b = 0; b < BwdSmem::QSTAGES; ++b) {
             mbar_init(&sm.q_full[b], 1);
             mbar_init(&sm.q_empty[b], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm.sdp_full[b], 1);
-            mbar_init(&sm.ds_full[b], 128);
-            mbar_init(&sm.ds_free[b], 1);
-            mbar_init(&sm.dq_full[b], 1);
-            mbar_init(&sm.dq_free[b], 128);
-        }
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.dp_full, 1);
+        mbar_init(&sm.p_ready, 128);
+        mbar_init(&sm.dv_done, 1);
+        mbar_init(&sm.ds_ready, 128);
+        mbar_init(&sm.dq_full, 1);
+        mbar_init(&sm.dq_free, 128);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -198,97 +232,96 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         if (lane == 0) {
             uint32_t g = 0, it_n = 0;
             for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
-                const BwdItem w = bwd_decode(meta, hd, item, hkv);
+                const BwdItem w = bwd_decode(meta, hd, item);
                 if (!bwait(&sm.kv_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
-                mbar_arrive_expect_tx(&sm.kv_full, 2 * BwdSmem::KV_BYTES);
+                mbar_arrive_expect_tx(&sm.kv_full, 2 * BwdSmem::TILE);
                 for (int c = 0; c < BWD_D / 64; ++c) {
-                    tma_load_3d(sm.k + c * BwdSmem::KV_CHUNK, &tmK, c * 64, w.kh, w.t.row0, &sm.kv_full);
-                    tma_load_3d(sm.v + c * BwdSmem::KV_CHUNK, &tmV, c * 64, w.kh, w.t.row0, &sm.kv_full);
+                    tma_load_3d(sm.k + c * BwdSmem::CHUNK, &tmK, c * 64, w.kh, w.t.row0, &sm.kv_full);
+                    tma_load_3d(sm.v + c * BwdSmem::CHUNK, &tmV, c * 64, w.kh, w.t.row0, &sm.kv_full);
                 }
                 const int n = (w.qb - w.qa) * r;
                 for (int t = 0; t < n; ++t, ++g) {
-                    const int b = g % BwdSmem::QSTAGES;
+                    const int st = g % BwdSmem::QSTAGES;
                     const int h = w.kh * r + t % r;
                     const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
-                    if (!bwait(&sm.q_empty[b], ((g / BwdSmem::QSTAGES) & 1) ^ 1, abort_flag)) goto done;
-                    mbar_arrive_expect_tx(&sm.q_full[b], 2 * BwdSmem::QT_BYTES + BwdSmem::LD_PAIRS * 8);
+                    if (!bwait(&sm.q_empty[st], ((g / BwdSmem::QSTAGES) & 1) ^ 1, abort_flag)) goto done;
+                    mbar_arrive_expect_tx(&sm.q_full[st], 2 * BwdSmem::TILE + BwdSmem::LD_BYTES);
                     for (int c = 0; c < BWD_D / 64; ++c) {
-                        tma_load_3d(sm.q[b] + c * BwdSmem::QT_CHUNK, &tmQ, c * 64, h, x0, &sm.q_full[b]);
-                        tma_load_3d(sm.dout[b] + c * BwdSmem::QT_CHUNK, &tmdO, c * 64, h, x0, &sm.q_full[b]);
+                        tma_load_3d(sm.q[st] + c * BwdSmem::CHUNK, &tmQ, c * 64, h, x0, &sm.q_full[st]);
+                        tma_load_3d(sm.dout[st] + c * BwdSmem::CHUNK, &tmdO, c * 64, h, x0, &sm.q_full[st]);
                     }
-                    // (lse, D) pairs of rows [x0 & ~1, +66): a 16-byte aligned, padded slice of the workspace
-                    bulk_load(sm.ld[b], ldg + int64_t(h) * rows_pad + (x0 & ~1), BwdSmem::LD_PAIRS * 8,
-                              &sm.q_full[b]);
+                    bulk_load(sm.ld[st], ldg + int64_t(h) * rows_pad + x0, BwdSmem::LD_BYTES, &sm.q_full[st]);
                 }
             }
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------------ MMA issuer (one thread)
         if (lane == 0) {
-            constexpr uint32_t ID_SDP = idesc_bf16(128, BWD_BM, 0, 0);     // S^T, dP^T
-            constexpr uint32_t ID_KV = idesc_bf16(128, BWD_D, 0, 1);       // dV, dK (B MN-major)
+            constexpr uint32_t ID_SDP = idesc_bf16(128, BWD_BM, 0, 0);     // S^T, dP^T (both K-major)
+            constexpr uint32_t ID_DV = idesc_bf16(128, BWD_D, 0, 1);       // dV (A TMEM, B MN-major)
+            constexpr uint32_t ID_DK = idesc_bf16(128, BWD_D, 0, 1);       // dK (A K-major smem, B MN-major)
             constexpr uint32_t ID_DQ = idesc_bf16(128, BWD_BM, 1, 1);      // dQ^T (A and B MN-major)
             const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
             uint32_t g = 0, it_n = 0;
-            auto issue_s = [&](int b, int qs) {
-                const uint32_t sq = smem_u32(sm.q[qs]);
+            // K-major x K-major product over d (S^T = K Q^T or dP^T = V dO^T)
+            auto issue_kk = [&](uint32_t col, uint32_t a, uint32_t b) {
 #pragma unroll
                 for (int kk = 0; kk < BWD_D / 16; ++kk) {
-                    const uint32_t ok = (kk >> 2) * BwdSmem::KV_CHUNK + (kk & 3) * 32;
-                    const uint32_t oq = (kk >> 2) * BwdSmem::QT_CHUNK + (kk & 3) * 32;
-                    umma_ss(tmem + COL_S + b * 64, smem_desc(sk + ok, 16, 1024), smem_desc(sq + oq, 16, 1024),
-                            ID_SDP, kk > 0);
+                    const uint32_t off = (kk >> 2) * BwdSmem::CHUNK + (kk & 3) * 32;
+                    umma_ss(tmem + col, smem_desc(a + off, 16, 1024), smem_desc(b + off, 16, 1024), ID_SDP, kk > 0);
                 }
             };
-            auto issue_dp = [&](int b, int qs) {
-                const uint32_t sdo = smem_u32(sm.dout[qs]);
-#pragma unroll
-                for (int kk = 0; kk < BWD_D / 16; ++kk) {
-                    const uint32_t ok = (kk >> 2) * BwdSmem::KV_CHUNK + (kk & 3) * 32;
-                    const uint32_t oq = (kk >> 2) * BwdSmem::QT_CHUNK + (kk & 3) * 32;
-                    umma_ss(tmem + COL_DP + b * 64, smem_desc(sv + ok, 16, 1024), smem_desc(sdo + oq, 16, 1024),
-                            ID_SDP, kk > 0);
-                }
+            auto issue_dp = [&](uint32_t gg) -> bool {      // dP^T(gg), once dQ^T(gg - 1) has been read out
+                if (gg > 0 && !bwait(&sm.dq_free, (gg - 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                issue_kk(COL_DP, sv, smem_u32(sm.dout[gg % BwdSmem::QSTAGES]));
+                umma_commit(&sm.dp_full);
+                return true;
             };
-            // S^T/dP^T of step g1 into buffers g1 & 1: S at once, dP once the dQ warps have read dQ^T(g1 - 2)
-            auto issue_sdp = [&](uint32_t g1) -> bool {
-                const int b = g1 & 1, qs = g1 % BwdSmem::QSTAGES;
-                if (!bwait(&sm.q_full[qs], (g1 / BwdSmem::QSTAGES) & 1, abort_flag)) return false;
+            auto issue_s = [&](uint32_t gg) -> bool {       // S^T(gg), once its Q tile has landed
+                const int st = gg % BwdSmem::QSTAGES;
+                if (!bwait(&sm.q_full[st], (gg / BwdSmem::QSTAGES) & 1, abort_flag)) return false;
                 tc_fence_after();
-                issue_s(b, qs);
-                if (!bwait(&sm.dq_free[b], ((g1 >> 1) & 1) ^ 1, abort_flag)) return false;
-                tc_fence_after();
-                issue_dp(b, qs);
-                umma_commit(&sm.sdp_full[b]);
+                issue_kk(COL_S, sk, smem_u32(sm.q[st]));
+                umma_commit(&sm.s_full);
                 return true;
             };
             for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
-                const BwdItem w = bwd_decode(meta, hd, item, hkv);
+                const BwdItem w = bwd_decode(meta, hd, item);
                 const int n = (w.qb - w.qa) * r;
                 if (!bwait(&sm.kv_full, it_n & 1, abort_flag)) goto done;
-                if (!issue_sdp(g)) goto done;
+                if (!issue_s(g)) goto done;
+                if (!issue_dp(g)) goto done;
                 if (!bwait(&sm.dkv_free, (it_n & 1) ^ 1, abort_flag)) goto done;
                 for (int t = 0; t < n; ++t, ++g) {
-                    const int b = g & 1, qs = g % BwdSmem::QSTAGES;
-                    if (t + 1 < n && !issue_sdp(g + 1)) goto done;
-                    if (!bwait(&sm.ds_full[b], (g >> 1) & 1, abort_flag)) goto done;
+                    const int st = g % BwdSmem::QSTAGES;
+                    const uint32_t sq = smem_u32(sm.q[st]), sdo = smem_u32(sm.dout[st]);
+                    // dV += P^T dO, as soon as the softmax warps have written P^T
+                    if (!bwait(&sm.p_ready, g & 1, abort_flag)) goto done;
                     tc_fence_after();
-                    const uint32_t sq = smem_u32(sm.q[qs]), sdo = smem_u32(sm.dout[qs]), sds = smem_u32(sm.ds[b]);
 #pragma unroll
-                    for (int kk = 0; kk < BWD_BM / 16; ++kk)       // dV += P^T dO
-                        umma_ts(tmem + COL_DV, tmem + COL_S + b * 64 + kk * 8,
-                                smem_desc(sdo + kk * 2048, BwdSmem::QT_CHUNK, 1024), ID_KV, (t > 0 || kk > 0));
+                    for (int kk = 0; kk < BWD_BM / 16; ++kk)
+                        umma_ts(tmem + COL_DV, tmem + COL_S + kk * 8, smem_desc(sdo + kk * 2048, BwdSmem::CHUNK, 1024),
+                                ID_DV, (t > 0 || kk > 0));
+                    umma_commit(&sm.dv_done);
+                    // S^T of the next step may overwrite P^T now (MMAs run in issue order)
+                    if (t + 1 < n && !issue_s(g + 1)) goto done;
+                    // dK += dS^T Q and dQ^T = K^T dS^T once dS^T is in shared memory
+                    if (!bwait(&sm.ds_ready, g & 1, abort_flag)) goto done;
+                    tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < BWD_BM / 16; ++kk)       // dK += dS^T Q
-                        umma_ts(tmem + COL_DK, tmem + COL_DP + b * 64 + kk * 8,
-                                smem_desc(sq + kk * 2048, BwdSmem::QT_CHUNK, 1024), ID_KV, (t > 0 || kk > 0));
-                    umma_commit(&sm.q_empty[qs]);
+                    for (int kk = 0; kk < BWD_BM / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * BwdSmem::CHUNK + (kk & 3) * 32;
+                        umma_ss(tmem + COL_DK, smem_desc(sdo + off, 16, 1024),
+                                smem_desc(sq + kk * 2048, BwdSmem::CHUNK, 1024), ID_DK, (t > 0 || kk > 0));
+                    }
 #pragma unroll
-                    for (int kk = 0; kk < 128 / 16; ++kk)          // dQ^T = K^T dS^T, into dP[b]
-                        umma_ss(tmem + COL_DP + b * 64, smem_desc(sk + kk * 2048, BwdSmem::KV_CHUNK, 1024),
-                                smem_desc(sds + kk * 2048, BwdSmem::DS_BYTES, 1024), ID_DQ, kk > 0);
-                    umma_commit(&sm.dq_full[b]);
-                    umma_commit(&sm.ds_free[b]);
+                    for (int kk = 0; kk < 128 / 16; ++kk)
+                        umma_ss(tmem + COL_DP, smem_desc(sk + kk * 2048, BwdSmem::CHUNK, 1024),
+                                smem_desc(sdo + kk * 2048, BwdSmem::CHUNK, 1024), ID_DQ, kk > 0);
+                    umma_commit(&sm.dq_full);
+                    umma_commit(&sm.q_empty[st]);
+                    if (t + 1 < n && !issue_dp(g + 1)) goto done;
                 }
                 umma_commit(&sm.dkv_full);
                 umma_commit(&sm.kv_empty);
@@ -301,125 +334,120 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         uint32_t g = 0, it_n = 0;
         const int32_t *key_end = meta_ptr<int32_t>(meta, hd.off_key_end);
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
-            const BwdItem w = bwd_decode(meta, hd, item, hkv);
+            const BwdItem w = bwd_decode(meta, hd, item);
             const int n = (w.qb - w.qa) * r;
             const int y = w.t.row0 + jr;
             const int gend = w.t.gstart + w.t.glen;
             const bool yin = y < gend;
             const int ke = yin ? key_end[y] : y;                       // queries [y, ke) attend key y
             for (int t = 0; t < n; ++t, ++g) {
-                const int b = g & 1, qs = g % BwdSmem::QSTAGES;
+                const int st = g % BwdSmem::QSTAGES;
                 const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
-                const float2 *ldp = sm.ld[qs] + (x0 & 1);
-                if (!bwait(&sm.ds_free[b], ((g >> 1) & 1) ^ 1, abort_flag)) goto done;
-                if (!bwait(&sm.sdp_full[b], (g >> 1) & 1, abort_flag)) goto done;
-                if (!bwait(&sm.q_full[qs], (g / BwdSmem::QSTAGES) & 1, abort_flag)) goto done;
-                tc_fence_after();
+                const float4 *ldp = sm.ld[st];
                 const int lo = y - x0, hi = ke - x0;                   // allowed query columns [lo, hi)
-                uint8_t *dsrow = sm.ds[b] + jr * 128;
+                // phase 1: P^T = exp2(S^T * scale * log2 e - lse * log2 e), kept packed for phase 2
+                if (!bwait(&sm.s_full, g & 1, abort_flag)) goto done;
+                if (!bwait(&sm.q_full[st], (g / BwdSmem::QSTAGES) & 1, abort_flag)) goto done;
+                tc_fence_after();
+                uint32_t pk[64];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t sr[32], pr[32];
-                    tmem_ld32(tmem + lane_off + COL_S + b * 64 + half * 32, sr);
-                    tmem_ld32(tmem + lane_off + COL_DP + b * 64 + half * 32, pr);
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t sr[32];
+                    tmem_ld32(tmem + lane_off + COL_S + c * 32, sr);
                     tmem_wait_ld();
-                    uint32_t pp[16], dd[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        float p2[2], d2[2];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int cl = 2 * e + u, c = half * 32 + cl;
-                            const float2 l2 = ldp[c];
-                            const bool ok = c >= lo && c < hi;
-                            const float p = ok ? ex2_approx(fmaf(__uint_as_float(sr[cl]), sl2, -l2.x)) : 0.f;
-                            p2[u] = p;
-                            d2[u] = p * (__uint_as_float(pr[cl]) - l2.y);
-                        }
-                        pp[e] = pack_bf16x2(p2[0], p2[1]);
-                        dd[e] = pack_bf16x2(d2[0], d2[1]);
+                        const int col = 32 * c + 2 * e;
+                        const float4 l = ldp[col];
+                        const float p0 = (col >= lo && col < hi) ? ex2_approx(fmaf(__uint_as_float(sr[2 * e]), sl2, -l.x)) : 0.f;
+                        const float p1 = (col + 1 >= lo && col + 1 < hi) ? ex2_approx(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, -l.z)) : 0.f;
+                        pk[16 * c + e] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st16(tmem + lane_off + COL_S + b * 64 + half * 16, pp);
-                    tmem_st16(tmem + lane_off + COL_DP + b * 64 + half * 16, dd);
-                    // dS^T row jr, queries [32 half, +32), into the 128-byte-swizzled [key][query] tile
+                    uint32_t tmp[16];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int ch = half * 4 + c;
-                        *reinterpret_cast<uint4 *>(dsrow + ((ch ^ (jr & 7)) << 4)) =
-                            make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
-                    }
+                    for (int e = 0; e < 16; ++e) tmp[e] = pk[16 * c + e];
+                    tmem_st16(tmem + lane_off + COL_S + c * 16, tmp);  // P^T cols [16c, 16c+16): S chunks <= c
                 }
                 tmem_wait_st();
-                fence_proxy_async_smem();
                 tc_fence_before();
-                mbar_arrive(&sm.ds_full[b]);
-            }
-            // item epilogue: dK (scaled) and dV from TMEM
-            if (!bwait(&sm.dkv_full, it_n & 1, abort_flag)) goto done;
-            tc_fence_after();
-            for (int which = 0; which < 2; ++which) {
-                const uint32_t col = which == 0 ? COL_DK : COL_DV;
-                const float f = which == 0 ? scale : 1.f;
-                float *acc = which == 0 ? dk_acc : dv_acc;
-                __nv_bfloat16 *dst = which == 0 ? dK : dV;
+                mbar_arrive(&sm.p_ready);
+                // phase 2: dS^T = P^T (dP^T - D) into the dO buffer, which dV has finished reading
+                if (!bwait(&sm.dp_full, g & 1, abort_flag)) goto done;
+                if (!bwait(&sm.dv_done, g & 1, abort_flag)) goto done;
+                tc_fence_after();
+                uint8_t *dsrow = sm.dout[st] + jr * 128;
 #pragma unroll
-                for (int c = 0; c < BWD_D / 32; ++c) {
-                    uint32_t rr[32];
-                    tmem_ld32(tmem + lane_off + col + c * 32, rr);
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pr[32];
+                    tmem_ld32(tmem + lane_off + COL_DP + c * 32, pr);
                     tmem_wait_ld();
-                    if (!yin) continue;
-                    if (w.split) {
-                        float *a = acc + (int64_t(y) * hkv + w.kh) * BWD_D + c * 32;
+                    uint32_t dd[16];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            red_add_v4(a + 4 * e, __uint_as_float(rr[4 * e]) * f, __uint_as_float(rr[4 * e + 1]) * f,
-                                       __uint_as_float(rr[4 * e + 2]) * f, __uint_as_float(rr[4 * e + 3]) * f);
-                    } else {
-                        uint32_t pk[16];
+                    for (int e = 0; e < 16; ++e) {
+                        const int col = 32 * c + 2 * e;
+                        const float4 l = ldp[col];
+                        const uint32_t p = pk[16 * c + e];
+                        dd[e] = pack_bf16x2(bf16lo(p) * (__uint_as_float(pr[2 * e]) - l.y),
+                                            bf16hi(p) * (__uint_as_float(pr[2 * e + 1]) - l.w));
+                    }
+                    // queries [32c, 32c+32): 64-column chunk c/2, 16-byte pieces 4(c%2)..4(c%2)+3, swizzled by row
 #pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            pk[e] = pack_bf16x2(__uint_as_float(rr[2 * e]) * f, __uint_as_float(rr[2 * e + 1]) * f);
-                        uint4 *o = reinterpret_cast<uint4 *>(dst + (int64_t(y) * hkv + w.kh) * BWD_D + c * 32);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) o[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    for (int u = 0; u < 4; ++u) {
+                        const int piece = 4 * (c & 1) + u;
+                        *reinterpret_cast<uint4 *>(dsrow + (c >> 1) * BwdSmem::CHUNK + ((piece ^ (jr & 7)) << 4)) =
+                            make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
                     }
                 }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&sm.ds_ready);
             }
+            // item epilogue: dK (scaled); the dQ warpgroup writes dV
+            if (!bwait(&sm.dkv_full, it_n & 1, abort_flag)) goto done;
+            tc_fence_after();
+            bwd_store_kv(tmem + lane_off + COL_DK, yin, w.split, scale, dk_acc, dK, (int64_t(y) * hkv + w.kh) * BWD_D);
             tc_fence_before();
             mbar_arrive(&sm.dkv_free);
         }
     } else {
         // ------------------------------------------------------------------ dQ warpgroup (warps 4-7)
-        const int dcol = (warp - 4) * 32 + lane;                       // head-dim index = TMEM lane
-        const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
-        uint32_t g = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-            const BwdItem w = bwd_decode(meta, hd, item, hkv);
+        const int wq = warp - 4;
+        const int dcol = wq * 32 + lane;                               // head-dim index = TMEM lane
+        const uint32_t lane_off = uint32_t(wq * 32) << 16;
+        uint32_t g = 0, it_n = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+            const BwdItem w = bwd_decode(meta, hd, item);
             const int n = (w.qb - w.qa) * r;
             for (int t = 0; t < n; ++t, ++g) {
-                const int b = g & 1;
                 const int h = w.kh * r + t % r;
                 const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
-                if (!bwait(&sm.dq_full[b], (g >> 1) & 1, abort_flag)) goto done;
+                if (!bwait(&sm.dq_full, g & 1, abort_flag)) goto done;
                 tc_fence_after();
-                uint32_t v[64];
-                {
+                uint32_t v[128];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
                     uint32_t tmp[32];
-                    tmem_ld32(tmem + lane_off + COL_DP + b * 64, tmp);
+                    tmem_ld32(tmem + lane_off + COL_DP + c * 32, tmp);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = tmp[e];
-                    tmem_ld32(tmem + lane_off + COL_DP + b * 64 + 32, tmp);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[32 + e] = tmp[e];
-                    tmem_wait_ld();
+                    for (int e = 0; e < 32; ++e) v[32 * c + e] = tmp[e];
                 }
+                tmem_wait_ld();
                 tc_fence_before();
-                mbar_arrive(&sm.dq_free[b]);
-                // dQ rows x0..x0+63, column dcol: one coalesced 128-byte add per warp and row
+                mbar_arrive(&sm.dq_free);
+                // dQ rows x0..x0+127, column dcol: one coalesced 128-byte add per warp and row
                 float *gdst = dq_acc + (int64_t(h) * rows_pad + x0) * BWD_D + dcol;
 #pragma unroll
-                for (int c = 0; c < 64; ++c) red_add_f32(gdst + c * BWD_D, __uint_as_float(v[c]) * scale);
+                for (int c = 0; c < BWD_BM; ++c) red_add_f32(gdst + c * BWD_D, __uint_as_float(v[c]) * scale);
             }
+            // item epilogue: dV rows (TMEM lane = key row for this read)
+            const int jr = wq * 32 + lane;
+            const int y = w.t.row0 + jr;
+            const bool yin = y < w.t.gstart + w.t.glen;
+            if (!bwait(&sm.dkv_full, it_n & 1, abort_flag)) goto done;
+            tc_fence_after();
+            bwd_store_kv(tmem + lane_off + COL_DV, yin, w.split, 1.f, dv_acc, dV, (int64_t(y) * hkv + w.kh) * BWD_D);
+            tc_fence_before();
+            mbar_arrive(&sm.dkv_free);
         }
     }
 done:
@@ -484,7 +512,7 @@ inline pp_status launch_bwd(const void *q, const void *k, const void *v, const v
     if (d != BWD_D) return fail(PP_ERR_UNSUPPORTED, "backward supports head dim 128 only (got %d)", d);
     const BwdWorkspace L = bwd_workspace_layout(T, hq, hkv, d);
     char *ws = static_cast<char *>(workspace);
-    float2 *ldg = reinterpret_cast<float2 *>(ws + L.off_delta);
+    float4 *ldg = reinterpret_cast<float4 *>(ws + L.off_delta);
     float *dq_acc = reinterpret_cast<float *>(ws + L.off_dq);
     float *dk_acc = reinterpret_cast<float *>(ws + L.off_dk);
     float *dv_acc = reinterpret_cast<float *>(ws + L.off_dv);

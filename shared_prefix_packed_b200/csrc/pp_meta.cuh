@@ -16,9 +16,9 @@ namespace pp {
 constexpr int FWD_BM = 128;
 constexpr int FWD_BN = 128;
 constexpr int BWD_BN = 128;   // key rows per backward tile (the MMA M dimension)
-constexpr int BWD_BM = 64;    // query rows per backward step (the MMA N dimension)
+constexpr int BWD_BM = 128;   // query rows per backward step (the MMA N dimension)
 constexpr int BWD_MAX_CHUNKS = 16;
-constexpr int BWD_CHUNK_QTILES = 16;   // target query tiles per backward work chunk (before the cap)
+constexpr int BWD_CHUNK_QTILES = 8;    // target query tiles per backward work chunk (before the cap)
 constexpr int SORT_BINS = 4096;
 constexpr int32_t META_MAGIC = 0x314d5050;  // "PPM1"
 

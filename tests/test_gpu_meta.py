@@ -33,7 +33,7 @@ def test_meta_small_cases(P, S):
     assert np.array_equal(b.pos_ids[: b.T].cpu().numpy(), oracle.position_ids(P, S))
     from shared_prefix_packed_b200 import PP_PASS_BWD, PP_PASS_FWD, pp_get_status
     assert b.tiles(PP_PASS_FWD) == oracle.tile_classes(P, S, 128, 128)
-    assert b.tiles(PP_PASS_BWD) == oracle.tile_classes(P, S, 64, 128)
+    assert b.tiles(PP_PASS_BWD) == oracle.tile_classes(P, S, 128, 128)
     pp_get_status()
 
 
@@ -44,7 +44,7 @@ def test_meta_random_groups(seed):
     from shared_prefix_packed_b200 import PP_PASS_BWD, PP_PASS_FWD
     assert np.array_equal(b.pos_ids[: b.T].cpu().numpy(), oracle.position_ids(P, S))
     assert b.tiles(PP_PASS_FWD) == oracle.tile_classes(P, S, 128, 128)
-    assert b.tiles(PP_PASS_BWD) == oracle.tile_classes(P, S, 64, 128)
+    assert b.tiles(PP_PASS_BWD) == oracle.tile_classes(P, S, 128, 128)
 
 
 @pytest.mark.parametrize("name", ["tiny", "dpo", "grpo", "longprefix", "hetero"])
@@ -55,7 +55,7 @@ def test_meta_full_workloads(name):
     from shared_prefix_packed_b200 import PP_PASS_BWD, PP_PASS_FWD
     assert np.array_equal(b.pos_ids[: b.T].cpu().numpy(), oracle.position_ids(P, S))
     assert b.tiles(PP_PASS_FWD) == oracle.tile_classes(P, S, 128, 128)
-    assert b.tiles(PP_PASS_BWD) == oracle.tile_classes(P, S, 64, 128)
+    assert b.tiles(PP_PASS_BWD) == oracle.tile_classes(P, S, 128, 128)
 
 
 def test_schedule_invariants():
