@@ -16,18 +16,25 @@
 //                   dP^T = V dO^T                         TMEM dP
 //                   softmax warps, phase 1: P^T = exp(S^T - lse) -> TMEM S (bf16)      -> dV may start
 //                   dV  += P^T dO        (A from TMEM)    TMEM dV
-//                   softmax warps, phase 2: dS^T = P^T (dP^T - D) -> smem, into the dO tile's buffer once
-//                                                          dV has read it
-//                   dK  += dS^T Q        (A from smem)    TMEM dK
-//                   dQ^T = K^T dS^T      (M = d)          TMEM dP (free once dS^T is computed)
+//                   softmax warps, phase 2: dS^T = scale P^T (dP^T - D) -> TMEM dP (bf16) and smem, into the
+//                                                          dO tile's buffer once dV has read it
+//                   dK  += dS^T Q        (A from TMEM)    TMEM dK
+//                   dQ^T = K^T dS^T      (M = d)          TMEM dP (dK has read dS^T: MMAs run in issue order)
 //                 dQ^T is read by a second warpgroup (TMEM lane = head-dim index), scaled and added to an fp32
 //                 accumulator from registers: per row one coalesced 128-byte red.global.add per warp. dK/dV stay
 //                 in TMEM for the whole item; an unsplit key tile writes them as bf16, a split one adds its fp32
 //                 partial into the workspace (one add per element and chunk).
 //   k_bwd_convert dQ (and the split tiles' dK/dV) from the fp32 accumulators to bf16.
-// TMEM (512 columns): S/P [0,128), dP/dQ [128,256), dV [256,384), dK [384,512).
-// Q/dO tiles come through a 2-stage ring; each step's (lse, D) values come with them in one bulk copy of a padded
-// float4 table ((lse_i, D_i, lse_i+1, D_i+1) at index i) so any first row starts on a 16-byte boundary.
+// TMEM (512 columns): S/P [0,128), dP/dS/dQ [128,256), dV [256,384), dK [384,512).
+// Per-query values folded into the MMAs: the softmax warps own a key row each and would otherwise need the lse
+// and D of all 128 query columns per step (a shared-memory or shuffle broadcast per element, which measured
+// several times slower than the exp itself). Instead one extra K = 16 slice is appended to the S^T and dP^T
+// products: K and V get columns (1, 1, 1, 0, ...), Q gets (-lse/scale) and dO gets (-D), each split exactly into
+// three bf16 parts (hi, mid, lo). The accumulators then hold s - lse/scale and dP - D directly, so
+// P^T = exp2(S'^T * scale * log2 e) and dS^T = P^T * dP'^T * scale need nothing but the TMEM values. The extra
+// slices cost 2 of 42 MMAs per step. They live in shared memory as 128 x 16 bf16 tiles in the no-swizzle core-matrix
+// layout; the producer warp writes the query side for each step.
+// Q/dO tiles come through a 2-stage ring.
 // Work items run kv-head-major: concurrently running CTAs share a kv head, so a group's Q/dO rows and dQ
 // accumulator rows are reused from L2 across its key tiles.
 #pragma once
@@ -44,7 +51,7 @@ constexpr int BWD_D = 128;
 
 struct BwdWorkspace {
     int64_t rows_pad;   // T + padding rows so tiles that stick out past T stay inside the buffers
-    int64_t off_delta;  // float4 [hq][rows_pad]: (lse_i * log2 e, D_i, lse_{i+1} * log2 e, D_{i+1})
+    int64_t off_delta;  // float2 [hq][rows_pad]: (-lse_i / scale, -D_i)
     int64_t off_dq;     // fp32 [hq][rows_pad][d]: dQ accumulator
     int64_t off_dk;     // fp32 [rows_pad][hkv][d]: dK accumulator of split key tiles
     int64_t off_dv;     // fp32 [rows_pad][hkv][d]: dV accumulator of split key tiles
@@ -55,7 +62,7 @@ inline BwdWorkspace bwd_workspace_layout(int64_t T, int hq, int hkv, int d) {
     BwdWorkspace w{};
     w.rows_pad = (T + 256 + 7) & ~int64_t(7);
     int64_t o = 0;
-    w.off_delta = o; o = align256(o + 16 * int64_t(hq) * w.rows_pad);
+    w.off_delta = o; o = align256(o + 8 * int64_t(hq) * w.rows_pad);
     w.off_dq = o;    o = align256(o + 4 * int64_t(hq) * w.rows_pad * d);
     w.off_dk = o;    o = align256(o + 4 * w.rows_pad * hkv * d);
     w.off_dv = o;    o = align256(o + 4 * w.rows_pad * hkv * d);
@@ -64,11 +71,11 @@ inline BwdWorkspace bwd_workspace_layout(int64_t T, int hq, int hkv, int d) {
 }
 
 // ------------------------------------------------------------------------------------------------- preprocess
-// One warp per (row, head): D = sum_d dO * O in fp32. Writes (lse * log2 e, D) into the .xy of entry i and the .zw
-// of entry i - 1 of the float4 table; padding rows get zeros.
+// One warp per (row, head): D = sum_d dO * O in fp32, stored with the lse as (-lse / scale, -D), the values the
+// query side of the extra MMA slice carries; padding rows get zeros.
 __global__ void k_bwd_pre(const __nv_bfloat16 *__restrict__ O, const __nv_bfloat16 *__restrict__ dO,
-                          const float *__restrict__ lse, float4 *__restrict__ ld, int64_t T, int64_t rows_pad,
-                          int hq) {
+                          const float *__restrict__ lse, float2 *__restrict__ ld, int64_t T, int64_t rows_pad,
+                          int hq, float inv_scale) {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = int64_t(gridDim.x) * (blockDim.x >> 5);
     for (int64_t w = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < rows_pad * hq; w += nwarps) {
@@ -87,21 +94,19 @@ __global__ void k_bwd_pre(const __nv_bfloat16 *__restrict__ O, const __nv_bfloat
         }
 #pragma unroll
         for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) {
-            const float l2 = i < T ? lse[int64_t(h) * T + i] * 1.4426950408889634f : 0.f;
-            float *row = reinterpret_cast<float *>(ld + int64_t(h) * rows_pad);
-            row[4 * i] = l2;
-            row[4 * i + 1] = acc;
-            if (i > 0) {
-                row[4 * (i - 1) + 2] = l2;
-                row[4 * (i - 1) + 3] = acc;
-            }
-            if (i == rows_pad - 1) {
-                row[4 * i + 2] = 0.f;
-                row[4 * i + 3] = 0.f;
-            }
-        }
+        if (lane == 0)
+            ld[int64_t(h) * rows_pad + i] = make_float2(i < T ? -lse[int64_t(h) * T + i] * inv_scale : 0.f, -acc);
     }
+}
+
+// Split x into three bf16 parts whose sum is x to about 2^-24 relative: the packed (hi, mid) and (lo, 0) words.
+__device__ __forceinline__ uint2 split3_bf16(float x) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 l = __float2bfloat16_rn(r1 - __bfloat162float(m));
+    return make_uint2(uint32_t(__bfloat16_as_ushort(h)) | (uint32_t(__bfloat16_as_ushort(m)) << 16),
+                      uint32_t(__bfloat16_as_ushort(l)));
 }
 
 // ------------------------------------------------------------------------------------------------- main kernel
@@ -109,12 +114,15 @@ struct BwdSmem {
     static constexpr int TILE = 128 * BWD_D * 2;         // 128 rows x d, bf16 (K, V, Q, dO; dS^T has the same size)
     static constexpr int CHUNK = 128 * 64 * 2;           // one 64-column 128-byte-swizzled chunk of such a tile
     static constexpr int QSTAGES = 2;
-    static constexpr int LD_BYTES = BWD_BM * 16;         // the step's (lse, D) float4 entries
+    static constexpr int AUG = 128 * 16 * 2;             // 128 rows x 16 bf16, no-swizzle core-matrix layout
+    static constexpr int AUG_LBO = 128, AUG_SBO = 256;   // next 8 columns / next 8 rows
     alignas(1024) uint8_t k[TILE];
     alignas(1024) uint8_t v[TILE];
     alignas(1024) uint8_t q[QSTAGES][TILE];
     alignas(1024) uint8_t dout[QSTAGES][TILE];          // dO(t), then dS^T(t) once dV(t) has read dO(t)
-    alignas(16) float4 ld[QSTAGES][BWD_BM];
+    alignas(1024) uint8_t aug_ones[AUG];                 // key side of the extra slice: (1, 1, 1, 0, ...)
+    alignas(1024) uint8_t aug_q[QSTAGES][AUG];           // query side for S^T: split(-lse / scale)
+    alignas(1024) uint8_t aug_do[QSTAGES][AUG];          // query side for dP^T: split(-D)
     uint64_t kv_full, kv_empty, dkv_full, dkv_free;
     uint64_t q_full[QSTAGES], q_empty[QSTAGES];
     uint64_t s_full, dp_full, p_ready, dv_done, ds_ready, dq_full, dq_free;
@@ -137,6 +145,9 @@ __device__ __forceinline__ BwdItem bwd_decode(const void *meta, const MetaHeader
     it.split = w.split;
     return it;
 }
+
+// Byte offset of row r, column 0 in a 128 x 16 bf16 no-swizzle K-major tile (8-row x 16-byte core matrices).
+__device__ __forceinline__ uint32_t aug_row_off(int r) { return (r >> 3) * 256 + (r & 7) * 16; }
 
 __device__ __forceinline__ void red_add_f32(float *addr, float a) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
@@ -178,7 +189,7 @@ __device__ __forceinline__ void bwd_store_kv(uint32_t taddr, bool yin, bool spli
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-         const void *__restrict__ meta, const float4 *__restrict__ ldg,
+         const void *__restrict__ meta, const float2 *__restrict__ ldg,
          float *__restrict__ dq_acc, float *__restrict__ dk_acc, float *__restrict__ dv_acc,
          __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV, int hq, int hkv, int64_t rows_pad,
          float scale, float sl2) {
@@ -196,7 +207,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         mbar_init(&sm.dkv_full, 1);
         mbar_init(&sm.dkv_free, 256);
         for (int b = 0; b < BwdSmem::QSTAGES; ++b) {
-            mbar_init(&sm.q_full[b], 1);
+            mbar_init(&sm.q_full[b], 32);
             mbar_init(&sm.q_empty[b], 1);
         }
         mbar_init(&sm.s_full, 1);
@@ -208,6 +219,18 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         mbar_init(&sm.dq_free, 128);
         sm.abort_flag = 0;
         fence_mbar_init();
+    }
+    {   // extra-slice tiles: zeros everywhere, ones in columns 0-2 of the key-side tile
+        uint4 *z = reinterpret_cast<uint4 *>(sm.aug_ones);
+        for (int i = threadIdx.x; i < (1 + 2 * BwdSmem::QSTAGES) * BwdSmem::AUG / 16; i += blockDim.x)
+            z[i] = make_uint4(0, 0, 0, 0);
+        __syncthreads();
+        if (threadIdx.x < 128) {
+            const uint32_t one = 0x3f80u;                          // bf16 1.0
+            *reinterpret_cast<uint2 *>(sm.aug_ones + aug_row_off(threadIdx.x)) =
+                make_uint2(one | (one << 16), one);
+        }
+        fence_proxy_async_smem();
     }
     if (warp == 9) {
         tmem_alloc(&sm.tmem_base, 512);
@@ -228,29 +251,42 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     if (hd.dev_err != 0) {
         // nothing to do: the metadata builder rejected its input
     } else if (warp == 8) {
-        // ------------------------------------------------------------------ producer (one thread)
-        if (lane == 0) {
-            uint32_t g = 0, it_n = 0;
-            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
-                const BwdItem w = bwd_decode(meta, hd, item);
+        // ------------------------------------------------------------------ producer warp
+        uint32_t g = 0, it_n = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+            const BwdItem w = bwd_decode(meta, hd, item);
+            if (lane == 0) {
                 if (!bwait(&sm.kv_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
                 mbar_arrive_expect_tx(&sm.kv_full, 2 * BwdSmem::TILE);
                 for (int c = 0; c < BWD_D / 64; ++c) {
                     tma_load_3d(sm.k + c * BwdSmem::CHUNK, &tmK, c * 64, w.kh, w.t.row0, &sm.kv_full);
                     tma_load_3d(sm.v + c * BwdSmem::CHUNK, &tmV, c * 64, w.kh, w.t.row0, &sm.kv_full);
                 }
-                const int n = (w.qb - w.qa) * r;
-                for (int t = 0; t < n; ++t, ++g) {
-                    const int st = g % BwdSmem::QSTAGES;
-                    const int h = w.kh * r + t % r;
-                    const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
-                    if (!bwait(&sm.q_empty[st], ((g / BwdSmem::QSTAGES) & 1) ^ 1, abort_flag)) goto done;
-                    mbar_arrive_expect_tx(&sm.q_full[st], 2 * BwdSmem::TILE + BwdSmem::LD_BYTES);
+            }
+            const int n = (w.qb - w.qa) * r;
+            for (int t = 0; t < n; ++t, ++g) {
+                const int st = g % BwdSmem::QSTAGES;
+                const int h = w.kh * r + t % r;
+                const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
+                float2 lv[4];                                          // rows lane + 32u of the step
+#pragma unroll
+                for (int u = 0; u < 4; ++u) lv[u] = ldg[int64_t(h) * rows_pad + x0 + lane + 32 * u];
+                if (!bwait(&sm.q_empty[st], ((g / BwdSmem::QSTAGES) & 1) ^ 1, abort_flag)) goto done;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t off = aug_row_off(lane + 32 * u);
+                    *reinterpret_cast<uint2 *>(sm.aug_q[st] + off) = split3_bf16(lv[u].x);
+                    *reinterpret_cast<uint2 *>(sm.aug_do[st] + off) = split3_bf16(lv[u].y);
+                }
+                fence_proxy_async_smem();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sm.q_full[st], 2 * BwdSmem::TILE);
                     for (int c = 0; c < BWD_D / 64; ++c) {
                         tma_load_3d(sm.q[st] + c * BwdSmem::CHUNK, &tmQ, c * 64, h, x0, &sm.q_full[st]);
                         tma_load_3d(sm.dout[st] + c * BwdSmem::CHUNK, &tmdO, c * 64, h, x0, &sm.q_full[st]);
                     }
-                    bulk_load(sm.ld[st], ldg + int64_t(h) * rows_pad + x0, BwdSmem::LD_BYTES, &sm.q_full[st]);
+                } else {
+                    mbar_arrive(&sm.q_full[st]);
                 }
             }
         }
@@ -259,22 +295,26 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         if (lane == 0) {
             constexpr uint32_t ID_SDP = idesc_bf16(128, BWD_BM, 0, 0);     // S^T, dP^T (both K-major)
             constexpr uint32_t ID_DV = idesc_bf16(128, BWD_D, 0, 1);       // dV (A TMEM, B MN-major)
-            constexpr uint32_t ID_DK = idesc_bf16(128, BWD_D, 0, 1);       // dK (A K-major smem, B MN-major)
+            constexpr uint32_t ID_DK = idesc_bf16(128, BWD_D, 0, 1);       // dK (A TMEM, B MN-major)
             constexpr uint32_t ID_DQ = idesc_bf16(128, BWD_BM, 1, 1);      // dQ^T (A and B MN-major)
             const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
             uint32_t g = 0, it_n = 0;
             // K-major x K-major product over d (S^T = K Q^T or dP^T = V dO^T)
-            auto issue_kk = [&](uint32_t col, uint32_t a, uint32_t b) {
+            const uint64_t ones_desc = smem_desc(smem_u32(sm.aug_ones), BwdSmem::AUG_LBO, BwdSmem::AUG_SBO, 0);
+            auto issue_kk = [&](uint32_t col, uint32_t a, uint32_t b, const uint8_t *aug) {
 #pragma unroll
                 for (int kk = 0; kk < BWD_D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * BwdSmem::CHUNK + (kk & 3) * 32;
                     umma_ss(tmem + col, smem_desc(a + off, 16, 1024), smem_desc(b + off, 16, 1024), ID_SDP, kk > 0);
                 }
+                // the extra slice: + (1,1,1) . split(value of the query row)
+                umma_ss(tmem + col, ones_desc, smem_desc(smem_u32(aug), BwdSmem::AUG_LBO, BwdSmem::AUG_SBO, 0),
+                        ID_SDP, 1u);
             };
             auto issue_dp = [&](uint32_t gg) -> bool {      // dP^T(gg), once dQ^T(gg - 1) has been read out
                 if (gg > 0 && !bwait(&sm.dq_free, (gg - 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                issue_kk(COL_DP, sv, smem_u32(sm.dout[gg % BwdSmem::QSTAGES]));
+                issue_kk(COL_DP, sv, smem_u32(sm.dout[gg % BwdSmem::QSTAGES]), sm.aug_do[gg % BwdSmem::QSTAGES]);
                 umma_commit(&sm.dp_full);
                 return true;
             };
@@ -282,7 +322,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 const int st = gg % BwdSmem::QSTAGES;
                 if (!bwait(&sm.q_full[st], (gg / BwdSmem::QSTAGES) & 1, abort_flag)) return false;
                 tc_fence_after();
-                issue_kk(COL_S, sk, smem_u32(sm.q[st]));
+                issue_kk(COL_S, sk, smem_u32(sm.q[st]), sm.aug_q[st]);
                 umma_commit(&sm.s_full);
                 return true;
             };
@@ -310,11 +350,9 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     if (!bwait(&sm.ds_ready, g & 1, abort_flag)) goto done;
                     tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < BWD_BM / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * BwdSmem::CHUNK + (kk & 3) * 32;
-                        umma_ss(tmem + COL_DK, smem_desc(sdo + off, 16, 1024),
-                                smem_desc(sq + kk * 2048, BwdSmem::CHUNK, 1024), ID_DK, (t > 0 || kk > 0));
-                    }
+                    for (int kk = 0; kk < BWD_BM / 16; ++kk)
+                        umma_ts(tmem + COL_DK, tmem + COL_DP + kk * 8, smem_desc(sq + kk * 2048, BwdSmem::CHUNK, 1024),
+                                ID_DK, (t > 0 || kk > 0));
 #pragma unroll
                     for (int kk = 0; kk < 128 / 16; ++kk)
                         umma_ss(tmem + COL_DP, smem_desc(sk + kk * 2048, BwdSmem::CHUNK, 1024),
@@ -343,11 +381,9 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             for (int t = 0; t < n; ++t, ++g) {
                 const int st = g % BwdSmem::QSTAGES;
                 const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
-                const float4 *ldp = sm.ld[st];
                 const int lo = y - x0, hi = ke - x0;                   // allowed query columns [lo, hi)
-                // phase 1: P^T = exp2(S^T * scale * log2 e - lse * log2 e), kept packed for phase 2
+                // phase 1: P^T = exp2(S'^T * scale * log2 e) (S' already holds s - lse / scale), kept packed
                 if (!bwait(&sm.s_full, g & 1, abort_flag)) goto done;
-                if (!bwait(&sm.q_full[st], (g / BwdSmem::QSTAGES) & 1, abort_flag)) goto done;
                 tc_fence_after();
                 uint32_t pk[64];
 #pragma unroll
@@ -358,9 +394,8 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const int col = 32 * c + 2 * e;
-                        const float4 l = ldp[col];
-                        const float p0 = (col >= lo && col < hi) ? ex2_approx(fmaf(__uint_as_float(sr[2 * e]), sl2, -l.x)) : 0.f;
-                        const float p1 = (col + 1 >= lo && col + 1 < hi) ? ex2_approx(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, -l.z)) : 0.f;
+                        const float p0 = (col >= lo && col < hi) ? ex2_approx(__uint_as_float(sr[2 * e]) * sl2) : 0.f;
+                        const float p1 = (col + 1 >= lo && col + 1 < hi) ? ex2_approx(__uint_as_float(sr[2 * e + 1]) * sl2) : 0.f;
                         pk[16 * c + e] = pack_bf16x2(p0, p1);
                     }
                     uint32_t tmp[16];
@@ -384,12 +419,11 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     uint32_t dd[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const int col = 32 * c + 2 * e;
-                        const float4 l = ldp[col];
-                        const uint32_t p = pk[16 * c + e];
-                        dd[e] = pack_bf16x2(bf16lo(p) * (__uint_as_float(pr[2 * e]) - l.y),
-                                            bf16hi(p) * (__uint_as_float(pr[2 * e + 1]) - l.w));
+                        const uint32_t p = pk[16 * c + e];                 // dP' = dP - D already
+                        dd[e] = pack_bf16x2(bf16lo(p) * __uint_as_float(pr[2 * e]) * scale,
+                                            bf16hi(p) * __uint_as_float(pr[2 * e + 1]) * scale);
                     }
+                    tmem_st16(tmem + lane_off + COL_DP + c * 16, dd);     // dS^T cols [16c, 16c+16): dP chunks <= c
                     // queries [32c, 32c+32): 64-column chunk c/2, 16-byte pieces 4(c%2)..4(c%2)+3, swizzled by row
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
@@ -398,14 +432,15 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                             make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
                     }
                 }
+                tmem_wait_st();
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(&sm.ds_ready);
             }
-            // item epilogue: dK (scaled); the dQ warpgroup writes dV
+            // item epilogue: dK (dS^T carried the scale); the dQ warpgroup writes dV
             if (!bwait(&sm.dkv_full, it_n & 1, abort_flag)) goto done;
             tc_fence_after();
-            bwd_store_kv(tmem + lane_off + COL_DK, yin, w.split, scale, dk_acc, dK, (int64_t(y) * hkv + w.kh) * BWD_D);
+            bwd_store_kv(tmem + lane_off + COL_DK, yin, w.split, 1.f, dk_acc, dK, (int64_t(y) * hkv + w.kh) * BWD_D);
             tc_fence_before();
             mbar_arrive(&sm.dkv_free);
         }
@@ -437,7 +472,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 // dQ rows x0..x0+127, column dcol: one coalesced 128-byte add per warp and row
                 float *gdst = dq_acc + (int64_t(h) * rows_pad + x0) * BWD_D + dcol;
 #pragma unroll
-                for (int c = 0; c < BWD_BM; ++c) red_add_f32(gdst + c * BWD_D, __uint_as_float(v[c]) * scale);
+                for (int c = 0; c < BWD_BM; ++c) red_add_f32(gdst + c * BWD_D, __uint_as_float(v[c]));
             }
             // item epilogue: dV rows (TMEM lane = key row for this read)
             const int jr = wq * 32 + lane;
@@ -512,7 +547,7 @@ inline pp_status launch_bwd(const void *q, const void *k, const void *v, const v
     if (d != BWD_D) return fail(PP_ERR_UNSUPPORTED, "backward supports head dim 128 only (got %d)", d);
     const BwdWorkspace L = bwd_workspace_layout(T, hq, hkv, d);
     char *ws = static_cast<char *>(workspace);
-    float4 *ldg = reinterpret_cast<float4 *>(ws + L.off_delta);
+    float2 *ldg = reinterpret_cast<float2 *>(ws + L.off_delta);
     float *dq_acc = reinterpret_cast<float *>(ws + L.off_dq);
     float *dk_acc = reinterpret_cast<float *>(ws + L.off_dk);
     float *dv_acc = reinterpret_cast<float *>(ws + L.off_dv);
@@ -529,7 +564,8 @@ inline pp_status launch_bwd(const void *q, const void *k, const void *v, const v
     if ((e = cudaMemsetAsync(ws + L.off_dq, 0, L.total - L.off_dq, s)) != cudaSuccess)
         return fail(PP_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
     k_bwd_pre<<<sm_count * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(o),
-                                           static_cast<const __nv_bfloat16 *>(dout), lse, ldg, T, L.rows_pad, hq);
+                                           static_cast<const __nv_bfloat16 *>(dout), lse, ldg, T, L.rows_pad, hq,
+                                           1.f / scale);
     if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_pre: %s", cudaGetErrorString(e));
     const size_t smem = sizeof(BwdSmem) + 1024;
     if ((e = cudaFuncSetAttribute(k_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem))) != cudaSuccess)

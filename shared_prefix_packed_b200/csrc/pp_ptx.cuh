@@ -150,13 +150,14 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // ------------------------------------------------------------------------------------------------ descriptors
 // Shared-memory matrix descriptor for UMMA (sm_100 format): start address, leading and stride byte offsets
 // (all >> 4), version 1 at bits 46-47, swizzle mode at bits 61-63 (2 = 128-byte swizzle).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t layout = 2u) {
     uint64_t d = 0;
     d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
     d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
     d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
     d |= static_cast<uint64_t>(1u) << 46;
-    d |= static_cast<uint64_t>(2u) << 61;
+    d |= static_cast<uint64_t>(layout) << 61;      // 2 = 128-byte swizzle, 0 = no swizzle (8x16-byte core matrices)
     return d;
 }
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D. a_mn/b_mn: operand is MN-major (1) or K-major (0).
