@@ -264,13 +264,32 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 }
             }
             const int n = (w.qb - w.qa) * r;
+            auto step_h = [&](int t) { return w.kh * r + t % r; };
+            auto step_x0 = [&](int t) { return w.t.gstart + (w.qa + t / r) * BWD_BM; };
+            float2 lv[4];                                              // rows lane + 32u of the current step
+#pragma unroll
+            for (int u = 0; u < 4; ++u) lv[u] = ldg[int64_t(step_h(0)) * rows_pad + step_x0(0) + lane + 32 * u];
+            if (lane == 0)
+                for (int t = 0; t < 2 && t < n; ++t)
+                    for (int c = 0; c < BWD_D / 64; ++c) {
+                        tma_prefetch_3d(&tmQ, c * 64, step_h(t), step_x0(t));
+                        tma_prefetch_3d(&tmdO, c * 64, step_h(t), step_x0(t));
+                    }
             for (int t = 0; t < n; ++t, ++g) {
                 const int st = g % BwdSmem::QSTAGES;
-                const int h = w.kh * r + t % r;
-                const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
-                float2 lv[4];                                          // rows lane + 32u of the step
+                const int h = step_h(t);
+                const int x0 = step_x0(t);
+                // next step's values and (two steps ahead) its tiles: their latency hides behind this step
+                float2 nv[4];
+                if (t + 1 < n) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) lv[u] = ldg[int64_t(h) * rows_pad + x0 + lane + 32 * u];
+                    for (int u = 0; u < 4; ++u) nv[u] = ldg[int64_t(step_h(t + 1)) * rows_pad + step_x0(t + 1) + lane + 32 * u];
+                }
+                if (lane == 0 && t + 2 < n)
+                    for (int c = 0; c < BWD_D / 64; ++c) {
+                        tma_prefetch_3d(&tmQ, c * 64, step_h(t + 2), step_x0(t + 2));
+                        tma_prefetch_3d(&tmdO, c * 64, step_h(t + 2), step_x0(t + 2));
+                    }
                 if (!bwait(&sm.q_empty[st], ((g / BwdSmem::QSTAGES) & 1) ^ 1, abort_flag)) goto done;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -287,6 +306,10 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     }
                 } else {
                     mbar_arrive(&sm.q_full[st]);
+                }
+                if (t + 1 < n) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) lv[u] = nv[u];
                 }
             }
         }
@@ -344,8 +367,13 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         umma_ts(tmem + COL_DV, tmem + COL_S + kk * 8, smem_desc(sdo + kk * 2048, BwdSmem::CHUNK, 1024),
                                 ID_DV, (t > 0 || kk > 0));
                     umma_commit(&sm.dv_done);
-                    // S^T of the next step may overwrite P^T now (MMAs run in issue order)
-                    if (t + 1 < n && !issue_s(g + 1)) goto done;
+                    // S^T of the next step may overwrite P^T now (MMAs run in issue order); issue it first only if
+                    // its tile has landed, so a late load never holds up dK/dQ^T of this step
+                    bool s_next = false;
+                    if (t + 1 < n && mbar_try_wait(&sm.q_full[(g + 1) % BwdSmem::QSTAGES], ((g + 1) / BwdSmem::QSTAGES) & 1)) {
+                        if (!issue_s(g + 1)) goto done;
+                        s_next = true;
+                    }
                     // dK += dS^T Q and dQ^T = K^T dS^T once dS^T is in shared memory
                     if (!bwait(&sm.ds_ready, g & 1, abort_flag)) goto done;
                     tc_fence_after();
@@ -359,6 +387,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                                 smem_desc(sdo + kk * 2048, BwdSmem::CHUNK, 1024), ID_DQ, kk > 0);
                     umma_commit(&sm.dq_full);
                     umma_commit(&sm.q_empty[st]);
+                    if (t + 1 < n && !s_next && !issue_s(g + 1)) goto done;
                     if (t + 1 < n && !issue_dp(g + 1)) goto done;
                 }
                 umma_commit(&sm.dkv_full);
