@@ -20,8 +20,9 @@
 //                                                          dO tile's buffer once dV has read it
 //                   dK  += dS^T Q        (A from TMEM)    TMEM dK
 //                   dQ^T = K^T dS^T      (M = d)          TMEM dP (dK has read dS^T: MMAs run in issue order)
-//                 dQ^T is read by a second warpgroup (TMEM lane = head-dim index), scaled and added to an fp32
-//                 accumulator from registers: per row one coalesced 128-byte red.global.add per warp. dK/dV stay
+//                 Two gradient warpgroups each own half of the query columns; they also read dQ^T (TMEM lane =
+//                 head-dim index) and add it to an fp32 accumulator from registers: per row one coalesced 128-byte
+//                 red.global.add per warp. dK/dV stay
 //                 in TMEM for the whole item; an unsplit key tile writes them as bf16, a split one adds its fp32
 //                 partial into the workspace (one add per element and chunk).
 //   k_bwd_convert dQ (and the split tiles' dK/dV) from the fp32 accumulators to bf16.
@@ -212,11 +213,11 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         }
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.dp_full, 1);
-        mbar_init(&sm.p_ready, 128);
+        mbar_init(&sm.p_ready, 256);
         mbar_init(&sm.dv_done, 1);
-        mbar_init(&sm.ds_ready, 128);
+        mbar_init(&sm.ds_ready, 256);
         mbar_init(&sm.dq_full, 1);
-        mbar_init(&sm.dq_free, 128);
+        mbar_init(&sm.dq_free, 256);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -364,8 +365,8 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < BWD_BM / 16; ++kk)
-                        umma_ts(tmem + COL_DV, tmem + COL_S + kk * 8, smem_desc(sdo + kk * 2048, BwdSmem::CHUNK, 1024),
-                                ID_DV, (t > 0 || kk > 0));
+                        umma_ts(tmem + COL_DV, tmem + COL_S + 64 * (kk >> 2) + 8 * (kk & 3),
+                                smem_desc(sdo + kk * 2048, BwdSmem::CHUNK, 1024), ID_DV, (t > 0 || kk > 0));
                     umma_commit(&sm.dv_done);
                     // S^T of the next step may overwrite P^T now (MMAs run in issue order); issue it first only if
                     // its tile has landed, so a late load never holds up dK/dQ^T of this step
@@ -379,8 +380,8 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < BWD_BM / 16; ++kk)
-                        umma_ts(tmem + COL_DK, tmem + COL_DP + kk * 8, smem_desc(sq + kk * 2048, BwdSmem::CHUNK, 1024),
-                                ID_DK, (t > 0 || kk > 0));
+                        umma_ts(tmem + COL_DK, tmem + COL_DP + 64 * (kk >> 2) + 8 * (kk & 3),
+                                smem_desc(sq + kk * 2048, BwdSmem::CHUNK, 1024), ID_DK, (t > 0 || kk > 0));
 #pragma unroll
                     for (int kk = 0; kk < 128 / 16; ++kk)
                         umma_ss(tmem + COL_DP, smem_desc(sk + kk * 2048, BwdSmem::CHUNK, 1024),
@@ -394,10 +395,17 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 umma_commit(&sm.kv_empty);
             }
         }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------------ softmax / gradient warpgroup
-        const int jr = warp * 32 + lane;                               // key row within the tile = TMEM lane
-        const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    } else {
+        // ------------------------------------------------------------------ gradient warpgroups (warps 0-7)
+        // Warpgroup x handles query columns [64x, 64x+64) of every step: P (phase 1), dS (phase 2) and the dQ^T
+        // read-out. Its P^T and dS^T (bf16) go into TMEM columns it has itself already read: S cols [64x, 64x+32)
+        // and dP cols [64x, 64x+32) of their regions. Per step the order is dS(t), P(t+1), dQ(t), so the next
+        // step's P overlaps this step's dK/dQ^T MMAs.
+        const int wx = warp >> 2;                                      // column half
+        const int wl = warp & 3;
+        const int jr = wl * 32 + lane;                                 // TMEM lane: key row (P, dS) or d (dQ^T)
+        const uint32_t lane_off = uint32_t(wl * 32) << 16;
+        const int cb = 64 * wx;                                        // first query column of this half
         uint32_t g = 0, it_n = 0;
         const int32_t *key_end = meta_ptr<int32_t>(meta, hd.off_key_end);
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
@@ -407,109 +415,115 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             const int gend = w.t.gstart + w.t.glen;
             const bool yin = y < gend;
             const int ke = yin ? key_end[y] : y;                       // queries [y, ke) attend key y
-            for (int t = 0; t < n; ++t, ++g) {
-                const int st = g % BwdSmem::QSTAGES;
+            uint32_t pk[32];                                           // P^T of the current step, packed bf16
+            // phase 1 of step gg: P^T = exp2(S'^T * scale * log2 e) (S' already holds s - lse / scale)
+            auto phase_p = [&](uint32_t gg, int t) -> bool {
                 const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
-                const int lo = y - x0, hi = ke - x0;                   // allowed query columns [lo, hi)
-                // phase 1: P^T = exp2(S'^T * scale * log2 e) (S' already holds s - lse / scale), kept packed
-                if (!bwait(&sm.s_full, g & 1, abort_flag)) goto done;
+                const int lo = y - x0 - cb, hi = ke - x0 - cb;         // allowed columns [lo, hi) of this half
+                const bool all_in = __all_sync(0xffffffffu, lo <= 0 && hi >= 64);
+                if (!bwait(&sm.s_full, gg & 1, abort_flag)) return false;
                 tc_fence_after();
-                uint32_t pk[64];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t sr[32];
-                    tmem_ld32(tmem + lane_off + COL_S + c * 32, sr);
+                uint32_t sr[64];
+                {
+                    uint32_t a0[32], a1[32];
+                    tmem_ld32(tmem + lane_off + COL_S + cb, a0);
+                    tmem_ld32(tmem + lane_off + COL_S + cb + 32, a1);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int col = 32 * c + 2 * e;
-                        const float p0 = (col >= lo && col < hi) ? ex2_approx(__uint_as_float(sr[2 * e]) * sl2) : 0.f;
-                        const float p1 = (col + 1 >= lo && col + 1 < hi) ? ex2_approx(__uint_as_float(sr[2 * e + 1]) * sl2) : 0.f;
-                        pk[16 * c + e] = pack_bf16x2(p0, p1);
-                    }
-                    uint32_t tmp[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) tmp[e] = pk[16 * c + e];
-                    tmem_st16(tmem + lane_off + COL_S + c * 16, tmp);  // P^T cols [16c, 16c+16): S chunks <= c
+                    for (int e = 0; e < 32; ++e) { sr[e] = a0[e]; sr[32 + e] = a1[e]; }
                 }
+                if (all_in) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        pk[e] = pack_bf16x2(ex2_approx(__uint_as_float(sr[2 * e]) * sl2),
+                                            ex2_approx(__uint_as_float(sr[2 * e + 1]) * sl2));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int c = 2 * e;
+                        const float p0 = (c >= lo && c < hi) ? ex2_approx(__uint_as_float(sr[c]) * sl2) : 0.f;
+                        const float p1 = (c + 1 >= lo && c + 1 < hi) ? ex2_approx(__uint_as_float(sr[c + 1]) * sl2) : 0.f;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                }
+                uint32_t t0[16], t1[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) { t0[e] = pk[e]; t1[e] = pk[16 + e]; }
+                tmem_st16(tmem + lane_off + COL_S + cb, t0);
+                tmem_st16(tmem + lane_off + COL_S + cb + 16, t1);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.p_ready);
-                // phase 2: dS^T = P^T (dP^T - D) into the dO buffer, which dV has finished reading
+                return true;
+            };
+            if (n > 0 && !phase_p(g, 0)) goto done;
+            for (int t = 0; t < n; ++t, ++g) {
+                const int st = g % BwdSmem::QSTAGES;
+                const int h = w.kh * r + t % r;
+                const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
+                // phase 2: dS^T = scale P^T dP'^T (dP' = dP - D already) -> TMEM and the dO buffer (dV has read it)
                 if (!bwait(&sm.dp_full, g & 1, abort_flag)) goto done;
                 if (!bwait(&sm.dv_done, g & 1, abort_flag)) goto done;
                 tc_fence_after();
-                uint8_t *dsrow = sm.dout[st] + jr * 128;
+                {
+                    uint32_t pr[64];
+                    {
+                        uint32_t a0[32], a1[32];
+                        tmem_ld32(tmem + lane_off + COL_DP + cb, a0);
+                        tmem_ld32(tmem + lane_off + COL_DP + cb + 32, a1);
+                        tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t pr[32];
-                    tmem_ld32(tmem + lane_off + COL_DP + c * 32, pr);
-                    tmem_wait_ld();
-                    uint32_t dd[16];
+                        for (int e = 0; e < 32; ++e) { pr[e] = a0[e]; pr[32 + e] = a1[e]; }
+                    }
+                    uint32_t dd[32];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const uint32_t p = pk[16 * c + e];                 // dP' = dP - D already
+                    for (int e = 0; e < 32; ++e) {
+                        const uint32_t p = pk[e];
                         dd[e] = pack_bf16x2(bf16lo(p) * __uint_as_float(pr[2 * e]) * scale,
                                             bf16hi(p) * __uint_as_float(pr[2 * e + 1]) * scale);
                     }
-                    tmem_st16(tmem + lane_off + COL_DP + c * 16, dd);     // dS^T cols [16c, 16c+16): dP chunks <= c
-                    // queries [32c, 32c+32): 64-column chunk c/2, 16-byte pieces 4(c%2)..4(c%2)+3, swizzled by row
+                    uint32_t t0[16], t1[16];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int piece = 4 * (c & 1) + u;
-                        *reinterpret_cast<uint4 *>(dsrow + (c >> 1) * BwdSmem::CHUNK + ((piece ^ (jr & 7)) << 4)) =
-                            make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
-                    }
+                    for (int e = 0; e < 16; ++e) { t0[e] = dd[e]; t1[e] = dd[16 + e]; }
+                    tmem_st16(tmem + lane_off + COL_DP + cb, t0);
+                    tmem_st16(tmem + lane_off + COL_DP + cb + 16, t1);
+                    // dS^T row jr, queries [cb, cb+64) = 64-column chunk wx of the swizzled [key][query] tile
+                    uint8_t *dsrow = sm.dout[st] + wx * BwdSmem::CHUNK + jr * 128;
+#pragma unroll
+                    for (int piece = 0; piece < 8; ++piece)
+                        *reinterpret_cast<uint4 *>(dsrow + ((piece ^ (jr & 7)) << 4)) =
+                            make_uint4(dd[4 * piece], dd[4 * piece + 1], dd[4 * piece + 2], dd[4 * piece + 3]);
                 }
                 tmem_wait_st();
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(&sm.ds_ready);
-            }
-            // item epilogue: dK (dS^T carried the scale); the dQ warpgroup writes dV
-            if (!bwait(&sm.dkv_full, it_n & 1, abort_flag)) goto done;
-            tc_fence_after();
-            bwd_store_kv(tmem + lane_off + COL_DK, yin, w.split, 1.f, dk_acc, dK, (int64_t(y) * hkv + w.kh) * BWD_D);
-            tc_fence_before();
-            mbar_arrive(&sm.dkv_free);
-        }
-    } else {
-        // ------------------------------------------------------------------ dQ warpgroup (warps 4-7)
-        const int wq = warp - 4;
-        const int dcol = wq * 32 + lane;                               // head-dim index = TMEM lane
-        const uint32_t lane_off = uint32_t(wq * 32) << 16;
-        uint32_t g = 0, it_n = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
-            const BwdItem w = bwd_decode(meta, hd, item);
-            const int n = (w.qb - w.qa) * r;
-            for (int t = 0; t < n; ++t, ++g) {
-                const int h = w.kh * r + t % r;
-                const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
+                // next step's phase 1 while this step's dK and dQ^T run
+                if (t + 1 < n && !phase_p(g + 1, t + 1)) goto done;
+                // dQ^T read-out: TMEM lane = d index, columns [cb, cb+64) = query rows x0 + cb + c
                 if (!bwait(&sm.dq_full, g & 1, abort_flag)) goto done;
                 tc_fence_after();
-                uint32_t v[128];
+                {
+                    uint32_t a0[32], a1[32];
+                    tmem_ld32(tmem + lane_off + COL_DP + cb, a0);
+                    tmem_ld32(tmem + lane_off + COL_DP + cb + 32, a1);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive(&sm.dq_free);
+                    float *gdst = dq_acc + (int64_t(h) * rows_pad + x0 + cb) * BWD_D + jr;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t tmp[32];
-                    tmem_ld32(tmem + lane_off + COL_DP + c * 32, tmp);
+                    for (int c = 0; c < 32; ++c) red_add_f32(gdst + c * BWD_D, __uint_as_float(a0[c]));
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[32 * c + e] = tmp[e];
+                    for (int c = 0; c < 32; ++c) red_add_f32(gdst + (32 + c) * BWD_D, __uint_as_float(a1[c]));
                 }
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(&sm.dq_free);
-                // dQ rows x0..x0+127, column dcol: one coalesced 128-byte add per warp and row
-                float *gdst = dq_acc + (int64_t(h) * rows_pad + x0) * BWD_D + dcol;
-#pragma unroll
-                for (int c = 0; c < BWD_BM; ++c) red_add_f32(gdst + c * BWD_D, __uint_as_float(v[c]));
             }
-            // item epilogue: dV rows (TMEM lane = key row for this read)
-            const int jr = wq * 32 + lane;
-            const int y = w.t.row0 + jr;
-            const bool yin = y < w.t.gstart + w.t.glen;
+            // item epilogue: warpgroup 0 writes dK (dS^T carried the scale), warpgroup 1 writes dV
             if (!bwait(&sm.dkv_full, it_n & 1, abort_flag)) goto done;
             tc_fence_after();
-            bwd_store_kv(tmem + lane_off + COL_DV, yin, w.split, 1.f, dv_acc, dV, (int64_t(y) * hkv + w.kh) * BWD_D);
+            if (wx == 0)
+                bwd_store_kv(tmem + lane_off + COL_DK, yin, w.split, 1.f, dk_acc, dK, (int64_t(y) * hkv + w.kh) * BWD_D);
+            else
+                bwd_store_kv(tmem + lane_off + COL_DV, yin, w.split, 1.f, dv_acc, dV, (int64_t(y) * hkv + w.kh) * BWD_D);
             tc_fence_before();
             mbar_arrive(&sm.dkv_free);
         }

@@ -253,13 +253,20 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 ++s_cnt;
                 tc_fence_after();
                 float s[FWD_BN];
-#pragma unroll
-                for (int c = 0; c < FWD_BN / 32; ++c) {
-                    uint32_t rr[32];
-                    tmem_ld32(t_s + c * 32, rr);
+                {   // all four loads in flight before one wait
+                    uint32_t r0[32], r1[32], r2[32], r3[32];
+                    tmem_ld32(t_s, r0);
+                    tmem_ld32(t_s + 32, r1);
+                    tmem_ld32(t_s + 64, r2);
+                    tmem_ld32(t_s + 96, r3);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[e]);
+                    for (int e = 0; e < 32; ++e) {
+                        s[e] = __uint_as_float(r0[e]);
+                        s[32 + e] = __uint_as_float(r1[e]);
+                        s[64 + e] = __uint_as_float(r2[e]);
+                        s[96 + e] = __uint_as_float(r3[e]);
+                    }
                 }
                 if (cls != TILE_FULL) {
                     // allowed iff y <= row, and y in the prefix or in row's own segment; nothing for rows outside
@@ -270,9 +277,10 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     for (int c = 0; c < FWD_BN; ++c)
                         if (!(c <= lim_diag && (c < lim_pfx || c >= lim_seg))) s[c] = -INFINITY;
                 }
-                float mx = s[0];
+                float m4[4] = {s[0], s[1], s[2], s[3]};                 // four independent max chains
 #pragma unroll
-                for (int c = 1; c < FWD_BN; ++c) mx = fmaxf(mx, s[c]);
+                for (int c = 4; c < FWD_BN; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
                 const float mt = mx * sl2;
                 bool rescale = false;
                 float alpha = 1.f;
@@ -285,7 +293,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     m = mt;
                 }
                 const float mu = (m == -INFINITY) ? 0.f : m;
-                float lsum = 0.f;
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};                      // four independent sum chains
 #pragma unroll
                 for (int c = 0; c < FWD_BN / 32; ++c) {
                     uint32_t pk[16];
@@ -293,12 +301,12 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     for (int e = 0; e < 16; ++e) {
                         const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * e], sl2, -mu));
                         const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * e + 1], sl2, -mu));
-                        lsum += p0 + p1;
+                        ls[e & 3] += p0 + p1;
                         pk[e] = pack_bf16x2(p0, p1);
                     }
                     tmem_st16(t_s + c * 16, pk);
                 }
-                l += lsum;
+                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
                 tmem_wait_st();
                 // tcgen05.ld/st are warp-collective: the whole warp takes the rescale path if any row needs it
                 if (__any_sync(0xffffffffu, rescale)) {
