@@ -20,9 +20,9 @@
 //                                                          dO tile's buffer once dV has read it
 //                   dK  += dS^T Q        (A from TMEM)    TMEM dK
 //                   dQ^T = K^T dS^T      (M = d)          TMEM dP (dK has read dS^T: MMAs run in issue order)
-//                 Two gradient warpgroups each own half of the query columns; they also read dQ^T (TMEM lane =
-//                 head-dim index) and add it to an fp32 accumulator from registers: per row one coalesced 128-byte
-//                 red.global.add per warp. dK/dV stay
+//                 Two gradient warpgroups each own half of the query columns; a third warpgroup reads dQ^T (TMEM
+//                 lane = head-dim index) and adds it to an fp32 accumulator from registers: per row one coalesced
+//                 128-byte red.global.add per warp, concurrently with the next step's softmax work. dK/dV stay
 //                 in TMEM for the whole item; an unsplit key tile writes them as bf16, a split one adds its fp32
 //                 partial into the workspace (one add per element and chunk).
 //   k_bwd_convert dQ (and the split tiles' dK/dV) from the fp32 accumulators to bf16.
@@ -47,7 +47,7 @@
 
 namespace pp {
 
-constexpr int BWD_THREADS = 320;
+constexpr int BWD_THREADS = 448;   // 8 gradient warps, 4 dQ warps, producer, MMA
 constexpr int BWD_D = 128;
 
 struct BwdWorkspace {
@@ -217,7 +217,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         mbar_init(&sm.dv_done, 1);
         mbar_init(&sm.ds_ready, 256);
         mbar_init(&sm.dq_full, 1);
-        mbar_init(&sm.dq_free, 256);
+        mbar_init(&sm.dq_free, 128);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -233,11 +233,11 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         }
         fence_proxy_async_smem();
     }
-    if (warp == 9) {
+    if (warp == 13) {
         tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == 12 && lane == 0) {
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
@@ -251,7 +251,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
 
     if (hd.dev_err != 0) {
         // nothing to do: the metadata builder rejected its input
-    } else if (warp == 8) {
+    } else if (warp == 12) {
         // ------------------------------------------------------------------ producer warp
         uint32_t g = 0, it_n = 0;
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
@@ -314,7 +314,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 }
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == 13) {
         // ------------------------------------------------------------------ MMA issuer (one thread)
         if (lane == 0) {
             constexpr uint32_t ID_SDP = idesc_bf16(128, BWD_BM, 0, 0);     // S^T, dP^T (both K-major)
@@ -395,12 +395,48 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 umma_commit(&sm.kv_empty);
             }
         }
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------------ dQ warpgroup (warps 8-11)
+        // dQ^T (TMEM lane = head-dim index) is read as soon as its MMA completes and added to the fp32
+        // accumulator: per query row one coalesced 128-byte red.global.add per warp. Running these adds on their own
+        // warps keeps the reduction traffic off the gradient warps' step.
+        const int wl = warp & 3;
+        const int dcol = wl * 32 + lane;
+        const uint32_t lane_off = uint32_t(wl * 32) << 16;
+        uint32_t g = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+            const BwdItem w = bwd_decode(meta, hd, item);
+            const int n = (w.qb - w.qa) * r;
+            for (int t = 0; t < n; ++t, ++g) {
+                const int h = w.kh * r + t % r;
+                const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
+                if (!bwait(&sm.dq_full, g & 1, abort_flag)) goto done;
+                tc_fence_after();
+                uint32_t a0[32], a1[32], a2[32], a3[32];
+                tmem_ld32(tmem + lane_off + COL_DP, a0);
+                tmem_ld32(tmem + lane_off + COL_DP + 32, a1);
+                tmem_ld32(tmem + lane_off + COL_DP + 64, a2);
+                tmem_ld32(tmem + lane_off + COL_DP + 96, a3);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&sm.dq_free);
+                float *gdst = dq_acc + (int64_t(h) * rows_pad + x0) * BWD_D + dcol;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) red_add_f32(gdst + c * BWD_D, __uint_as_float(a0[c]));
+#pragma unroll
+                for (int c = 0; c < 32; ++c) red_add_f32(gdst + (32 + c) * BWD_D, __uint_as_float(a1[c]));
+#pragma unroll
+                for (int c = 0; c < 32; ++c) red_add_f32(gdst + (64 + c) * BWD_D, __uint_as_float(a2[c]));
+#pragma unroll
+                for (int c = 0; c < 32; ++c) red_add_f32(gdst + (96 + c) * BWD_D, __uint_as_float(a3[c]));
+            }
+        }
     } else {
         // ------------------------------------------------------------------ gradient warpgroups (warps 0-7)
-        // Warpgroup x handles query columns [64x, 64x+64) of every step: P (phase 1), dS (phase 2) and the dQ^T
-        // read-out. Its P^T and dS^T (bf16) go into TMEM columns it has itself already read: S cols [64x, 64x+32)
-        // and dP cols [64x, 64x+32) of their regions. Per step the order is dS(t), P(t+1), dQ(t), so the next
-        // step's P overlaps this step's dK/dQ^T MMAs.
+        // Warpgroup x handles query columns [64x, 64x+64) of every step: P (phase 1) and dS (phase 2). Its P^T and
+        // dS^T (bf16) go into TMEM columns it has itself already read: S cols [64x, 64x+32) and dP cols
+        // [64x, 64x+32) of their regions. Per step the order is dS(t), P(t+1), so the next step's P overlaps this
+        // step's dK/dQ^T MMAs.
         const int wx = warp >> 2;                                      // column half
         const int wl = warp & 3;
         const int jr = wl * 32 + lane;                                 // TMEM lane: key row (P, dS) or d (dQ^T)
@@ -459,8 +495,6 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             if (n > 0 && !phase_p(g, 0)) goto done;
             for (int t = 0; t < n; ++t, ++g) {
                 const int st = g % BwdSmem::QSTAGES;
-                const int h = w.kh * r + t % r;
-                const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
                 // phase 2: dS^T = scale P^T dP'^T (dP' = dP - D already) -> TMEM and the dO buffer (dV has read it)
                 if (!bwait(&sm.dp_full, g & 1, abort_flag)) goto done;
                 if (!bwait(&sm.dv_done, g & 1, abort_flag)) goto done;
@@ -500,22 +534,6 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 mbar_arrive(&sm.ds_ready);
                 // next step's phase 1 while this step's dK and dQ^T run
                 if (t + 1 < n && !phase_p(g + 1, t + 1)) goto done;
-                // dQ^T read-out: TMEM lane = d index, columns [cb, cb+64) = query rows x0 + cb + c
-                if (!bwait(&sm.dq_full, g & 1, abort_flag)) goto done;
-                tc_fence_after();
-                {
-                    uint32_t a0[32], a1[32];
-                    tmem_ld32(tmem + lane_off + COL_DP + cb, a0);
-                    tmem_ld32(tmem + lane_off + COL_DP + cb + 32, a1);
-                    tmem_wait_ld();
-                    tc_fence_before();
-                    mbar_arrive(&sm.dq_free);
-                    float *gdst = dq_acc + (int64_t(h) * rows_pad + x0 + cb) * BWD_D + jr;
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) red_add_f32(gdst + c * BWD_D, __uint_as_float(a0[c]));
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) red_add_f32(gdst + (32 + c) * BWD_D, __uint_as_float(a1[c]));
-                }
             }
             // item epilogue: warpgroup 0 writes dK (dS^T carried the scale), warpgroup 1 writes dV
             if (!bwait(&sm.dkv_full, it_n & 1, abort_flag)) goto done;
@@ -531,7 +549,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
 done:
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == 13) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
