@@ -4,56 +4,54 @@
 //   dS_ij = p_ij (dO_i . v_j - D_i),  dQ_i = scale sum_j dS_ij k_j,
 //   dK_j = scale sum_h sum_i dS_ij q_i,  dV_j = sum_h sum_i p_ij dO_i   (h over the q heads of j's kv head).
 //
-// Three kernels:
-//   k_bwd_pre     (lse * log2 e, D = rowsum(dO * O)) per row and head, fp32 (HBM-bound).
-//   k_bwd_tc      key/value-stationary tensor-core kernel. A work item is (key tile of 128 rows, kv head, chunk of
-//                 the query tiles that attend it). Seen from key y the attending queries are one interval
-//                 [y, e(y)) (pp_meta.cuh), so a key tile's query tiles are one contiguous range; prefix key tiles
-//                 (attended by every response of the group) get long ranges and are split into chunks so the
-//                 persistent grid stays balanced. Per step (query tile of 128 rows, one q head of the kv head),
-//                 five MMAs, all with N = 128 (an N = 64 MMA costs as long as an N = 128 one on this part):
-//                   S^T  = K Q^T                          TMEM S
-//                   dP^T = V dO^T                         TMEM dP
-//                   softmax warps, phase 1: P^T = exp(S^T - lse) -> TMEM S (bf16)      -> dV may start
-//                   dV  += P^T dO        (A from TMEM)    TMEM dV
-//                   softmax warps, phase 2: dS^T = scale P^T (dP^T - D) -> TMEM dP (bf16) and smem, into the
-//                                                          dO tile's buffer once dV has read it
-//                   dK  += dS^T Q        (A from TMEM)    TMEM dK
-//                   dQ^T = K^T dS^T      (M = d)          TMEM dP (dK has read dS^T: MMAs run in issue order)
-//                 Two gradient warpgroups each own half of the query columns; a third warpgroup reads dQ^T (TMEM
-//                 lane = head-dim index) and adds it to an fp32 accumulator from registers: per row one coalesced
-//                 128-byte red.global.add per warp, concurrently with the next step's softmax work. dK/dV stay
-//                 in TMEM for the whole item; an unsplit key tile writes them as bf16, a split one adds its fp32
-//                 partial into the workspace (one add per element and chunk).
-//   k_bwd_convert dQ (and the split tiles' dK/dV) from the fp32 accumulators to bf16.
-// TMEM (512 columns): S/P [0,128), dP/dS/dQ [128,256), dV [256,384), dK [384,512).
-// Per-query values folded into the MMAs: the softmax warps own a key row each and would otherwise need the lse
+// Four kernels:
+//   k_bwd_pre     (-lse / scale, -D) per row and head, D = rowsum(dO * O) in fp32 (HBM-bound).
+//   k_bwd_tc      dK and dV: key/value-stationary tensor-core kernel (below).
+//   k_bwd_dq      dQ: query-stationary tensor-core kernel (pp_attn_bwd_dq.cuh); recomputes S and dP per tile so
+//                 that every dQ row is produced by exactly one CTA (no fp32 accumulator, no reduction traffic).
+//   k_bwd_convert the fp32 dK/dV partials of split key tiles to bf16.
+// k_bwd_tc: a work item is (key tile of 128 rows, kv head, chunk of the query tiles that attend it). Seen from key
+// y the attending queries are one interval [y, e(y)) (pp_meta.cuh), so a key tile's query tiles are one contiguous
+// range; prefix key tiles (attended by every response of the group) get long ranges and are split into chunks so
+// the persistent grid stays balanced. Per step (query tile of 128 rows, one q head of the kv head), four MMAs, all
+// with N = 128 (an N = 64 MMA costs as long as an N = 128 one on this part):
+//   S^T  = K Q^T                          TMEM S
+//   dP^T = V dO^T                         TMEM dP
+//   gradient warps, phase 1: P^T = exp(S^T - lse) -> TMEM S (bf16)          -> dV may start
+//   dV  += P^T dO        (A from TMEM)    TMEM dV
+//   gradient warps, phase 2: dS^T = scale P^T (dP^T - D) -> TMEM dP (bf16)
+//   dK  += dS^T Q        (A from TMEM)    TMEM dK
+// Two gradient warpgroups each own half of the query columns of a step, and run dS(t) before P(t+1) so the next
+// step's P overlaps this step's dK. dK/dV stay in TMEM for the whole item; an unsplit key tile writes them as bf16,
+// a split one adds its fp32 partial into the workspace (one add per element and chunk).
+// TMEM (512 columns): S/P [0,128), dP/dS [128,256), dV [256,384), dK [384,512).
+// Per-query values folded into the MMAs: the gradient warps own a key row each and would otherwise need the lse
 // and D of all 128 query columns per step (a shared-memory or shuffle broadcast per element, which measured
 // several times slower than the exp itself). Instead one extra K = 16 slice is appended to the S^T and dP^T
 // products: K and V get columns (1, 1, 1, 0, ...), Q gets (-lse/scale) and dO gets (-D), each split exactly into
 // three bf16 parts (hi, mid, lo). The accumulators then hold s - lse/scale and dP - D directly, so
 // P^T = exp2(S'^T * scale * log2 e) and dS^T = P^T * dP'^T * scale need nothing but the TMEM values. The extra
-// slices cost 2 of 42 MMAs per step. They live in shared memory as 128 x 16 bf16 tiles in the no-swizzle core-matrix
-// layout; the producer warp writes the query side for each step.
-// Q/dO tiles come through a 2-stage ring.
-// Work items run kv-head-major: concurrently running CTAs share a kv head, so a group's Q/dO rows and dQ
-// accumulator rows are reused from L2 across its key tiles.
+// slices cost 2 of 34 MMAs per step. They live in shared memory as 128 x 16 bf16 tiles in the no-swizzle
+// core-matrix layout; the producer warp writes the query side for each step.
+// Q/dO tiles come through a 2-stage ring, prefetched into L2 two steps ahead.
+// Work items run kv-head-major: concurrently running CTAs share a kv head, so a group's Q/dO rows are reused from
+// L2 across its key tiles.
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include "pp_meta.cuh"
 #include "pp_ptx.cuh"
 #include "pp_attn_fwd.cuh"   // bwait, globaltimer_ns
+#include "pp_attn_bwd_dq.cuh"
 
 namespace pp {
 
-constexpr int BWD_THREADS = 448;   // 8 gradient warps, 4 dQ warps, producer, MMA
+constexpr int BWD_THREADS = 320;   // 8 gradient warps, producer, MMA
 constexpr int BWD_D = 128;
 
 struct BwdWorkspace {
     int64_t rows_pad;   // T + padding rows so tiles that stick out past T stay inside the buffers
     int64_t off_delta;  // float2 [hq][rows_pad]: (-lse_i / scale, -D_i)
-    int64_t off_dq;     // fp32 [hq][rows_pad][d]: dQ accumulator
     int64_t off_dk;     // fp32 [rows_pad][hkv][d]: dK accumulator of split key tiles
     int64_t off_dv;     // fp32 [rows_pad][hkv][d]: dV accumulator of split key tiles
     int64_t total;
@@ -64,7 +62,6 @@ inline BwdWorkspace bwd_workspace_layout(int64_t T, int hq, int hkv, int d) {
     w.rows_pad = (T + 256 + 7) & ~int64_t(7);
     int64_t o = 0;
     w.off_delta = o; o = align256(o + 8 * int64_t(hq) * w.rows_pad);
-    w.off_dq = o;    o = align256(o + 4 * int64_t(hq) * w.rows_pad * d);
     w.off_dk = o;    o = align256(o + 4 * w.rows_pad * hkv * d);
     w.off_dv = o;    o = align256(o + 4 * w.rows_pad * hkv * d);
     w.total = o;
@@ -120,13 +117,13 @@ struct BwdSmem {
     alignas(1024) uint8_t k[TILE];
     alignas(1024) uint8_t v[TILE];
     alignas(1024) uint8_t q[QSTAGES][TILE];
-    alignas(1024) uint8_t dout[QSTAGES][TILE];          // dO(t), then dS^T(t) once dV(t) has read dO(t)
+    alignas(1024) uint8_t dout[QSTAGES][TILE];
     alignas(1024) uint8_t aug_ones[AUG];                 // key side of the extra slice: (1, 1, 1, 0, ...)
     alignas(1024) uint8_t aug_q[QSTAGES][AUG];           // query side for S^T: split(-lse / scale)
     alignas(1024) uint8_t aug_do[QSTAGES][AUG];          // query side for dP^T: split(-D)
     uint64_t kv_full, kv_empty, dkv_full, dkv_free;
     uint64_t q_full[QSTAGES], q_empty[QSTAGES];
-    uint64_t s_full, dp_full, p_ready, dv_done, ds_ready, dq_full, dq_free;
+    uint64_t s_full, dp_full, p_ready, ds_ready;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -157,8 +154,6 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
 }
-__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
 // dK (scaled) or dV of the item from TMEM: bf16 rows for an unsplit tile, fp32 adds into the workspace otherwise.
 __device__ __forceinline__ void bwd_store_kv(uint32_t taddr, bool yin, bool split, float f, float *acc,
@@ -191,7 +186,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
          const void *__restrict__ meta, const float2 *__restrict__ ldg,
-         float *__restrict__ dq_acc, float *__restrict__ dk_acc, float *__restrict__ dv_acc,
+         float *__restrict__ dk_acc, float *__restrict__ dv_acc,
          __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV, int hq, int hkv, int64_t rows_pad,
          float scale, float sl2) {
     extern __shared__ uint8_t smem_raw[];
@@ -214,10 +209,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.dp_full, 1);
         mbar_init(&sm.p_ready, 256);
-        mbar_init(&sm.dv_done, 1);
         mbar_init(&sm.ds_ready, 256);
-        mbar_init(&sm.dq_full, 1);
-        mbar_init(&sm.dq_free, 128);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -233,11 +225,11 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         }
         fence_proxy_async_smem();
     }
-    if (warp == 13) {
+    if (warp == 9) {
         tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
     }
-    if (warp == 12 && lane == 0) {
+    if (warp == 8 && lane == 0) {
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
@@ -251,7 +243,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
 
     if (hd.dev_err != 0) {
         // nothing to do: the metadata builder rejected its input
-    } else if (warp == 12) {
+    } else if (warp == 8) {
         // ------------------------------------------------------------------ producer warp
         uint32_t g = 0, it_n = 0;
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
@@ -314,13 +306,12 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 }
             }
         }
-    } else if (warp == 13) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------------ MMA issuer (one thread)
         if (lane == 0) {
             constexpr uint32_t ID_SDP = idesc_bf16(128, BWD_BM, 0, 0);     // S^T, dP^T (both K-major)
             constexpr uint32_t ID_DV = idesc_bf16(128, BWD_D, 0, 1);       // dV (A TMEM, B MN-major)
             constexpr uint32_t ID_DK = idesc_bf16(128, BWD_D, 0, 1);       // dK (A TMEM, B MN-major)
-            constexpr uint32_t ID_DQ = idesc_bf16(128, BWD_BM, 1, 1);      // dQ^T (A and B MN-major)
             const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
             uint32_t g = 0, it_n = 0;
             // K-major x K-major product over d (S^T = K Q^T or dP^T = V dO^T)
@@ -335,8 +326,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 umma_ss(tmem + col, ones_desc, smem_desc(smem_u32(aug), BwdSmem::AUG_LBO, BwdSmem::AUG_SBO, 0),
                         ID_SDP, 1u);
             };
-            auto issue_dp = [&](uint32_t gg) -> bool {      // dP^T(gg), once dQ^T(gg - 1) has been read out
-                if (gg > 0 && !bwait(&sm.dq_free, (gg - 1) & 1, abort_flag)) return false;
+            auto issue_dp = [&](uint32_t gg) -> bool {      // dP^T(gg): dK(gg - 1) has read dS^T (issue order)
                 tc_fence_after();
                 issue_kk(COL_DP, sv, smem_u32(sm.dout[gg % BwdSmem::QSTAGES]), sm.aug_do[gg % BwdSmem::QSTAGES]);
                 umma_commit(&sm.dp_full);
@@ -367,68 +357,26 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     for (int kk = 0; kk < BWD_BM / 16; ++kk)
                         umma_ts(tmem + COL_DV, tmem + COL_S + 64 * (kk >> 2) + 8 * (kk & 3),
                                 smem_desc(sdo + kk * 2048, BwdSmem::CHUNK, 1024), ID_DV, (t > 0 || kk > 0));
-                    umma_commit(&sm.dv_done);
                     // S^T of the next step may overwrite P^T now (MMAs run in issue order); issue it first only if
-                    // its tile has landed, so a late load never holds up dK/dQ^T of this step
+                    // its tile has landed, so a late load never holds up dK of this step
                     bool s_next = false;
                     if (t + 1 < n && mbar_try_wait(&sm.q_full[(g + 1) % BwdSmem::QSTAGES], ((g + 1) / BwdSmem::QSTAGES) & 1)) {
                         if (!issue_s(g + 1)) goto done;
                         s_next = true;
                     }
-                    // dK += dS^T Q and dQ^T = K^T dS^T once dS^T is in shared memory
+                    // dK += dS^T Q once dS^T is in TMEM
                     if (!bwait(&sm.ds_ready, g & 1, abort_flag)) goto done;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < BWD_BM / 16; ++kk)
                         umma_ts(tmem + COL_DK, tmem + COL_DP + 64 * (kk >> 2) + 8 * (kk & 3),
                                 smem_desc(sq + kk * 2048, BwdSmem::CHUNK, 1024), ID_DK, (t > 0 || kk > 0));
-#pragma unroll
-                    for (int kk = 0; kk < 128 / 16; ++kk)
-                        umma_ss(tmem + COL_DP, smem_desc(sk + kk * 2048, BwdSmem::CHUNK, 1024),
-                                smem_desc(sdo + kk * 2048, BwdSmem::CHUNK, 1024), ID_DQ, kk > 0);
-                    umma_commit(&sm.dq_full);
                     umma_commit(&sm.q_empty[st]);
                     if (t + 1 < n && !s_next && !issue_s(g + 1)) goto done;
                     if (t + 1 < n && !issue_dp(g + 1)) goto done;
                 }
                 umma_commit(&sm.dkv_full);
                 umma_commit(&sm.kv_empty);
-            }
-        }
-    } else if (warp >= 8) {
-        // ------------------------------------------------------------------ dQ warpgroup (warps 8-11)
-        // dQ^T (TMEM lane = head-dim index) is read as soon as its MMA completes and added to the fp32
-        // accumulator: per query row one coalesced 128-byte red.global.add per warp. Running these adds on their own
-        // warps keeps the reduction traffic off the gradient warps' step.
-        const int wl = warp & 3;
-        const int dcol = wl * 32 + lane;
-        const uint32_t lane_off = uint32_t(wl * 32) << 16;
-        uint32_t g = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-            const BwdItem w = bwd_decode(meta, hd, item);
-            const int n = (w.qb - w.qa) * r;
-            for (int t = 0; t < n; ++t, ++g) {
-                const int h = w.kh * r + t % r;
-                const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
-                if (!bwait(&sm.dq_full, g & 1, abort_flag)) goto done;
-                tc_fence_after();
-                uint32_t a0[32], a1[32], a2[32], a3[32];
-                tmem_ld32(tmem + lane_off + COL_DP, a0);
-                tmem_ld32(tmem + lane_off + COL_DP + 32, a1);
-                tmem_ld32(tmem + lane_off + COL_DP + 64, a2);
-                tmem_ld32(tmem + lane_off + COL_DP + 96, a3);
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(&sm.dq_free);
-                float *gdst = dq_acc + (int64_t(h) * rows_pad + x0) * BWD_D + dcol;
-#pragma unroll
-                for (int c = 0; c < 32; ++c) red_add_f32(gdst + c * BWD_D, __uint_as_float(a0[c]));
-#pragma unroll
-                for (int c = 0; c < 32; ++c) red_add_f32(gdst + (32 + c) * BWD_D, __uint_as_float(a1[c]));
-#pragma unroll
-                for (int c = 0; c < 32; ++c) red_add_f32(gdst + (64 + c) * BWD_D, __uint_as_float(a2[c]));
-#pragma unroll
-                for (int c = 0; c < 32; ++c) red_add_f32(gdst + (96 + c) * BWD_D, __uint_as_float(a3[c]));
             }
         }
     } else {
@@ -494,10 +442,8 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             };
             if (n > 0 && !phase_p(g, 0)) goto done;
             for (int t = 0; t < n; ++t, ++g) {
-                const int st = g % BwdSmem::QSTAGES;
-                // phase 2: dS^T = scale P^T dP'^T (dP' = dP - D already) -> TMEM and the dO buffer (dV has read it)
+                // phase 2: dS^T = scale P^T dP'^T (dP' = dP - D already) -> TMEM dP columns this warpgroup has read
                 if (!bwait(&sm.dp_full, g & 1, abort_flag)) goto done;
-                if (!bwait(&sm.dv_done, g & 1, abort_flag)) goto done;
                 tc_fence_after();
                 {
                     uint32_t pr[64];
@@ -509,30 +455,21 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
 #pragma unroll
                         for (int e = 0; e < 32; ++e) { pr[e] = a0[e]; pr[32 + e] = a1[e]; }
                     }
-                    uint32_t dd[32];
+                    uint32_t t0[16], t1[16];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const uint32_t p = pk[e];
-                        dd[e] = pack_bf16x2(bf16lo(p) * __uint_as_float(pr[2 * e]) * scale,
-                                            bf16hi(p) * __uint_as_float(pr[2 * e + 1]) * scale);
+                        const uint32_t dd = pack_bf16x2(bf16lo(p) * __uint_as_float(pr[2 * e]) * scale,
+                                                        bf16hi(p) * __uint_as_float(pr[2 * e + 1]) * scale);
+                        if (e < 16) t0[e] = dd; else t1[e - 16] = dd;
                     }
-                    uint32_t t0[16], t1[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) { t0[e] = dd[e]; t1[e] = dd[16 + e]; }
                     tmem_st16(tmem + lane_off + COL_DP + cb, t0);
                     tmem_st16(tmem + lane_off + COL_DP + cb + 16, t1);
-                    // dS^T row jr, queries [cb, cb+64) = 64-column chunk wx of the swizzled [key][query] tile
-                    uint8_t *dsrow = sm.dout[st] + wx * BwdSmem::CHUNK + jr * 128;
-#pragma unroll
-                    for (int piece = 0; piece < 8; ++piece)
-                        *reinterpret_cast<uint4 *>(dsrow + ((piece ^ (jr & 7)) << 4)) =
-                            make_uint4(dd[4 * piece], dd[4 * piece + 1], dd[4 * piece + 2], dd[4 * piece + 3]);
                 }
                 tmem_wait_st();
-                fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(&sm.ds_ready);
-                // next step's phase 1 while this step's dK and dQ^T run
+                // next step's phase 1 while this step's dK runs
                 if (t + 1 < n && !phase_p(g + 1, t + 1)) goto done;
             }
             // item epilogue: warpgroup 0 writes dK (dS^T carried the scale), warpgroup 1 writes dV
@@ -549,34 +486,20 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
 done:
     tc_fence_before();
     __syncthreads();
-    if (warp == 13) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
 }
 
 // ------------------------------------------------------------------------------------------------- convert
-// dQ[i][h][:] = bf16(dq_acc[h][i][:]); dK/dV rows of split key tiles = bf16(accumulators).
-__global__ void k_bwd_convert(const void *__restrict__ meta, const float *__restrict__ dq_acc,
-                              const float *__restrict__ dk_acc, const float *__restrict__ dv_acc,
-                              __nv_bfloat16 *__restrict__ dQ, __nv_bfloat16 *__restrict__ dK,
-                              __nv_bfloat16 *__restrict__ dV, int hq, int hkv, int64_t rows_pad) {
+// dK/dV rows of split key tiles = bf16(fp32 accumulators).
+__global__ void k_bwd_convert(const void *__restrict__ meta, const float *__restrict__ dk_acc,
+                              const float *__restrict__ dv_acc, __nv_bfloat16 *__restrict__ dK,
+                              __nv_bfloat16 *__restrict__ dV, int hkv) {
     const MetaHeader hd = *meta_ptr<MetaHeader>(meta, 0);
-    if (hd.dev_err) return;
-    const int64_t T = hd.T;
-    const int64_t nvec_q = T * hq * (BWD_D / 4);
+    if (hd.dev_err || hd.n_split == 0) return;
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < nvec_q; e += stride) {
-        const int64_t row = e / (int64_t(hq) * (BWD_D / 4));
-        const int64_t rem = e % (int64_t(hq) * (BWD_D / 4));
-        const int h = static_cast<int>(rem / (BWD_D / 4)), c = static_cast<int>(rem % (BWD_D / 4));
-        const float4 a = reinterpret_cast<const float4 *>(dq_acc + (int64_t(h) * rows_pad + row) * BWD_D)[c];
-        __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
-        uint2 u;
-        u.x = *reinterpret_cast<uint32_t *>(&lo);
-        u.y = *reinterpret_cast<uint32_t *>(&hi);
-        reinterpret_cast<uint2 *>(dQ + (row * hq + h) * BWD_D)[c] = u;
-    }
     const KTile *kts = meta_ptr<KTile>(meta, hd.off_kt);
     const int64_t per_tile = int64_t(128) * hkv * (BWD_D / 4);
     for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < int64_t(hd.n_kt) * per_tile; e += stride) {
@@ -609,7 +532,6 @@ inline pp_status launch_bwd(const void *q, const void *k, const void *v, const v
     const BwdWorkspace L = bwd_workspace_layout(T, hq, hkv, d);
     char *ws = static_cast<char *>(workspace);
     float2 *ldg = reinterpret_cast<float2 *>(ws + L.off_delta);
-    float *dq_acc = reinterpret_cast<float *>(ws + L.off_dq);
     float *dk_acc = reinterpret_cast<float *>(ws + L.off_dk);
     float *dv_acc = reinterpret_cast<float *>(ws + L.off_dv);
     const void *ptrs[8] = {q, k, v, o, dout, dq, dk, dv};
@@ -622,7 +544,7 @@ inline pp_status launch_bwd(const void *q, const void *k, const void *v, const v
     if ((st = make_map(&mv, v, T, hkv, d, BWD_BN)) != PP_OK) return st;
     if ((st = make_map(&mdo, dout, T, hq, d, BWD_BM)) != PP_OK) return st;
     cudaError_t e;
-    if ((e = cudaMemsetAsync(ws + L.off_dq, 0, L.total - L.off_dq, s)) != cudaSuccess)
+    if ((e = cudaMemsetAsync(ws + L.off_dk, 0, L.total - L.off_dk, s)) != cudaSuccess)
         return fail(PP_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
     k_bwd_pre<<<sm_count * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(o),
                                            static_cast<const __nv_bfloat16 *>(dout), lse, ldg, T, L.rows_pad, hq,
@@ -631,13 +553,18 @@ inline pp_status launch_bwd(const void *q, const void *k, const void *v, const v
     const size_t smem = sizeof(BwdSmem) + 1024;
     if ((e = cudaFuncSetAttribute(k_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem))) != cudaSuccess)
         return fail(PP_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    k_bwd_tc<<<sm_count, BWD_THREADS, smem, s>>>(mq, mk, mv, mdo, meta, ldg, dq_acc, dk_acc, dv_acc,
+    k_bwd_tc<<<sm_count, BWD_THREADS, smem, s>>>(mq, mk, mv, mdo, meta, ldg, dk_acc, dv_acc,
                                                  static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv),
                                                  hq, hkv, L.rows_pad, scale, scale * 1.4426950408889634f);
     if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_tc: %s", cudaGetErrorString(e));
-    k_bwd_convert<<<sm_count * 8, 256, 0, s>>>(meta, dq_acc, dk_acc, dv_acc, static_cast<__nv_bfloat16 *>(dq),
-                                               static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv),
-                                               hq, hkv, L.rows_pad);
+    const size_t smem_dq = sizeof(DqSmem) + 1024;
+    if ((e = cudaFuncSetAttribute(k_bwd_dq, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_dq))) != cudaSuccess)
+        return fail(PP_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    k_bwd_dq<<<sm_count, DQ_THREADS, smem_dq, s>>>(mq, mk, mv, mdo, meta, ldg, static_cast<__nv_bfloat16 *>(dq),
+                                                   hq, hkv, L.rows_pad, scale, scale * 1.4426950408889634f);
+    if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_dq: %s", cudaGetErrorString(e));
+    k_bwd_convert<<<sm_count * 8, 256, 0, s>>>(meta, dk_acc, dv_acc, static_cast<__nv_bfloat16 *>(dk),
+                                               static_cast<__nv_bfloat16 *>(dv), hkv);
     if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_convert: %s", cudaGetErrorString(e));
     return PP_OK;
 }

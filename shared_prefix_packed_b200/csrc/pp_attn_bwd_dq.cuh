@@ -1,0 +1,303 @@
+// pp_attn_bwd_dq.cuh - the dQ half of the backward: query-stationary tcgen05 kernel, no atomics.
+//
+// dQ_i = scale sum_j dS_ij k_j with dS_ij = p_ij (dO_i . v_j - D_i) and p_ij = exp(s_ij - lse_i), over the allowed
+// keys j of query row i (pp_meta.cuh). A work item is (query tile of 128 rows, one q head); it walks the same key
+// tiles as the forward pass (the two runs of the QTile) and owns its 128 dQ rows, so dQ is written once, in bf16,
+// with no reduction across CTAs. Per key tile:
+//   S  = Q K^T      (M = 128 queries, N = 128 keys)          TMEM S
+//   dP = dO V^T                                               TMEM dP
+//   gradient warps: P = exp2(S * scale log2 e - lse log2 e); dS = scale P (dP - D)  -> TMEM dP (bf16)
+//   dQ += dS K      (A from TMEM, B = the K tile read N-major) TMEM dQ
+// Here the thread owns a query row, so lse and D are per-thread constants: no per-column broadcast is needed.
+// Recomputing S and dP costs 16 of the 24 MMAs per tile; in exchange dQ needs no fp32 accumulator and no
+// reduction traffic (which measured about 6 TB/s at best on L2-resident data, below what the key-side kernel
+// would otherwise need).
+// Warp roles (320 threads): warps 0-3 and 4-7 take key columns [0,64) and [64,128) of every tile (each its own
+// half of S and dP, P kept packed in registers, its dS written into dP columns it has itself read); warp 8 is the
+// TMA producer (Q and dO once per item, K and V through a 2-stage ring); warp 9 allocates TMEM and issues MMAs.
+// TMEM: S [0,128), dP/dS [128,256), dQ [256,384).
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include "pp_meta.cuh"
+#include "pp_ptx.cuh"
+#include "pp_attn_fwd.cuh"   // bwait, FwdItem helpers
+
+namespace pp {
+
+constexpr int DQ_THREADS = 320;
+constexpr int DQ_STAGES = 2;
+
+struct DqSmem {
+    static constexpr int TILE = 128 * 128 * 2;
+    static constexpr int CHUNK = 128 * 64 * 2;
+    alignas(1024) uint8_t q[TILE];
+    alignas(1024) uint8_t dout[TILE];
+    alignas(1024) uint8_t k[DQ_STAGES][TILE];
+    alignas(1024) uint8_t v[DQ_STAGES][TILE];
+    uint64_t qd_full, qd_empty, dq_full, dq_free;
+    uint64_t kv_full[DQ_STAGES], kv_empty[DQ_STAGES];
+    uint64_t s_full, s_free, dp_full, ds_ready;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+struct DqItem {
+    QTile t;
+    int h, kh;
+};
+
+__device__ __forceinline__ DqItem dq_decode(const void *meta, const MetaHeader &hd, int item, int hq, int hkv) {
+    const int32_t *qorder = meta_ptr<int32_t>(meta, hd.off_qorder);
+    DqItem it;
+    it.t = meta_ptr<QTile>(meta, hd.off_qt)[qorder[item / hq]];
+    it.h = item % hq;
+    it.kh = it.h / (hq / hkv);
+    return it;
+}
+
+__global__ void __launch_bounds__(DQ_THREADS, 1)
+k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+         const void *__restrict__ meta, const float2 *__restrict__ ldg, __nv_bfloat16 *__restrict__ dQ, int hq,
+         int hkv, int64_t rows_pad, float scale, float sl2) {
+    extern __shared__ uint8_t smem_raw[];
+    DqSmem &sm = *reinterpret_cast<DqSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const MetaHeader hd = *meta_ptr<MetaHeader>(meta, 0);
+    const int n_items = hd.n_qt * hq;
+    volatile int *abort_flag = &sm.abort_flag;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.qd_full, 1);
+        mbar_init(&sm.qd_empty, 1);
+        mbar_init(&sm.dq_full, 1);
+        mbar_init(&sm.dq_free, 256);
+        for (int s = 0; s < DQ_STAGES; ++s) {
+            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.kv_empty[s], 1);
+        }
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.s_free, 256);
+        mbar_init(&sm.dp_full, 1);
+        mbar_init(&sm.ds_ready, 256);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmdO);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 256;
+
+    if (hd.dev_err != 0) {
+        // nothing to do: the metadata builder rejected its input
+    } else if (warp == 8) {
+        // ------------------------------------------------------------------ TMA producer (one thread)
+        if (lane == 0) {
+            uint32_t kv_it = 0, it_n = 0;
+            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+                const DqItem w = dq_decode(meta, hd, item, hq, hkv);
+                const int n = qtile_nkv(w.t);
+                if (!bwait(&sm.qd_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
+                mbar_arrive_expect_tx(&sm.qd_full, 2 * DqSmem::TILE);
+                for (int c = 0; c < 2; ++c) {
+                    tma_load_3d(sm.q + c * DqSmem::CHUNK, &tmQ, c * 64, w.h, w.t.row0, &sm.qd_full);
+                    tma_load_3d(sm.dout + c * DqSmem::CHUNK, &tmdO, c * 64, w.h, w.t.row0, &sm.qd_full);
+                }
+                for (int j = 0; j < n; ++j, ++kv_it) {
+                    const int y0 = w.t.gstart + qtile_kv(w.t, j) * FWD_BN;
+                    const int s = kv_it % DQ_STAGES;
+                    if (!bwait(&sm.kv_empty[s], ((kv_it / DQ_STAGES) & 1) ^ 1, abort_flag)) goto done;
+                    mbar_arrive_expect_tx(&sm.kv_full[s], 2 * DqSmem::TILE);
+                    for (int c = 0; c < 2; ++c) {
+                        tma_load_3d(sm.k[s] + c * DqSmem::CHUNK, &tmK, c * 64, w.kh, y0, &sm.kv_full[s]);
+                        tma_load_3d(sm.v[s] + c * DqSmem::CHUNK, &tmV, c * 64, w.kh, y0, &sm.kv_full[s]);
+                    }
+                }
+            }
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------------------------ MMA issuer (one thread)
+        if (lane == 0) {
+            constexpr uint32_t ID_SP = idesc_bf16(128, 128, 0, 0);         // S, dP: K-major x K-major over d
+            constexpr uint32_t ID_DQ = idesc_bf16(128, 128, 0, 1);         // dQ: A = dS (TMEM), B = K N-major
+            const uint32_t sq = smem_u32(sm.q), sdo = smem_u32(sm.dout);
+            uint32_t kv_it = 0, it_n = 0, g = 0;                           // g: global key-tile step counter
+            auto issue_kk = [&](uint32_t col, uint32_t a, uint32_t b) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * DqSmem::CHUNK + (kk & 3) * 32;
+                    umma_ss(tmem + col, smem_desc(a + off, 16, 1024), smem_desc(b + off, 16, 1024), ID_SP, kk > 0);
+                }
+            };
+            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+                const DqItem w = dq_decode(meta, hd, item, hq, hkv);
+                const int n = qtile_nkv(w.t);
+                if (!bwait(&sm.qd_full, it_n & 1, abort_flag)) goto done;
+                // S and dP of the first key tile (the gradient warps have released both regions: s_free and
+                // ds_ready of the previous step were waited for before that step's dQ MMA)
+                {
+                    const int s0 = kv_it % DQ_STAGES;
+                    if (!bwait(&sm.kv_full[s0], (kv_it / DQ_STAGES) & 1, abort_flag)) goto done;
+                    if (g > 0 && !bwait(&sm.s_free, (g - 1) & 1, abort_flag)) goto done;
+                    tc_fence_after();
+                    issue_kk(COL_S, sq, smem_u32(sm.k[s0]));
+                    umma_commit(&sm.s_full);
+                    issue_kk(COL_DP, sdo, smem_u32(sm.v[s0]));
+                    umma_commit(&sm.dp_full);
+                }
+                if (!bwait(&sm.dq_free, (it_n & 1) ^ 1, abort_flag)) goto done;
+                for (int j = 0; j < n; ++j, ++kv_it, ++g) {
+                    const int st = kv_it % DQ_STAGES, st1 = (kv_it + 1) % DQ_STAGES;
+                    // next tile's S as soon as the gradient warps have read this tile's S
+                    if (j + 1 < n) {
+                        if (!bwait(&sm.kv_full[st1], ((kv_it + 1) / DQ_STAGES) & 1, abort_flag)) goto done;
+                        if (!bwait(&sm.s_free, g & 1, abort_flag)) goto done;
+                        tc_fence_after();
+                        issue_kk(COL_S, sq, smem_u32(sm.k[st1]));
+                        umma_commit(&sm.s_full);
+                    }
+                    // dQ += dS K once dS is in TMEM
+                    if (!bwait(&sm.ds_ready, g & 1, abort_flag)) goto done;
+                    tc_fence_after();
+                    const uint32_t sk = smem_u32(sm.k[st]);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_ts(tmem + COL_DQ, tmem + COL_DP + 64 * (kk >> 2) + 8 * (kk & 3),
+                                smem_desc(sk + kk * 2048, DqSmem::CHUNK, 1024), ID_DQ, (j > 0 || kk > 0));
+                    umma_commit(&sm.kv_empty[st]);
+                    // next tile's dP (dQ above has read dS out of the dP region: MMAs run in issue order)
+                    if (j + 1 < n) {
+                        issue_kk(COL_DP, sdo, smem_u32(sm.v[st1]));
+                        umma_commit(&sm.dp_full);
+                    }
+                }
+                umma_commit(&sm.dq_full);
+                umma_commit(&sm.qd_empty);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------ gradient warpgroups (warps 0-7)
+        const int wx = warp >> 2, wl = warp & 3;
+        const int rt = wl * 32 + lane;                                 // query row within the tile = TMEM lane
+        const uint32_t lane_off = uint32_t(wl * 32) << 16;
+        const int cb = 64 * wx;                                        // this warpgroup's key columns
+        uint32_t g = 0, it_n = 0;
+        const int32_t *seg_start = meta_ptr<int32_t>(meta, hd.off_seg_start);
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+            const DqItem w = dq_decode(meta, hd, item, hq, hkv);
+            const int n = qtile_nkv(w.t);
+            const int row = w.t.row0 + rt;
+            const bool in_group = row < w.t.gstart + w.t.glen;
+            const int s0 = in_group ? seg_start[row] : 0;
+            const int pfx_end = w.t.gstart + w.t.plen;
+            const int x0 = w.t.row0 - w.t.gstart;
+            const float2 lv = ldg[int64_t(w.h) * rows_pad + row];     // (-lse / scale, -D); padded past T
+            const float c0 = lv.x * sl2;                               // - lse * log2 e
+            for (int j = 0; j < n; ++j, ++g) {
+                const int yt = qtile_kv(w.t, j) * FWD_BN;
+                const int y0 = w.t.gstart + yt + cb;                   // first key of this warpgroup's columns
+                const int cls = tile_class(x0, FWD_BM, yt, FWD_BN, w.t.glen, w.t.plen, w.t.s0first, w.t.s0last);
+                const int lim_diag = in_group ? row - y0 : -1;         // allowed: c <= lim_diag and
+                const int lim_pfx = pfx_end - y0;                      //   (c < lim_pfx or c >= lim_seg)
+                const int lim_seg = s0 - y0;
+                // P = exp2(S scale log2 e - lse log2 e), packed bf16, kept for the dS step
+                if (!bwait(&sm.s_full, g & 1, abort_flag)) goto done;
+                tc_fence_after();
+                uint32_t pk[32];
+                {
+                    uint32_t a0[32], a1[32];
+                    tmem_ld32(tmem + lane_off + COL_S + cb, a0);
+                    tmem_ld32(tmem + lane_off + COL_S + cb + 32, a1);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive(&sm.s_free);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int c = 2 * e;
+                        const uint32_t u0 = c < 32 ? a0[c] : a1[c - 32];
+                        const uint32_t u1 = c + 1 < 32 ? a0[c + 1] : a1[c - 31];
+                        float p0 = ex2_approx(fmaf(__uint_as_float(u0), sl2, c0));
+                        float p1 = ex2_approx(fmaf(__uint_as_float(u1), sl2, c0));
+                        if (cls != TILE_FULL) {
+                            if (!(c <= lim_diag && (c < lim_pfx || c >= lim_seg))) p0 = 0.f;
+                            if (!(c + 1 <= lim_diag && (c + 1 < lim_pfx || c + 1 >= lim_seg))) p1 = 0.f;
+                        }
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                }
+                // dS = scale P (dP - D) -> TMEM dP columns [cb, cb+32) (already read)
+                if (!bwait(&sm.dp_full, g & 1, abort_flag)) goto done;
+                tc_fence_after();
+                {
+                    uint32_t a0[32], a1[32];
+                    tmem_ld32(tmem + lane_off + COL_DP + cb, a0);
+                    tmem_ld32(tmem + lane_off + COL_DP + cb + 32, a1);
+                    tmem_wait_ld();
+                    uint32_t d0[16], d1[16];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int c = 2 * e;
+                        const uint32_t u0 = c < 32 ? a0[c] : a1[c - 32];
+                        const uint32_t u1 = c + 1 < 32 ? a0[c + 1] : a1[c - 31];
+                        const uint32_t p = pk[e];
+                        const uint32_t dd = pack_bf16x2(bf16lo(p) * (__uint_as_float(u0) + lv.y) * scale,
+                                                        bf16hi(p) * (__uint_as_float(u1) + lv.y) * scale);
+                        if (e < 16) d0[e] = dd; else d1[e - 16] = dd;
+                    }
+                    tmem_st16(tmem + lane_off + COL_DP + cb, d0);
+                    tmem_st16(tmem + lane_off + COL_DP + cb + 16, d1);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.ds_ready);
+            }
+            // epilogue: dQ rows (dS carried the scale); warpgroup x writes head dims [64x, 64x+64)
+            if (!bwait(&sm.dq_full, it_n & 1, abort_flag)) goto done;
+            tc_fence_after();
+            {
+                uint32_t a0[32], a1[32];
+                tmem_ld32(tmem + lane_off + COL_DQ + cb, a0);
+                tmem_ld32(tmem + lane_off + COL_DQ + cb + 32, a1);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&sm.dq_free);
+                if (in_group) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(dQ + (int64_t(row) * hq + w.h) * 128 + cb);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(pack_bf16x2(__uint_as_float(a0[8 * e]), __uint_as_float(a0[8 * e + 1])),
+                                            pack_bf16x2(__uint_as_float(a0[8 * e + 2]), __uint_as_float(a0[8 * e + 3])),
+                                            pack_bf16x2(__uint_as_float(a0[8 * e + 4]), __uint_as_float(a0[8 * e + 5])),
+                                            pack_bf16x2(__uint_as_float(a0[8 * e + 6]), __uint_as_float(a0[8 * e + 7])));
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[4 + e] = make_uint4(pack_bf16x2(__uint_as_float(a1[8 * e]), __uint_as_float(a1[8 * e + 1])),
+                                                pack_bf16x2(__uint_as_float(a1[8 * e + 2]), __uint_as_float(a1[8 * e + 3])),
+                                                pack_bf16x2(__uint_as_float(a1[8 * e + 4]), __uint_as_float(a1[8 * e + 5])),
+                                                pack_bf16x2(__uint_as_float(a1[8 * e + 6]), __uint_as_float(a1[8 * e + 7])));
+                }
+            }
+        }
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace pp
