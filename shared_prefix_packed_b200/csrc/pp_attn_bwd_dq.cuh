@@ -15,7 +15,9 @@
 // Warp roles (320 threads): warps 0-3 and 4-7 take key columns [0,64) and [64,128) of every tile (each its own
 // half of S and dP, P kept packed in registers, its dS written into dP columns it has itself read); warp 8 is the
 // TMA producer (Q and dO once per item, K and V through a 2-stage ring); warp 9 allocates TMEM and issues MMAs.
-// TMEM: S [0,128), dP/dS [128,256), dQ [256,384).
+// TMEM: S [0,128), dP/dS double-buffered [128,256) and [256,384), dQ [384,512). The second dP buffer lets dP of
+// the next key tile run while dS of this one is still being formed, so the gradient warps go from P(j+1) straight
+// to dS(j+1) without waiting on dQ(j).
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -37,7 +39,7 @@ struct DqSmem {
     alignas(1024) uint8_t v[DQ_STAGES][TILE];
     uint64_t qd_full, qd_empty, dq_full, dq_free;
     uint64_t kv_full[DQ_STAGES], kv_empty[DQ_STAGES];
-    uint64_t s_full, s_free, dp_full, ds_ready;
+    uint64_t s_full, s_free, dp_full[2], ds_ready;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -79,7 +81,8 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         }
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.s_free, 256);
-        mbar_init(&sm.dp_full, 1);
+        mbar_init(&sm.dp_full[0], 1);
+        mbar_init(&sm.dp_full[1], 1);
         mbar_init(&sm.ds_ready, 256);
         sm.abort_flag = 0;
         fence_mbar_init();
@@ -98,7 +101,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 256;
+    constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 384;   // dP buffer b at COL_DP + 128 b
 
     if (hd.dev_err != 0) {
         // nothing to do: the metadata builder rejected its input
@@ -145,8 +148,8 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 const DqItem w = dq_decode(meta, hd, item, hq, hkv);
                 const int n = qtile_nkv(w.t);
                 if (!bwait(&sm.qd_full, it_n & 1, abort_flag)) goto done;
-                // S and dP of the first key tile (the gradient warps have released both regions: s_free and
-                // ds_ready of the previous step were waited for before that step's dQ MMA)
+                // S and dP of the first key tile. Buffer reuse is safe by issue order: dP buffer g%2 last held
+                // dS(g-2), read by dQ(g-2); the S region was released by s_free(g-1).
                 {
                     const int s0 = kv_it % DQ_STAGES;
                     if (!bwait(&sm.kv_full[s0], (kv_it / DQ_STAGES) & 1, abort_flag)) goto done;
@@ -154,15 +157,19 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     tc_fence_after();
                     issue_kk(COL_S, sq, smem_u32(sm.k[s0]));
                     umma_commit(&sm.s_full);
-                    issue_kk(COL_DP, sdo, smem_u32(sm.v[s0]));
-                    umma_commit(&sm.dp_full);
+                    issue_kk(COL_DP + 128 * (g & 1), sdo, smem_u32(sm.v[s0]));
+                    umma_commit(&sm.dp_full[g & 1]);
                 }
                 if (!bwait(&sm.dq_free, (it_n & 1) ^ 1, abort_flag)) goto done;
                 for (int j = 0; j < n; ++j, ++kv_it, ++g) {
                     const int st = kv_it % DQ_STAGES, st1 = (kv_it + 1) % DQ_STAGES;
-                    // next tile's S as soon as the gradient warps have read this tile's S
                     if (j + 1 < n) {
+                        // next tile's dP into the other buffer (its dS(g-1) was read by dQ(g-1), issued earlier)
                         if (!bwait(&sm.kv_full[st1], ((kv_it + 1) / DQ_STAGES) & 1, abort_flag)) goto done;
+                        tc_fence_after();
+                        issue_kk(COL_DP + 128 * ((g + 1) & 1), sdo, smem_u32(sm.v[st1]));
+                        umma_commit(&sm.dp_full[(g + 1) & 1]);
+                        // next tile's S as soon as the gradient warps have read this tile's S
                         if (!bwait(&sm.s_free, g & 1, abort_flag)) goto done;
                         tc_fence_after();
                         issue_kk(COL_S, sq, smem_u32(sm.k[st1]));
@@ -172,16 +179,12 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     if (!bwait(&sm.ds_ready, g & 1, abort_flag)) goto done;
                     tc_fence_after();
                     const uint32_t sk = smem_u32(sm.k[st]);
+                    const uint32_t cds = COL_DP + 128 * (g & 1);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_ts(tmem + COL_DQ, tmem + COL_DP + 64 * (kk >> 2) + 8 * (kk & 3),
+                        umma_ts(tmem + COL_DQ, tmem + cds + 64 * (kk >> 2) + 8 * (kk & 3),
                                 smem_desc(sk + kk * 2048, DqSmem::CHUNK, 1024), ID_DQ, (j > 0 || kk > 0));
                     umma_commit(&sm.kv_empty[st]);
-                    // next tile's dP (dQ above has read dS out of the dP region: MMAs run in issue order)
-                    if (j + 1 < n) {
-                        issue_kk(COL_DP, sdo, smem_u32(sm.v[st1]));
-                        umma_commit(&sm.dp_full);
-                    }
                 }
                 umma_commit(&sm.dq_full);
                 umma_commit(&sm.qd_empty);
@@ -237,13 +240,14 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         pk[e] = pack_bf16x2(p0, p1);
                     }
                 }
-                // dS = scale P (dP - D) -> TMEM dP columns [cb, cb+32) (already read)
-                if (!bwait(&sm.dp_full, g & 1, abort_flag)) goto done;
+                // dS = scale P (dP - D) -> this step's dP buffer, columns [cb, cb+32) (already read)
+                const uint32_t cdp = COL_DP + 128 * (g & 1);
+                if (!bwait(&sm.dp_full[g & 1], (g >> 1) & 1, abort_flag)) goto done;
                 tc_fence_after();
                 {
                     uint32_t a0[32], a1[32];
-                    tmem_ld32(tmem + lane_off + COL_DP + cb, a0);
-                    tmem_ld32(tmem + lane_off + COL_DP + cb + 32, a1);
+                    tmem_ld32(tmem + lane_off + cdp + cb, a0);
+                    tmem_ld32(tmem + lane_off + cdp + cb + 32, a1);
                     tmem_wait_ld();
                     uint32_t d0[16], d1[16];
 #pragma unroll
@@ -256,8 +260,8 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                                                         bf16hi(p) * (__uint_as_float(u1) + lv.y) * scale);
                         if (e < 16) d0[e] = dd; else d1[e - 16] = dd;
                     }
-                    tmem_st16(tmem + lane_off + COL_DP + cb, d0);
-                    tmem_st16(tmem + lane_off + COL_DP + cb + 16, d1);
+                    tmem_st16(tmem + lane_off + cdp + cb, d0);
+                    tmem_st16(tmem + lane_off + cdp + cb + 16, d1);
                     tmem_wait_st();
                 }
                 tc_fence_before();
