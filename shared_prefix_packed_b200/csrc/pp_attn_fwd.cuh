@@ -44,8 +44,8 @@ __device__ __forceinline__ bool bwait(uint64_t *bar, uint32_t parity, volatile i
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63) == 0) {
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+        if ((it & 7) == 0) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > WAIT_TIMEOUT_NS) {
                 *abort_flag = 1;
