@@ -12,9 +12,10 @@
 // Recomputing S and dP costs 16 of the 24 MMAs per tile; in exchange dQ needs no fp32 accumulator and no
 // reduction traffic (which measured about 6 TB/s at best on L2-resident data, below what the key-side kernel
 // would otherwise need).
-// Warp roles (320 threads): warps 0-3 and 4-7 take key columns [0,64) and [64,128) of every tile (each its own
-// half of S and dP, P kept packed in registers, its dS written into dP columns it has itself read); warp 8 is the
-// TMA producer (Q and dO once per item, K and V through a 2-stage ring); warp 9 allocates TMEM and issues MMAs.
+// Warp roles (576 threads): warps 0-15 form four gradient warpgroups, each taking 32 key columns of every tile
+// (its own slice of S and dP, P kept packed in registers, its dS written into dP columns it has itself read);
+// warp 16 is the TMA producer (Q and dO once per item, K and V through a 2-stage ring); warp 17 allocates TMEM and
+// issues MMAs.
 // TMEM: S [0,128), dP/dS double-buffered [128,256) and [256,384), dQ [384,512). The second dP buffer lets dP of
 // the next key tile run while dS of this one is still being formed, so the gradient warps go from P(j+1) straight
 // to dS(j+1) without waiting on dQ(j).
@@ -27,8 +28,9 @@
 
 namespace pp {
 
-constexpr int DQ_THREADS = 320;
+constexpr int DQ_THREADS = 576;      // 16 gradient warps, producer, MMA
 constexpr int DQ_STAGES = 2;
+constexpr int DQ_GRAD = 512;          // gradient threads (4 warpgroups x 32 key columns)
 
 struct DqSmem {
     static constexpr int TILE = 128 * 128 * 2;
@@ -74,24 +76,24 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         mbar_init(&sm.qd_full, 1);
         mbar_init(&sm.qd_empty, 1);
         mbar_init(&sm.dq_full, 1);
-        mbar_init(&sm.dq_free, 256);
+        mbar_init(&sm.dq_free, DQ_GRAD);
         for (int s = 0; s < DQ_STAGES; ++s) {
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
         }
         mbar_init(&sm.s_full, 1);
-        mbar_init(&sm.s_free, 256);
+        mbar_init(&sm.s_free, DQ_GRAD);
         mbar_init(&sm.dp_full[0], 1);
         mbar_init(&sm.dp_full[1], 1);
-        mbar_init(&sm.ds_ready, 256);
+        mbar_init(&sm.ds_ready, DQ_GRAD);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 9) {
+    if (warp == 17) {
         tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == 16 && lane == 0) {
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
@@ -105,7 +107,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
 
     if (hd.dev_err != 0) {
         // nothing to do: the metadata builder rejected its input
-    } else if (warp == 8) {
+    } else if (warp == 16) {
         // ------------------------------------------------------------------ TMA producer (one thread)
         if (lane == 0) {
             uint32_t kv_it = 0, it_n = 0;
@@ -130,7 +132,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 }
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == 17) {
         // ------------------------------------------------------------------ MMA issuer (one thread)
         if (lane == 0) {
             constexpr uint32_t ID_SP = idesc_bf16(128, 128, 0, 0);         // S, dP: K-major x K-major over d
@@ -182,7 +184,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     const uint32_t cds = COL_DP + 128 * (g & 1);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_ts(tmem + COL_DQ, tmem + cds + 64 * (kk >> 2) + 8 * (kk & 3),
+                        umma_ts(tmem + COL_DQ, tmem + cds + 32 * (kk >> 1) + 8 * (kk & 1),
                                 smem_desc(sk + kk * 2048, DqSmem::CHUNK, 1024), ID_DQ, (j > 0 || kk > 0));
                     umma_commit(&sm.kv_empty[st]);
                 }
@@ -191,11 +193,13 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             }
         }
     } else {
-        // ------------------------------------------------------------------ gradient warpgroups (warps 0-7)
+        // ------------------------------------------------------------------ gradient warpgroups (warps 0-15)
+        // Four warpgroups, each taking 32 key columns of every tile: more warps per scheduler hide the latency of
+        // the TMEM loads (a thread's tcgen05.wait::ld waits for all of its loads, so only other warps can).
         const int wx = warp >> 2, wl = warp & 3;
         const int rt = wl * 32 + lane;                                 // query row within the tile = TMEM lane
         const uint32_t lane_off = uint32_t(wl * 32) << 16;
-        const int cb = 64 * wx;                                        // this warpgroup's key columns
+        const int cb = 32 * wx;                                        // this warpgroup's key columns
         uint32_t g = 0, it_n = 0;
         const int32_t *seg_start = meta_ptr<int32_t>(meta, hd.off_seg_start);
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
@@ -218,21 +222,18 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 // P = exp2(S scale log2 e - lse log2 e), packed bf16, kept for the dS step
                 if (!bwait(&sm.s_full, g & 1, abort_flag)) goto done;
                 tc_fence_after();
-                uint32_t pk[32];
+                uint32_t pk[16];
                 {
-                    uint32_t a0[32], a1[32];
+                    uint32_t a0[32];
                     tmem_ld32(tmem + lane_off + COL_S + cb, a0);
-                    tmem_ld32(tmem + lane_off + COL_S + cb + 32, a1);
                     tmem_wait_ld();
                     tc_fence_before();
                     mbar_arrive(&sm.s_free);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
+                    for (int e = 0; e < 16; ++e) {
                         const int c = 2 * e;
-                        const uint32_t u0 = c < 32 ? a0[c] : a1[c - 32];
-                        const uint32_t u1 = c + 1 < 32 ? a0[c + 1] : a1[c - 31];
-                        float p0 = ex2_approx(fmaf(__uint_as_float(u0), sl2, c0));
-                        float p1 = ex2_approx(fmaf(__uint_as_float(u1), sl2, c0));
+                        float p0 = ex2_approx(fmaf(__uint_as_float(a0[c]), sl2, c0));
+                        float p1 = ex2_approx(fmaf(__uint_as_float(a0[c + 1]), sl2, c0));
                         if (cls != TILE_FULL) {
                             if (!(c <= lim_diag && (c < lim_pfx || c >= lim_seg))) p0 = 0.f;
                             if (!(c + 1 <= lim_diag && (c + 1 < lim_pfx || c + 1 >= lim_seg))) p1 = 0.f;
@@ -240,40 +241,33 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         pk[e] = pack_bf16x2(p0, p1);
                     }
                 }
-                // dS = scale P (dP - D) -> this step's dP buffer, columns [cb, cb+32) (already read)
+                // dS = scale P (dP - D) -> this step's dP buffer, columns [cb, cb+16) (already read)
                 const uint32_t cdp = COL_DP + 128 * (g & 1);
                 if (!bwait(&sm.dp_full[g & 1], (g >> 1) & 1, abort_flag)) goto done;
                 tc_fence_after();
                 {
-                    uint32_t a0[32], a1[32];
+                    uint32_t a0[32];
                     tmem_ld32(tmem + lane_off + cdp + cb, a0);
-                    tmem_ld32(tmem + lane_off + cdp + cb + 32, a1);
                     tmem_wait_ld();
-                    uint32_t d0[16], d1[16];
+                    uint32_t d0[16];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int c = 2 * e;
-                        const uint32_t u0 = c < 32 ? a0[c] : a1[c - 32];
-                        const uint32_t u1 = c + 1 < 32 ? a0[c + 1] : a1[c - 31];
+                    for (int e = 0; e < 16; ++e) {
                         const uint32_t p = pk[e];
-                        const uint32_t dd = pack_bf16x2(bf16lo(p) * (__uint_as_float(u0) + lv.y) * scale,
-                                                        bf16hi(p) * (__uint_as_float(u1) + lv.y) * scale);
-                        if (e < 16) d0[e] = dd; else d1[e - 16] = dd;
+                        d0[e] = pack_bf16x2(bf16lo(p) * (__uint_as_float(a0[2 * e]) + lv.y) * scale,
+                                            bf16hi(p) * (__uint_as_float(a0[2 * e + 1]) + lv.y) * scale);
                     }
                     tmem_st16(tmem + lane_off + cdp + cb, d0);
-                    tmem_st16(tmem + lane_off + cdp + cb + 16, d1);
                     tmem_wait_st();
                 }
                 tc_fence_before();
                 mbar_arrive(&sm.ds_ready);
             }
-            // epilogue: dQ rows (dS carried the scale); warpgroup x writes head dims [64x, 64x+64)
+            // epilogue: dQ rows (dS carried the scale); warpgroup x writes head dims [32x, 32x+32)
             if (!bwait(&sm.dq_full, it_n & 1, abort_flag)) goto done;
             tc_fence_after();
             {
-                uint32_t a0[32], a1[32];
+                uint32_t a0[32];
                 tmem_ld32(tmem + lane_off + COL_DQ + cb, a0);
-                tmem_ld32(tmem + lane_off + COL_DQ + cb + 32, a1);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&sm.dq_free);
@@ -285,12 +279,6 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                                             pack_bf16x2(__uint_as_float(a0[8 * e + 2]), __uint_as_float(a0[8 * e + 3])),
                                             pack_bf16x2(__uint_as_float(a0[8 * e + 4]), __uint_as_float(a0[8 * e + 5])),
                                             pack_bf16x2(__uint_as_float(a0[8 * e + 6]), __uint_as_float(a0[8 * e + 7])));
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[4 + e] = make_uint4(pack_bf16x2(__uint_as_float(a1[8 * e]), __uint_as_float(a1[8 * e + 1])),
-                                                pack_bf16x2(__uint_as_float(a1[8 * e + 2]), __uint_as_float(a1[8 * e + 3])),
-                                                pack_bf16x2(__uint_as_float(a1[8 * e + 4]), __uint_as_float(a1[8 * e + 5])),
-                                                pack_bf16x2(__uint_as_float(a1[8 * e + 6]), __uint_as_float(a1[8 * e + 7])));
                 }
             }
         }
@@ -298,7 +286,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
 done:
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == 17) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
