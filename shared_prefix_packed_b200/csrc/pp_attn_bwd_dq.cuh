@@ -14,8 +14,8 @@
 // would otherwise need).
 // Warp roles (576 threads): warps 0-15 form four gradient warpgroups, each taking 32 key columns of every tile
 // (its own slice of S and dP, P kept packed in registers, its dS written into dP columns it has itself read);
-// warp 16 is the TMA producer (Q and dO once per item, K and V through a 2-stage ring); warp 17 allocates TMEM and
-// issues MMAs.
+// warp 16 is the TMA producer (Q and dO once per item, K through a 3-stage ring, V through a 2-stage ring); warp 17
+// allocates TMEM and issues MMAs.
 // TMEM: S [0,128), dP/dS double-buffered [128,256) and [256,384), dQ [384,512). The second dP buffer lets dP of
 // the next key tile run while dS of this one is still being formed, so the gradient warps go from P(j+1) straight
 // to dS(j+1) without waiting on dQ(j).
@@ -29,7 +29,8 @@
 namespace pp {
 
 constexpr int DQ_THREADS = 576;      // 16 gradient warps, producer, MMA
-constexpr int DQ_STAGES = 2;
+constexpr int DQ_KSTAGES = 3;         // K is held from S(j) (issued one tile early) to dQ(j)
+constexpr int DQ_VSTAGES = 2;         // V only feeds dP(j)
 constexpr int DQ_GRAD = 512;          // gradient threads (4 warpgroups x 32 key columns)
 
 struct DqSmem {
@@ -37,14 +38,15 @@ struct DqSmem {
     static constexpr int CHUNK = 128 * 64 * 2;
     alignas(1024) uint8_t q[TILE];
     alignas(1024) uint8_t dout[TILE];
-    alignas(1024) uint8_t k[DQ_STAGES][TILE];
-    alignas(1024) uint8_t v[DQ_STAGES][TILE];
-    uint64_t qd_full, qd_empty, dq_full, dq_free;
-    uint64_t kv_full[DQ_STAGES], kv_empty[DQ_STAGES];
+    alignas(1024) uint8_t k[DQ_KSTAGES][TILE];
+    alignas(1024) uint8_t v[DQ_VSTAGES][TILE];
+    uint64_t q_full, q_empty, do_full, do_empty, dq_full, dq_free;
+    uint64_t k_full[DQ_KSTAGES], k_empty[DQ_KSTAGES], v_full[DQ_VSTAGES], v_empty[DQ_VSTAGES];
     uint64_t s_full, s_free, dp_full[2], ds_ready;
     uint32_t tmem_base;
     int abort_flag;
 };
+static_assert(sizeof(DqSmem) + 1024 <= 232448, "dQ kernel shared memory exceeds 227 KB");
 
 struct DqItem {
     QTile t;
@@ -73,13 +75,19 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     volatile int *abort_flag = &sm.abort_flag;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sm.qd_full, 1);
-        mbar_init(&sm.qd_empty, 1);
+        mbar_init(&sm.q_full, 1);
+        mbar_init(&sm.q_empty, 1);
+        mbar_init(&sm.do_full, 1);
+        mbar_init(&sm.do_empty, 1);
         mbar_init(&sm.dq_full, 1);
         mbar_init(&sm.dq_free, DQ_GRAD);
-        for (int s = 0; s < DQ_STAGES; ++s) {
-            mbar_init(&sm.kv_full[s], 1);
-            mbar_init(&sm.kv_empty[s], 1);
+        for (int s = 0; s < DQ_KSTAGES; ++s) {
+            mbar_init(&sm.k_full[s], 1);
+            mbar_init(&sm.k_empty[s], 1);
+        }
+        for (int s = 0; s < DQ_VSTAGES; ++s) {
+            mbar_init(&sm.v_full[s], 1);
+            mbar_init(&sm.v_empty[s], 1);
         }
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.s_free, DQ_GRAD);
@@ -109,26 +117,32 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         // nothing to do: the metadata builder rejected its input
     } else if (warp == 16) {
         // ------------------------------------------------------------------ TMA producer (one thread)
+        // Q and dO have their own buffers, released once the item's last S / dP is issued, so the next item's
+        // tiles arrive while this one finishes; K and V come through separate rings, each freed by its last use.
         if (lane == 0) {
             uint32_t kv_it = 0, it_n = 0;
             for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
                 const DqItem w = dq_decode(meta, hd, item, hq, hkv);
                 const int n = qtile_nkv(w.t);
-                if (!bwait(&sm.qd_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
-                mbar_arrive_expect_tx(&sm.qd_full, 2 * DqSmem::TILE);
-                for (int c = 0; c < 2; ++c) {
-                    tma_load_3d(sm.q + c * DqSmem::CHUNK, &tmQ, c * 64, w.h, w.t.row0, &sm.qd_full);
-                    tma_load_3d(sm.dout + c * DqSmem::CHUNK, &tmdO, c * 64, w.h, w.t.row0, &sm.qd_full);
-                }
+                if (!bwait(&sm.q_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
+                mbar_arrive_expect_tx(&sm.q_full, DqSmem::TILE);
+                for (int c = 0; c < 2; ++c)
+                    tma_load_3d(sm.q + c * DqSmem::CHUNK, &tmQ, c * 64, w.h, w.t.row0, &sm.q_full);
+                if (!bwait(&sm.do_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
+                mbar_arrive_expect_tx(&sm.do_full, DqSmem::TILE);
+                for (int c = 0; c < 2; ++c)
+                    tma_load_3d(sm.dout + c * DqSmem::CHUNK, &tmdO, c * 64, w.h, w.t.row0, &sm.do_full);
                 for (int j = 0; j < n; ++j, ++kv_it) {
                     const int y0 = w.t.gstart + qtile_kv(w.t, j) * FWD_BN;
-                    const int s = kv_it % DQ_STAGES;
-                    if (!bwait(&sm.kv_empty[s], ((kv_it / DQ_STAGES) & 1) ^ 1, abort_flag)) goto done;
-                    mbar_arrive_expect_tx(&sm.kv_full[s], 2 * DqSmem::TILE);
-                    for (int c = 0; c < 2; ++c) {
-                        tma_load_3d(sm.k[s] + c * DqSmem::CHUNK, &tmK, c * 64, w.kh, y0, &sm.kv_full[s]);
-                        tma_load_3d(sm.v[s] + c * DqSmem::CHUNK, &tmV, c * 64, w.kh, y0, &sm.kv_full[s]);
-                    }
+                    const int sk = kv_it % DQ_KSTAGES, sv = kv_it % DQ_VSTAGES;
+                    if (!bwait(&sm.k_empty[sk], ((kv_it / DQ_KSTAGES) & 1) ^ 1, abort_flag)) goto done;
+                    mbar_arrive_expect_tx(&sm.k_full[sk], DqSmem::TILE);
+                    for (int c = 0; c < 2; ++c)
+                        tma_load_3d(sm.k[sk] + c * DqSmem::CHUNK, &tmK, c * 64, w.kh, y0, &sm.k_full[sk]);
+                    if (!bwait(&sm.v_empty[sv], ((kv_it / DQ_VSTAGES) & 1) ^ 1, abort_flag)) goto done;
+                    mbar_arrive_expect_tx(&sm.v_full[sv], DqSmem::TILE);
+                    for (int c = 0; c < 2; ++c)
+                        tma_load_3d(sm.v[sv] + c * DqSmem::CHUNK, &tmV, c * 64, w.kh, y0, &sm.v_full[sv]);
                 }
             }
         }
@@ -146,50 +160,59 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     umma_ss(tmem + col, smem_desc(a + off, 16, 1024), smem_desc(b + off, 16, 1024), ID_SP, kk > 0);
                 }
             };
+            // S of key tile `it` (ring position) into the S region; releases Q after the item's last tile
+            auto issue_s = [&](uint32_t it, bool last) -> bool {
+                const int sk = it % DQ_KSTAGES;
+                if (!bwait(&sm.k_full[sk], (it / DQ_KSTAGES) & 1, abort_flag)) return false;
+                tc_fence_after();
+                issue_kk(COL_S, sq, smem_u32(sm.k[sk]));
+                umma_commit(&sm.s_full);
+                if (last) umma_commit(&sm.q_empty);
+                return true;
+            };
+            // dP of key tile `it` into dP buffer `b`; frees its V stage, and dO after the item's last tile
+            auto issue_dp = [&](uint32_t it, uint32_t b, bool last) -> bool {
+                const int sv = it % DQ_VSTAGES;
+                if (!bwait(&sm.v_full[sv], (it / DQ_VSTAGES) & 1, abort_flag)) return false;
+                tc_fence_after();
+                issue_kk(COL_DP + 128 * b, sdo, smem_u32(sm.v[sv]));
+                umma_commit(&sm.dp_full[b]);
+                umma_commit(&sm.v_empty[sv]);
+                if (last) umma_commit(&sm.do_empty);
+                return true;
+            };
             for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
                 const DqItem w = dq_decode(meta, hd, item, hq, hkv);
                 const int n = qtile_nkv(w.t);
-                if (!bwait(&sm.qd_full, it_n & 1, abort_flag)) goto done;
                 // S and dP of the first key tile. Buffer reuse is safe by issue order: dP buffer g%2 last held
                 // dS(g-2), read by dQ(g-2); the S region was released by s_free(g-1).
-                {
-                    const int s0 = kv_it % DQ_STAGES;
-                    if (!bwait(&sm.kv_full[s0], (kv_it / DQ_STAGES) & 1, abort_flag)) goto done;
-                    if (g > 0 && !bwait(&sm.s_free, (g - 1) & 1, abort_flag)) goto done;
-                    tc_fence_after();
-                    issue_kk(COL_S, sq, smem_u32(sm.k[s0]));
-                    umma_commit(&sm.s_full);
-                    issue_kk(COL_DP + 128 * (g & 1), sdo, smem_u32(sm.v[s0]));
-                    umma_commit(&sm.dp_full[g & 1]);
-                }
+                if (!bwait(&sm.q_full, it_n & 1, abort_flag)) goto done;
+                if (g > 0 && !bwait(&sm.s_free, (g - 1) & 1, abort_flag)) goto done;
+                if (!issue_s(kv_it, n == 1)) goto done;
+                if (!bwait(&sm.do_full, it_n & 1, abort_flag)) goto done;
+                if (!issue_dp(kv_it, g & 1, n == 1)) goto done;
                 if (!bwait(&sm.dq_free, (it_n & 1) ^ 1, abort_flag)) goto done;
                 for (int j = 0; j < n; ++j, ++kv_it, ++g) {
-                    const int st = kv_it % DQ_STAGES, st1 = (kv_it + 1) % DQ_STAGES;
                     if (j + 1 < n) {
-                        // next tile's dP into the other buffer (its dS(g-1) was read by dQ(g-1), issued earlier)
-                        if (!bwait(&sm.kv_full[st1], ((kv_it + 1) / DQ_STAGES) & 1, abort_flag)) goto done;
-                        tc_fence_after();
-                        issue_kk(COL_DP + 128 * ((g + 1) & 1), sdo, smem_u32(sm.v[st1]));
-                        umma_commit(&sm.dp_full[(g + 1) & 1]);
-                        // next tile's S as soon as the gradient warps have read this tile's S
+                        // next tile's dP into the other buffer (its dS(g-1) was read by dQ(g-1), issued earlier),
+                        // then its S once the gradient warps have read this tile's S
+                        if (!issue_dp(kv_it + 1, (g + 1) & 1, j + 2 == n)) goto done;
                         if (!bwait(&sm.s_free, g & 1, abort_flag)) goto done;
-                        tc_fence_after();
-                        issue_kk(COL_S, sq, smem_u32(sm.k[st1]));
-                        umma_commit(&sm.s_full);
+                        if (!issue_s(kv_it + 1, j + 2 == n)) goto done;
                     }
-                    // dQ += dS K once dS is in TMEM
+                    // dQ += dS K once dS is in TMEM; frees the K stage
                     if (!bwait(&sm.ds_ready, g & 1, abort_flag)) goto done;
                     tc_fence_after();
-                    const uint32_t sk = smem_u32(sm.k[st]);
+                    const int sk = kv_it % DQ_KSTAGES;
+                    const uint32_t skd = smem_u32(sm.k[sk]);
                     const uint32_t cds = COL_DP + 128 * (g & 1);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         umma_ts(tmem + COL_DQ, tmem + cds + 32 * (kk >> 1) + 8 * (kk & 1),
-                                smem_desc(sk + kk * 2048, DqSmem::CHUNK, 1024), ID_DQ, (j > 0 || kk > 0));
-                    umma_commit(&sm.kv_empty[st]);
+                                smem_desc(skd + kk * 2048, DqSmem::CHUNK, 1024), ID_DQ, (j > 0 || kk > 0));
+                    umma_commit(&sm.k_empty[sk]);
                 }
                 umma_commit(&sm.dq_full);
-                umma_commit(&sm.qd_empty);
             }
         }
     } else {
