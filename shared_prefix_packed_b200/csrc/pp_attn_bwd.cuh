@@ -155,30 +155,24 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
                  : "memory");
 }
 
-// dK (scaled) or dV of the item from TMEM: bf16 rows for an unsplit tile, fp32 adds into the workspace otherwise.
-__device__ __forceinline__ void bwd_store_kv(uint32_t taddr, bool yin, bool split, float f, float *acc,
+// dK (dS^T carried the scale) or dV of one item, from registers: bf16 rows for an unsplit key tile, fp32 adds
+// into the workspace for a split one.
+__device__ __forceinline__ void bwd_store_kv(const uint32_t (&rr)[BWD_D], bool split, float *acc,
                                              __nv_bfloat16 *dst, int64_t rowoff) {
+    if (split) {
+        float *a = acc + rowoff;
 #pragma unroll
-    for (int c = 0; c < BWD_D / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(taddr + c * 32, rr);
-        tmem_wait_ld();
-        if (!yin) continue;
-        if (split) {
-            float *a = acc + rowoff + c * 32;
+        for (int e = 0; e < BWD_D / 4; ++e)
+            red_add_v4(a + 4 * e, __uint_as_float(rr[4 * e]), __uint_as_float(rr[4 * e + 1]),
+                       __uint_as_float(rr[4 * e + 2]), __uint_as_float(rr[4 * e + 3]));
+    } else {
+        uint4 *o = reinterpret_cast<uint4 *>(dst + rowoff);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                red_add_v4(a + 4 * e, __uint_as_float(rr[4 * e]) * f, __uint_as_float(rr[4 * e + 1]) * f,
-                           __uint_as_float(rr[4 * e + 2]) * f, __uint_as_float(rr[4 * e + 3]) * f);
-        } else {
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                pk[e] = pack_bf16x2(__uint_as_float(rr[2 * e]) * f, __uint_as_float(rr[2 * e + 1]) * f);
-            uint4 *o = reinterpret_cast<uint4 *>(dst + rowoff + c * 32);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) o[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-        }
+        for (int e = 0; e < BWD_D / 8; ++e)
+            o[e] = make_uint4(pack_bf16x2(__uint_as_float(rr[8 * e]), __uint_as_float(rr[8 * e + 1])),
+                              pack_bf16x2(__uint_as_float(rr[8 * e + 2]), __uint_as_float(rr[8 * e + 3])),
+                              pack_bf16x2(__uint_as_float(rr[8 * e + 4]), __uint_as_float(rr[8 * e + 5])),
+                              pack_bf16x2(__uint_as_float(rr[8 * e + 6]), __uint_as_float(rr[8 * e + 7])));
     }
 }
 
@@ -346,6 +340,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 if (!bwait(&sm.kv_full, it_n & 1, abort_flag)) goto done;
                 if (!issue_s(g)) goto done;
                 if (!issue_dp(g)) goto done;
+                if (n == 1) umma_commit(&sm.kv_empty);           // K and V feed S^T and dP^T only
                 if (!bwait(&sm.dkv_free, (it_n & 1) ^ 1, abort_flag)) goto done;
                 for (int t = 0; t < n; ++t, ++g) {
                     const int st = g % BwdSmem::QSTAGES;
@@ -374,9 +369,9 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     umma_commit(&sm.q_empty[st]);
                     if (t + 1 < n && !s_next && !issue_s(g + 1)) goto done;
                     if (t + 1 < n && !issue_dp(g + 1)) goto done;
+                    if (t + 2 == n) umma_commit(&sm.kv_empty);
                 }
                 umma_commit(&sm.dkv_full);
-                umma_commit(&sm.kv_empty);
             }
         }
     } else {
@@ -392,6 +387,25 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         const int cb = 64 * wx;                                        // first query column of this half
         uint32_t g = 0, it_n = 0;
         const int32_t *key_end = meta_ptr<int32_t>(meta, hd.off_key_end);
+        // Item epilogue, run after the next item's first P so the MMA warp has S^T/dP^T work meanwhile:
+        // warpgroup 0 takes dK, warpgroup 1 dV; the accumulator is released as soon as it is in registers.
+        bool ep_yin = false, ep_split = false;
+        int64_t ep_row = 0;
+        auto epilogue = [&](uint32_t en) -> bool {
+            if (!bwait(&sm.dkv_full, en & 1, abort_flag)) return false;
+            tc_fence_after();
+            uint32_t rr[BWD_D];
+#pragma unroll
+            for (int c = 0; c < BWD_D / 32; ++c)
+                tmem_ld32(tmem + lane_off + (wx == 0 ? COL_DK : COL_DV) + 32 * c,
+                          *reinterpret_cast<uint32_t(*)[32]>(rr + 32 * c));
+            tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(rr), *reinterpret_cast<uint32_t(*)[32]>(rr + 32),
+                         *reinterpret_cast<uint32_t(*)[32]>(rr + 64), *reinterpret_cast<uint32_t(*)[32]>(rr + 96));
+            tc_fence_before();
+            mbar_arrive(&sm.dkv_free);
+            if (ep_yin) bwd_store_kv(rr, ep_split, wx == 0 ? dk_acc : dv_acc, wx == 0 ? dK : dV, ep_row);
+            return true;
+        };
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
             const BwdItem w = bwd_decode(meta, hd, item);
             const int n = (w.qb - w.qa) * r;
@@ -412,7 +426,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     uint32_t a0[32], a1[32];
                     tmem_ld32(tmem + lane_off + COL_S + cb, a0);
                     tmem_ld32(tmem + lane_off + COL_S + cb + 32, a1);
-                    tmem_wait_ld();
+                    tmem_wait_ld(a0, a1);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) { sr[e] = a0[e]; sr[32 + e] = a1[e]; }
                 }
@@ -441,6 +455,10 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 return true;
             };
             if (n > 0 && !phase_p(g, 0)) goto done;
+            if (it_n > 0 && !epilogue(it_n - 1)) goto done;
+            ep_yin = yin;
+            ep_split = w.split;
+            ep_row = (int64_t(y) * hkv + w.kh) * BWD_D;
             for (int t = 0; t < n; ++t, ++g) {
                 // phase 2: dS^T = scale P^T dP'^T (dP' = dP - D already) -> TMEM dP columns this warpgroup has read
                 if (!bwait(&sm.dp_full, g & 1, abort_flag)) goto done;
@@ -451,7 +469,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         uint32_t a0[32], a1[32];
                         tmem_ld32(tmem + lane_off + COL_DP + cb, a0);
                         tmem_ld32(tmem + lane_off + COL_DP + cb + 32, a1);
-                        tmem_wait_ld();
+                        tmem_wait_ld(a0, a1);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) { pr[e] = a0[e]; pr[32 + e] = a1[e]; }
                     }
@@ -472,16 +490,8 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 // next step's phase 1 while this step's dK runs
                 if (t + 1 < n && !phase_p(g + 1, t + 1)) goto done;
             }
-            // item epilogue: warpgroup 0 writes dK (dS^T carried the scale), warpgroup 1 writes dV
-            if (!bwait(&sm.dkv_full, it_n & 1, abort_flag)) goto done;
-            tc_fence_after();
-            if (wx == 0)
-                bwd_store_kv(tmem + lane_off + COL_DK, yin, w.split, 1.f, dk_acc, dK, (int64_t(y) * hkv + w.kh) * BWD_D);
-            else
-                bwd_store_kv(tmem + lane_off + COL_DV, yin, w.split, 1.f, dv_acc, dV, (int64_t(y) * hkv + w.kh) * BWD_D);
-            tc_fence_before();
-            mbar_arrive(&sm.dkv_free);
         }
+        if (it_n > 0 && !epilogue(it_n - 1)) goto done;
     }
 done:
     tc_fence_before();

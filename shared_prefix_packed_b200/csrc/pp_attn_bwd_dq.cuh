@@ -42,7 +42,7 @@ struct DqSmem {
     alignas(1024) uint8_t v[DQ_VSTAGES][TILE];
     uint64_t q_full, q_empty, do_full, do_empty, dq_full, dq_free;
     uint64_t k_full[DQ_KSTAGES], k_empty[DQ_KSTAGES], v_full[DQ_VSTAGES], v_empty[DQ_VSTAGES];
-    uint64_t s_full, s_free, dp_full[2], ds_ready;
+    uint64_t s_full, s_free, dp_full[2], ds_ready[2];   // ds_ready by step parity (see the gradient warps)
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -93,7 +93,8 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         mbar_init(&sm.s_free, DQ_GRAD);
         mbar_init(&sm.dp_full[0], 1);
         mbar_init(&sm.dp_full[1], 1);
-        mbar_init(&sm.ds_ready, DQ_GRAD);
+        mbar_init(&sm.ds_ready[0], DQ_GRAD);
+        mbar_init(&sm.ds_ready[1], DQ_GRAD);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -191,7 +192,6 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 if (!issue_s(kv_it, n == 1)) goto done;
                 if (!bwait(&sm.do_full, it_n & 1, abort_flag)) goto done;
                 if (!issue_dp(kv_it, g & 1, n == 1)) goto done;
-                if (!bwait(&sm.dq_free, (it_n & 1) ^ 1, abort_flag)) goto done;
                 for (int j = 0; j < n; ++j, ++kv_it, ++g) {
                     if (j + 1 < n) {
                         // next tile's dP into the other buffer (its dS(g-1) was read by dQ(g-1), issued earlier),
@@ -200,8 +200,9 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         if (!bwait(&sm.s_free, g & 1, abort_flag)) goto done;
                         if (!issue_s(kv_it + 1, j + 2 == n)) goto done;
                     }
-                    // dQ += dS K once dS is in TMEM; frees the K stage
-                    if (!bwait(&sm.ds_ready, g & 1, abort_flag)) goto done;
+                    // dQ += dS K once dS is in TMEM (and, for the first tile, the last item's dQ has been read)
+                    if (!bwait(&sm.ds_ready[g & 1], (g >> 1) & 1, abort_flag)) goto done;
+                    if (j == 0 && !bwait(&sm.dq_free, (it_n & 1) ^ 1, abort_flag)) goto done;
                     tc_fence_after();
                     const int sk = kv_it % DQ_KSTAGES;
                     const uint32_t skd = smem_u32(sm.k[sk]);
@@ -219,12 +220,39 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         // ------------------------------------------------------------------ gradient warpgroups (warps 0-15)
         // Four warpgroups, each taking 32 key columns of every tile: more warps per scheduler hide the latency of
         // the TMEM loads (a thread's tcgen05.wait::ld waits for all of its loads, so only other warps can).
+        // dP(j+1) is issued before S(j+1), so a warp may finish dS(j+1) while another is still on dS(j): ds_ready
+        // alternates between two barriers by step parity so that such an early arrival never completes step j's
+        // phase. Two steps ahead cannot happen: dP(j+2) waits for all of step j's arrivals.
         const int wx = warp >> 2, wl = warp & 3;
         const int rt = wl * 32 + lane;                                 // query row within the tile = TMEM lane
         const uint32_t lane_off = uint32_t(wl * 32) << 16;
         const int cb = 32 * wx;                                        // this warpgroup's key columns
         uint32_t g = 0, it_n = 0;
         const int32_t *seg_start = meta_ptr<int32_t>(meta, hd.off_seg_start);
+        // Item epilogue, run after the next item's first P (so S and dP of the next tiles keep the tensor pipe
+        // busy): dQ rows in bf16 (dS carried the scale); warpgroup x writes head dims [32x, 32x+32). The
+        // accumulator is released as soon as it is in registers.
+        bool ep_in = false;
+        __nv_bfloat16 *ep_dst = dQ;
+        auto epilogue = [&](uint32_t en) -> bool {
+            if (!bwait(&sm.dq_full, en & 1, abort_flag)) return false;
+            tc_fence_after();
+            uint32_t a0[32];
+            tmem_ld32(tmem + lane_off + COL_DQ + cb, a0);
+            tmem_wait_ld(a0);
+            tc_fence_before();
+            mbar_arrive(&sm.dq_free);
+            if (ep_in) {
+                uint4 *dst = reinterpret_cast<uint4 *>(ep_dst);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    dst[e] = make_uint4(pack_bf16x2(__uint_as_float(a0[8 * e]), __uint_as_float(a0[8 * e + 1])),
+                                        pack_bf16x2(__uint_as_float(a0[8 * e + 2]), __uint_as_float(a0[8 * e + 3])),
+                                        pack_bf16x2(__uint_as_float(a0[8 * e + 4]), __uint_as_float(a0[8 * e + 5])),
+                                        pack_bf16x2(__uint_as_float(a0[8 * e + 6]), __uint_as_float(a0[8 * e + 7])));
+            }
+            return true;
+        };
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
             const DqItem w = dq_decode(meta, hd, item, hq, hkv);
             const int n = qtile_nkv(w.t);
@@ -249,7 +277,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 {
                     uint32_t a0[32];
                     tmem_ld32(tmem + lane_off + COL_S + cb, a0);
-                    tmem_wait_ld();
+                    tmem_wait_ld(a0);
                     tc_fence_before();
                     mbar_arrive(&sm.s_free);
 #pragma unroll
@@ -264,14 +292,19 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         pk[e] = pack_bf16x2(p0, p1);
                     }
                 }
-                // dS = scale P (dP - D) -> this step's dP buffer, columns [cb, cb+16) (already read)
+                if (j == 0) {
+                    if (it_n > 0 && !epilogue(it_n - 1)) goto done;
+                    ep_in = in_group;
+                    ep_dst = dQ + (int64_t(row) * hq + w.h) * 128 + cb;
+                }
+                // dS = scale P (dP - D) -> this step's dP buffer, TMEM columns [cb, cb+16) (already read)
                 const uint32_t cdp = COL_DP + 128 * (g & 1);
                 if (!bwait(&sm.dp_full[g & 1], (g >> 1) & 1, abort_flag)) goto done;
                 tc_fence_after();
                 {
                     uint32_t a0[32];
                     tmem_ld32(tmem + lane_off + cdp + cb, a0);
-                    tmem_wait_ld();
+                    tmem_wait_ld(a0);
                     uint32_t d0[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
@@ -283,28 +316,10 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     tmem_wait_st();
                 }
                 tc_fence_before();
-                mbar_arrive(&sm.ds_ready);
-            }
-            // epilogue: dQ rows (dS carried the scale); warpgroup x writes head dims [32x, 32x+32)
-            if (!bwait(&sm.dq_full, it_n & 1, abort_flag)) goto done;
-            tc_fence_after();
-            {
-                uint32_t a0[32];
-                tmem_ld32(tmem + lane_off + COL_DQ + cb, a0);
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(&sm.dq_free);
-                if (in_group) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(dQ + (int64_t(row) * hq + w.h) * 128 + cb);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(pack_bf16x2(__uint_as_float(a0[8 * e]), __uint_as_float(a0[8 * e + 1])),
-                                            pack_bf16x2(__uint_as_float(a0[8 * e + 2]), __uint_as_float(a0[8 * e + 3])),
-                                            pack_bf16x2(__uint_as_float(a0[8 * e + 4]), __uint_as_float(a0[8 * e + 5])),
-                                            pack_bf16x2(__uint_as_float(a0[8 * e + 6]), __uint_as_float(a0[8 * e + 7])));
-                }
+                mbar_arrive(&sm.ds_ready[g & 1]);
             }
         }
+        if (it_n > 0 && !epilogue(it_n - 1)) goto done;
     }
 done:
     tc_fence_before();

@@ -259,7 +259,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     tmem_ld32(t_s + 32, r1);
                     tmem_ld32(t_s + 64, r2);
                     tmem_ld32(t_s + 96, r3);
-                    tmem_wait_ld();
+                    tmem_wait_ld(r0, r1, r2, r3);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         s[e] = __uint_as_float(r0[e]);
@@ -317,7 +317,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t rr[32];
                         tmem_ld32(t_o + c * 32, rr);
-                        tmem_wait_ld();
+                        tmem_wait_ld(rr);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
                         tmem_st32(t_o + c * 32, rr);
@@ -338,7 +338,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t rr[32];
                     tmem_ld32(t_o + c * 32, rr);
-                    tmem_wait_ld();
+                    tmem_wait_ld(rr);
                     if (in_group) {
                         uint32_t pk[16];
 #pragma unroll
