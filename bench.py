@@ -216,7 +216,9 @@ def run_gpu(args):
         if marks is not None:
             marks[4].record(stream)
 
-    launches_per_step = 5 + (1 if w.rope else 0) + 1 + (3 if w.backward else 0)
+    # our kernels per step: metadata (header + 4 stages), RoPE, forward, and the backward's lse/D pass, dK/dV kernel,
+    # dQ kernel and split-tile conversion (the workspace memset is a driver memset, not counted)
+    launches_per_step = 5 + (1 if w.rope else 0) + 1 + (4 if w.backward else 0)
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)                      # nvidia-smi needs a moment before its first sample

@@ -133,11 +133,14 @@ struct BwdItem {
     int qa, qb, split, kh;
 };
 
-__device__ __forceinline__ BwdItem bwd_decode(const void *meta, const MetaHeader &hd, int item) {
-    const BWork w = meta_ptr<BWork>(meta, hd.off_bw)[item % hd.n_bw];
+__device__ __forceinline__ BwdItem bwd_decode(const void *meta, const MetaHeader &hd, int item, int hkv) {
+    const BWork w = meta_ptr<BWork>(meta, hd.off_bw)[item / hkv];
     BwdItem it;
-    it.kh = item / hd.n_bw;
-    it.t = meta_ptr<KTile>(meta, hd.off_kt)[w.kt];
+    it.kh = item % hkv;
+    it.t = KTile{};
+    it.t.row0 = w.row0;
+    it.t.gstart = w.gstart;
+    it.t.glen = w.glen;
     it.qa = w.qa;
     it.qb = w.qb;
     it.split = w.split;
@@ -155,24 +158,33 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
                  : "memory");
 }
 
-// dK (dS^T carried the scale) or dV of one item, from registers: bf16 rows for an unsplit key tile, fp32 adds
-// into the workspace for a split one.
-__device__ __forceinline__ void bwd_store_kv(const uint32_t (&rr)[BWD_D], bool split, float *acc,
-                                             __nv_bfloat16 *dst, int64_t rowoff) {
+// 64 columns of dK (dS^T carried the scale) or dV of one key row, from registers: bf16 for an unsplit key tile,
+// fp32 adds into the workspace for a split one.
+__device__ __forceinline__ void bwd_store_kv64(const uint32_t (&a)[32], const uint32_t (&b)[32], bool split,
+                                               float *acc, __nv_bfloat16 *dst) {
     if (split) {
-        float *a = acc + rowoff;
 #pragma unroll
-        for (int e = 0; e < BWD_D / 4; ++e)
-            red_add_v4(a + 4 * e, __uint_as_float(rr[4 * e]), __uint_as_float(rr[4 * e + 1]),
-                       __uint_as_float(rr[4 * e + 2]), __uint_as_float(rr[4 * e + 3]));
+        for (int e = 0; e < 8; ++e)
+            red_add_v4(acc + 4 * e, __uint_as_float(a[4 * e]), __uint_as_float(a[4 * e + 1]),
+                       __uint_as_float(a[4 * e + 2]), __uint_as_float(a[4 * e + 3]));
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            red_add_v4(acc + 32 + 4 * e, __uint_as_float(b[4 * e]), __uint_as_float(b[4 * e + 1]),
+                       __uint_as_float(b[4 * e + 2]), __uint_as_float(b[4 * e + 3]));
     } else {
-        uint4 *o = reinterpret_cast<uint4 *>(dst + rowoff);
+        uint4 *o = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-        for (int e = 0; e < BWD_D / 8; ++e)
-            o[e] = make_uint4(pack_bf16x2(__uint_as_float(rr[8 * e]), __uint_as_float(rr[8 * e + 1])),
-                              pack_bf16x2(__uint_as_float(rr[8 * e + 2]), __uint_as_float(rr[8 * e + 3])),
-                              pack_bf16x2(__uint_as_float(rr[8 * e + 4]), __uint_as_float(rr[8 * e + 5])),
-                              pack_bf16x2(__uint_as_float(rr[8 * e + 6]), __uint_as_float(rr[8 * e + 7])));
+        for (int e = 0; e < 4; ++e)
+            o[e] = make_uint4(pack_bf16x2(__uint_as_float(a[8 * e]), __uint_as_float(a[8 * e + 1])),
+                              pack_bf16x2(__uint_as_float(a[8 * e + 2]), __uint_as_float(a[8 * e + 3])),
+                              pack_bf16x2(__uint_as_float(a[8 * e + 4]), __uint_as_float(a[8 * e + 5])),
+                              pack_bf16x2(__uint_as_float(a[8 * e + 6]), __uint_as_float(a[8 * e + 7])));
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            o[4 + e] = make_uint4(pack_bf16x2(__uint_as_float(b[8 * e]), __uint_as_float(b[8 * e + 1])),
+                                  pack_bf16x2(__uint_as_float(b[8 * e + 2]), __uint_as_float(b[8 * e + 3])),
+                                  pack_bf16x2(__uint_as_float(b[8 * e + 4]), __uint_as_float(b[8 * e + 5])),
+                                  pack_bf16x2(__uint_as_float(b[8 * e + 6]), __uint_as_float(b[8 * e + 7])));
     }
 }
 
@@ -241,7 +253,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         // ------------------------------------------------------------------ producer warp
         uint32_t g = 0, it_n = 0;
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
-            const BwdItem w = bwd_decode(meta, hd, item);
+            const BwdItem w = bwd_decode(meta, hd, item, hkv);
             if (lane == 0) {
                 if (!bwait(&sm.kv_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
                 mbar_arrive_expect_tx(&sm.kv_full, 2 * BwdSmem::TILE);
@@ -334,9 +346,12 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 umma_commit(&sm.s_full);
                 return true;
             };
+            const BWork *bws = meta_ptr<BWork>(meta, hd.off_bw);
+            auto item_steps = [&](int it) { const BWork b = bws[it / hkv]; return (b.qb - b.qa) * r; };
+            int n_next = blockIdx.x < n_items ? item_steps(blockIdx.x) : 0;
             for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
-                const BwdItem w = bwd_decode(meta, hd, item);
-                const int n = (w.qb - w.qa) * r;
+                const int n = n_next;                                  // loaded one item ahead
+                if (item + int(gridDim.x) < n_items) n_next = item_steps(item + gridDim.x);
                 if (!bwait(&sm.kv_full, it_n & 1, abort_flag)) goto done;
                 if (!issue_s(g)) goto done;
                 if (!issue_dp(g)) goto done;
@@ -394,25 +409,44 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         auto epilogue = [&](uint32_t en) -> bool {
             if (!bwait(&sm.dkv_full, en & 1, abort_flag)) return false;
             tc_fence_after();
-            uint32_t rr[BWD_D];
+            const uint32_t src = tmem + lane_off + (wx == 0 ? COL_DK : COL_DV);
+            float *acc = (wx == 0 ? dk_acc : dv_acc) + ep_row;
+            __nv_bfloat16 *dst = (wx == 0 ? dK : dV) + ep_row;
 #pragma unroll
-            for (int c = 0; c < BWD_D / 32; ++c)
-                tmem_ld32(tmem + lane_off + (wx == 0 ? COL_DK : COL_DV) + 32 * c,
-                          *reinterpret_cast<uint32_t(*)[32]>(rr + 32 * c));
-            tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(rr), *reinterpret_cast<uint32_t(*)[32]>(rr + 32),
-                         *reinterpret_cast<uint32_t(*)[32]>(rr + 64), *reinterpret_cast<uint32_t(*)[32]>(rr + 96));
-            tc_fence_before();
-            mbar_arrive(&sm.dkv_free);
-            if (ep_yin) bwd_store_kv(rr, ep_split, wx == 0 ? dk_acc : dv_acc, wx == 0 ? dK : dV, ep_row);
+            for (int half = 0; half < 2; ++half) {                     // 64 columns at a time
+                uint32_t a[32], b[32];
+                tmem_ld32(src + 64 * half, a);
+                tmem_ld32(src + 64 * half + 32, b);
+                tmem_wait_ld(a, b);
+                if (half == 1) {                                       // the accumulator is no longer needed
+                    tc_fence_before();
+                    mbar_arrive(&sm.dkv_free);
+                }
+                if (ep_yin) bwd_store_kv64(a, b, ep_split, acc + 64 * half, dst + 64 * half);
+            }
             return true;
         };
+        // The next item's work chunk is loaded at the start of this one and its key_end after this item's first P,
+        // so no global load latency sits on the first step of an item.
+        auto key_end_of = [&](const BwdItem &b) {
+            const int yy = b.t.row0 + jr;
+            return yy < b.t.gstart + b.t.glen ? key_end[yy] : yy;
+        };
+        BwdItem wn{};
+        int ken = 0;
+        if (blockIdx.x < n_items) {
+            wn = bwd_decode(meta, hd, blockIdx.x, hkv);
+            ken = key_end_of(wn);
+        }
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
-            const BwdItem w = bwd_decode(meta, hd, item);
+            const BwdItem w = wn;
+            const int ke = ken;                                        // queries [y, ke) attend key y
+            const int nxt = item + gridDim.x;
+            if (nxt < n_items) wn = bwd_decode(meta, hd, nxt, hkv);
             const int n = (w.qb - w.qa) * r;
             const int y = w.t.row0 + jr;
             const int gend = w.t.gstart + w.t.glen;
             const bool yin = y < gend;
-            const int ke = yin ? key_end[y] : y;                       // queries [y, ke) attend key y
             uint32_t pk[32];                                           // P^T of the current step, packed bf16
             // phase 1 of step gg: P^T = exp2(S'^T * scale * log2 e) (S' already holds s - lse / scale)
             auto phase_p = [&](uint32_t gg, int t) -> bool {
@@ -456,6 +490,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             };
             if (n > 0 && !phase_p(g, 0)) goto done;
             if (it_n > 0 && !epilogue(it_n - 1)) goto done;
+            if (nxt < n_items) ken = key_end_of(wn);
             ep_yin = yin;
             ep_split = w.split;
             ep_row = (int64_t(y) * hkv + w.kh) * BWD_D;

@@ -54,9 +54,8 @@ struct DqItem {
 };
 
 __device__ __forceinline__ DqItem dq_decode(const void *meta, const MetaHeader &hd, int item, int hq, int hkv) {
-    const int32_t *qorder = meta_ptr<int32_t>(meta, hd.off_qorder);
     DqItem it;
-    it.t = meta_ptr<QTile>(meta, hd.off_qt)[qorder[item / hq]];
+    it.t = meta_ptr<QTile>(meta, hd.off_qts)[item / hq];
     it.h = item % hq;
     it.kh = it.h / (hq / hkv);
     return it;
@@ -182,9 +181,11 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 if (last) umma_commit(&sm.do_empty);
                 return true;
             };
+            const QTile *qts = meta_ptr<QTile>(meta, hd.off_qts);
+            int n_next = blockIdx.x < n_items ? qtile_nkv(qts[blockIdx.x / hq]) : 0;
             for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
-                const DqItem w = dq_decode(meta, hd, item, hq, hkv);
-                const int n = qtile_nkv(w.t);
+                const int n = n_next;                                  // loaded one item ahead
+                if (item + int(gridDim.x) < n_items) n_next = qtile_nkv(qts[(item + gridDim.x) / hq]);
                 // S and dP of the first key tile. Buffer reuse is safe by issue order: dP buffer g%2 last held
                 // dS(g-2), read by dQ(g-2); the S region was released by s_free(g-1).
                 if (!bwait(&sm.q_full, it_n & 1, abort_flag)) goto done;
@@ -253,15 +254,34 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             }
             return true;
         };
+        // The next item's tile is loaded at the start of this one and its per-row values (segment start, -lse/scale,
+        // -D) after this item's first P, so no global load latency sits on the first step of an item.
+        const QTile *qts = meta_ptr<QTile>(meta, hd.off_qts);
+        auto row_values = [&](const QTile &t, int item, int &s0, float2 &lv) {
+            const int row = t.row0 + rt;
+            s0 = row < t.gstart + t.glen ? seg_start[row] : 0;
+            lv = ldg[int64_t(item % hq) * rows_pad + row];            // padded past T
+        };
+        QTile tn{};
+        int s0n = 0;
+        float2 lvn = make_float2(0.f, 0.f);
+        if (blockIdx.x < n_items) {
+            tn = qts[blockIdx.x / hq];
+            row_values(tn, blockIdx.x, s0n, lvn);
+        }
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
-            const DqItem w = dq_decode(meta, hd, item, hq, hkv);
+            DqItem w;
+            w.t = tn;
+            w.h = item % hq;
+            const int nxt = item + gridDim.x;
+            if (nxt < n_items) tn = qts[nxt / hq];
             const int n = qtile_nkv(w.t);
             const int row = w.t.row0 + rt;
             const bool in_group = row < w.t.gstart + w.t.glen;
-            const int s0 = in_group ? seg_start[row] : 0;
+            const int s0 = s0n;
             const int pfx_end = w.t.gstart + w.t.plen;
             const int x0 = w.t.row0 - w.t.gstart;
-            const float2 lv = ldg[int64_t(w.h) * rows_pad + row];     // (-lse / scale, -D); padded past T
+            const float2 lv = lvn;                                     // (-lse / scale, -D)
             const float c0 = lv.x * sl2;                               // - lse * log2 e
             for (int j = 0; j < n; ++j, ++g) {
                 const int yt = qtile_kv(w.t, j) * FWD_BN;
@@ -296,6 +316,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     if (it_n > 0 && !epilogue(it_n - 1)) goto done;
                     ep_in = in_group;
                     ep_dst = dQ + (int64_t(row) * hq + w.h) * 128 + cb;
+                    if (nxt < n_items) row_values(tn, nxt, s0n, lvn);
                 }
                 // dS = scale P (dP - D) -> this step's dP buffer, TMEM columns [cb, cb+16) (already read)
                 const uint32_t cdp = COL_DP + 128 * (g & 1);

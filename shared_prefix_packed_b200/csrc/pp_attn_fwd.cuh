@@ -85,8 +85,7 @@ __device__ __forceinline__ FwdItem fwd_decode(const void *meta, const MetaHeader
     const int pr = slot % spk;
     it.h0 = it.kh * r + 2 * pr;
     it.nh = (2 * pr + 1 < r) ? 2 : 1;
-    const int32_t *qorder = meta_ptr<int32_t>(meta, hd.off_qorder);
-    it.t = meta_ptr<QTile>(meta, hd.off_qt)[qorder[qi]];
+    it.t = meta_ptr<QTile>(meta, hd.off_qts)[qi];
     return it;
 }
 
@@ -381,12 +380,11 @@ __global__ void __launch_bounds__(128) k_attn_fwd_simt(const T *__restrict__ q, 
     if (hd.dev_err) return;
     const int Tn = hd.T;
     const int r = hq / hkv;
-    const int32_t *qorder = meta_ptr<int32_t>(meta, hd.off_qorder);
-    const QTile *qts = meta_ptr<QTile>(meta, hd.off_qt);
+    const QTile *qts = meta_ptr<QTile>(meta, hd.off_qts);
     const int32_t *seg_start = meta_ptr<int32_t>(meta, hd.off_seg_start);
     const int n_items = hd.n_qt * hq;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const QTile t = qts[qorder[item / hq]];
+        const QTile t = qts[item / hq];
         const int h = item % hq, kh = h / r;
         const int row = t.row0 + threadIdx.x;
         const bool in_group = row < t.gstart + t.glen;

@@ -215,6 +215,7 @@ __global__ void __launch_bounds__(NT) k_meta_sort(void *meta, int32_t *chunk_off
     const QTile *qt = meta_ptr<QTile>(meta, h->off_qt);
     const KTile *kt = meta_ptr<KTile>(meta, h->off_kt);
     int32_t *qorder = meta_ptr<int32_t>(meta, h->off_qorder);
+    QTile *qts = meta_ptr<QTile>(meta, h->off_qts);
     BWork *bw = meta_ptr<BWork>(meta, h->off_bw);
 
     // ---- forward query tiles by decreasing key-tile count
@@ -231,6 +232,7 @@ __global__ void __launch_bounds__(NT) k_meta_sort(void *meta, int32_t *chunk_off
     for (int i = threadIdx.x; i < nq; i += NT) {
         const int p = atomicAdd(&s_hist[min(qtile_nkv(qt[i]), SORT_BINS - 1)], 1);
         qorder[p] = i;
+        qts[p] = qt[i];
     }
     __syncthreads();
 
@@ -249,6 +251,10 @@ __global__ void __launch_bounds__(NT) k_meta_sort(void *meta, int32_t *chunk_off
             w.qa = t.qa + (nqt * c) / t.nch;
             w.qb = t.qa + (nqt * (c + 1)) / t.nch;
             w.split = t.nch > 1 ? 1 : 0;
+            w.row0 = t.row0;
+            w.gstart = t.gstart;
+            w.glen = t.glen;
+            w.pad = 0;
             bw_tmp[chunk_off[i] + c] = w;
         }
     }

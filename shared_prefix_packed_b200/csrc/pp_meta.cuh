@@ -59,6 +59,8 @@ struct alignas(16) BWork {      // backward work chunk: key tile kt, query tiles
     int32_t kt;
     int32_t qa, qb;
     int32_t split;    // 1 if the key tile is split over several chunks (partials are added into fp32 scratch)
+    int32_t row0, gstart, glen;   // the key tile's first row, group offset and group length (copied from kt)
+    int32_t pad;
 };
 
 struct alignas(16) MetaHeader {
@@ -77,6 +79,7 @@ struct alignas(16) MetaHeader {
     int64_t off_gseg;        // int32[G+1]: first segment index of each group
     int64_t off_qt;          // QTile[cap_qt], in group order
     int64_t off_qorder;      // int32[cap_qt]: query tiles sorted by decreasing cost
+    int64_t off_qts;         // QTile[cap_qt]: the query tiles in that order (one load per work item)
     int64_t off_kt;          // KTile[cap_kt]
     int64_t off_bw;          // BWork[cap_bw], sorted by decreasing cost
     int64_t off_scratch;     // builder scratch: qoff int32[G+1], koff int32[G+1], tmp int32[max(cap_kt, SORT_BINS)]
@@ -105,6 +108,7 @@ __host__ __device__ inline MetaHeader meta_layout(int64_t T, int32_t G, int32_t 
     h.off_gseg = o;      o = align256(o + 4 * int64_t(G + 1));
     h.off_qt = o;        o = align256(o + int64_t(sizeof(QTile)) * h.cap_qt);
     h.off_qorder = o;    o = align256(o + 4 * int64_t(h.cap_qt));
+    h.off_qts = o;       o = align256(o + int64_t(sizeof(QTile)) * h.cap_qt);
     h.off_kt = o;        o = align256(o + int64_t(sizeof(KTile)) * h.cap_kt);
     h.off_bw = o;        o = align256(o + int64_t(sizeof(BWork)) * h.cap_bw);
     h.off_scratch = o;

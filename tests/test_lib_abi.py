@@ -41,7 +41,12 @@ def test_host_only_calls_and_validation():
     from shared_prefix_packed_b200 import _lib
     n = _lib.pp_meta_bounds(8, 24, 17801, 32, 8)
     assert n > 8 * 17801
-    assert _lib.pp_workspace_bytes(_lib.PP_PASS_BWD, 1000, 32, 8, 128) > 4 * 32 * 1000 * 128
+    # backward workspace: (-lse/scale, -D) per q head and row, plus fp32 dK and dV for split key tiles, over the
+    # padded rows (T + 256, rounded to 8), each section 256-byte aligned
+    rows = (1000 + 256 + 7) & ~7
+    a256 = lambda x: (x + 255) & ~255
+    want = a256(8 * 32 * rows) + 2 * a256(4 * rows * 8 * 128)
+    assert _lib.pp_workspace_bytes(_lib.PP_PASS_BWD, 1000, 32, 8, 128) == want
     with pytest.raises(_lib.PPError, match="INVALID_ARG"):
         _lib.pp_meta_bounds(0, 1, 10, 32, 8)
     with pytest.raises(_lib.PPError, match="INVALID_ARG"):
