@@ -34,8 +34,10 @@
 // slices cost 2 of 34 MMAs per step. They live in shared memory as 128 x 16 bf16 tiles in the no-swizzle
 // core-matrix layout; the producer warp writes the query side for each step.
 // Q/dO tiles come through a 2-stage ring, prefetched into L2 two steps ahead.
-// Work items run kv-head-major: concurrently running CTAs share a kv head, so a group's Q/dO rows are reused from
-// L2 across its key tiles.
+// Work items run in cost order within groups of four kv heads (bwd_item_split): cost order balances the static
+// round-robin, and the head groups bound the Q/dO rows that concurrently running items read, so they are reused
+// from L2 across key tiles. Each item's metadata is loaded one item ahead, and an item's epilogue (dK/dV out of
+// TMEM) runs after the next item's first P, so the next item's S^T/dP^T keep the tensor pipe busy meanwhile.
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -69,31 +71,47 @@ inline BwdWorkspace bwd_workspace_layout(int64_t T, int hq, int hkv, int d) {
 }
 
 // ------------------------------------------------------------------------------------------------- preprocess
-// One warp per (row, head): D = sum_d dO * O in fp32, stored with the lse as (-lse / scale, -D), the values the
-// query side of the extra MMA slice carries; padding rows get zeros.
+// D = sum_d dO * O in fp32 per (row, head), stored with the lse as (-lse / scale, -D), the values the query side of
+// the extra MMA slice carries; padding rows get zeros. (row, head) pairs are contiguous 256-byte rows of O and dO,
+// so a warp takes eight consecutive pairs: half-warps of 16 lanes x 16 bytes, four loads of each tensor in flight
+// per lane (HBM-bound).
 __global__ void k_bwd_pre(const __nv_bfloat16 *__restrict__ O, const __nv_bfloat16 *__restrict__ dO,
                           const float *__restrict__ lse, float2 *__restrict__ ld, int64_t T, int64_t rows_pad,
                           int hq, float inv_scale) {
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
+    const int64_t n_pairs = rows_pad * hq, n_real = T * hq;
     const int64_t nwarps = int64_t(gridDim.x) * (blockDim.x >> 5);
-    for (int64_t w = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < rows_pad * hq; w += nwarps) {
-        const int64_t i = w / hq;
-        const int h = static_cast<int>(w % hq);
-        float acc = 0.f;
-        if (i < T) {
-            const uint2 a = reinterpret_cast<const uint2 *>(O + (i * hq + h) * BWD_D)[lane];
-            const uint2 b = reinterpret_cast<const uint2 *>(dO + (i * hq + h) * BWD_D)[lane];
-            const uint32_t av[2] = {a.x, a.y}, bv[2] = {b.x, b.y};
+    for (int64_t c = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); c * 8 < n_pairs; c += nwarps) {
+        uint4 a[4], b[4];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(bv[e] << 16), acc);
-                acc = fmaf(__uint_as_float(av[e] & 0xffff0000u), __uint_as_float(bv[e] & 0xffff0000u), acc);
+        for (int k = 0; k < 4; ++k) {
+            const int64_t w = c * 8 + 2 * k + half;                   // pair index = row * hq + head
+            if (w < n_real) {
+                a[k] = reinterpret_cast<const uint4 *>(O + w * BWD_D)[hl];
+                b[k] = reinterpret_cast<const uint4 *>(dO + w * BWD_D)[hl];
+            } else {
+                a[k] = make_uint4(0, 0, 0, 0);
+                b[k] = make_uint4(0, 0, 0, 0);
             }
         }
 #pragma unroll
-        for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0)
-            ld[int64_t(h) * rows_pad + i] = make_float2(i < T ? -lse[int64_t(h) * T + i] * inv_scale : 0.f, -acc);
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t av[4] = {a[k].x, a[k].y, a[k].z, a[k].w}, bv[4] = {b[k].x, b[k].y, b[k].z, b[k].w};
+            float acc = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(bv[e] << 16), acc);
+                acc = fmaf(__uint_as_float(av[e] & 0xffff0000u), __uint_as_float(bv[e] & 0xffff0000u), acc);
+            }
+#pragma unroll
+            for (int off = 8; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            const int64_t w = c * 8 + 2 * k + half;
+            if (hl == 0 && w < n_pairs) {
+                const int64_t i = w / hq;
+                const int h = static_cast<int>(w % hq);
+                ld[int64_t(h) * rows_pad + i] = make_float2(i < T ? -lse[int64_t(h) * T + i] * inv_scale : 0.f, -acc);
+            }
+        }
     }
 }
 
@@ -133,10 +151,21 @@ struct BwdItem {
     int qa, qb, split, kh;
 };
 
+// Work item -> (work chunk, kv head). Items run in groups of up to four kv heads; within a group, chunks in cost
+// order with the group's heads interleaved. Cost order keeps the static round-robin balanced; the head groups keep
+// the Q/dO tiles that concurrently running items read (those of the group's q heads) small enough to stay in L2.
+__device__ __forceinline__ int2 bwd_item_split(int item, int n_bw, int hkv) {
+    const int G = (hkv % 4 == 0) ? 4 : (hkv % 2 == 0 ? 2 : 1);
+    const int per = n_bw * G;
+    const int grp = item / per, pos = item % per;
+    return make_int2(pos / G, grp * G + pos % G);
+}
+
 __device__ __forceinline__ BwdItem bwd_decode(const void *meta, const MetaHeader &hd, int item, int hkv) {
-    const BWork w = meta_ptr<BWork>(meta, hd.off_bw)[item / hkv];
+    const int2 bk = bwd_item_split(item, hd.n_bw, hkv);
+    const BWork w = meta_ptr<BWork>(meta, hd.off_bw)[bk.x];
     BwdItem it;
-    it.kh = item % hkv;
+    it.kh = bk.y;
     it.t = KTile{};
     it.t.row0 = w.row0;
     it.t.gstart = w.gstart;
@@ -347,7 +376,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 return true;
             };
             const BWork *bws = meta_ptr<BWork>(meta, hd.off_bw);
-            auto item_steps = [&](int it) { const BWork b = bws[it / hkv]; return (b.qb - b.qa) * r; };
+            auto item_steps = [&](int it) { const BWork b = bws[bwd_item_split(it, hd.n_bw, hkv).x]; return (b.qb - b.qa) * r; };
             int n_next = blockIdx.x < n_items ? item_steps(blockIdx.x) : 0;
             for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
                 const int n = n_next;                                  // loaded one item ahead
