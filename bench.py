@@ -93,21 +93,25 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current kernel sources."""
+def recorded_traffic(kernels):
+    """DRAM bytes per launch summed over `kernels`, from the committed ncu summary, if every one of them was taken
+    on the current kernel sources (None otherwise)."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
     src = kernel_source_hash()
+    found = {}
     with open(path) as f:
         for ln in f:
             parts = dict(p.split("=", 1) for p in ln.strip().split() if "=" in p)
-            if parts.get("kernel") == kernel and parts.get("sources") == src:
+            if parts.get("kernel") in kernels and parts.get("sources") == src:
                 try:
-                    return float(parts["dram_bytes_per_launch"])
+                    found[parts["kernel"]] = float(parts["dram_bytes_per_launch"])
                 except (KeyError, ValueError):
                     return None
-    return None
+    if set(found) != set(kernels):
+        return None
+    return sum(found.values())
 
 
 class ClockSampler:
@@ -299,10 +303,10 @@ def run_gpu(args):
     dom = "attn_bwd" if w.backward and parts["attn_bwd"] >= parts["attn_fwd"] else "attn_fwd"
     dom_flops = f_bwd if dom == "attn_bwd" else f_fwd
     achieved = dom_flops / (parts[dom] * 1e-3) / 1e12
-    kernel_name = "k_bwd_tc" if dom == "attn_bwd" else "k_attn_fwd_tc"
-    roofline = {"bound": "tensor", "kernel": f"pp_{dom} ({kernel_name} + its helper kernels)",
+    kernels = ["k_bwd_pre", "k_bwd_tc", "k_bwd_dq", "k_bwd_convert"] if dom == "attn_bwd" else ["k_attn_fwd_tc"]
+    roofline = {"bound": "tensor", "kernel": f"pp_{dom} ({' + '.join(kernels)})",
                 "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": recorded_traffic(kernel_name),
+                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": recorded_traffic(kernels),
                 "peak_source": peaks["source"] + " bf16_tflops (burst)",
                 "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4)
                 if peaks.get("bf16_tflops_sustained") else None,

@@ -141,8 +141,11 @@ PP_API pp_status pp_attn_fwd(const void *q, const void *k, const void *v, const 
  *   (sums over the q heads h that share kv head j's head). q, k, v, o, lse: the forward's inputs and outputs;
  *   dout: [T, hq, d]. dq, dk, dv: outputs in bf16 with the shapes of q, k, v (fully overwritten).
  *   workspace: ws_bytes >= pp_workspace_bytes(PP_PASS_BWD, ...), 256-byte aligned, contents need not be
- *   initialised. Prefix key tiles, attended by every response of their group, are split into chunks whose fp32
- *   partial dK/dV are added tile by tile into the workspace (bounded: one bulk add per chunk and tile).
+ *   initialised. It holds (-lse/scale, -D) per row and q head, and fp32 dK/dV for the prefix key tiles, which are
+ *   attended by every response of their group and so are split into chunks whose partials are added there (fp32
+ *   reduction adds, one per element and chunk) before conversion to bf16. dq needs no scratch: each row tile of
+ *   dq is produced by exactly one CTA, which recomputes the tile's scores and dP instead of exchanging partials.
+ *   The result is deterministic except for the order of those dK/dV adds.
  */
 PP_API pp_status pp_attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
                       const void *dout, const void *meta_d, int64_t T, int32_t hq, int32_t hkv, int32_t d,
@@ -159,7 +162,7 @@ PP_API pp_status pp_attn_bwd(const void *q, const void *k, const void *v, const 
  * PP_NOALLOC_SCRATCH_BYTES = 64 MiB; every GPU that loads libpp holds it until the process exits). It calls no
  * allocator at all.
  *   Limit: the scratch a call needs (pp_workspace_bytes(PP_PASS_BWD, T, hq, hkv, d)) must fit in 64 MiB, e.g.
- *   T <= about 2,400 tokens at 32/8 heads and d = 128; a larger call returns PP_ERR_WORKSPACE and enqueues nothing.
+ *   T <= about 7,600 tokens at 32/8 heads and d = 128; a larger call returns PP_ERR_WORKSPACE and enqueues nothing.
  *   Set-up: the first call on each device looks up the array's device address (cudaGetSymbolAddress) with that
  *   device current; make that first call before any stream capture.
  *   Sharing: every call on a device uses the same array, which keeps the last call's contents; the call clears the
