@@ -85,6 +85,29 @@ def test_fwd_fp32_random():
     _compare_full(P, S, inp, o, lse)
 
 
+def test_fwd_running_max_rescale():
+    """Scores that rise by about 6 (natural units) from each key tile to the next, so the running max of every row
+    jumps past the lazy-rescale threshold (8 in log2 units, 5.5 natural) at almost every tile: the path that scales
+    the O accumulator before P is handed to the PV MMA."""
+    from shared_prefix_packed_b200 import PackedBatch, pp_get_status
+    P, S = [640], [[200, 130]]
+    hq, hkv, d = 4, 2, 128
+    T = P[0] + sum(S[0])
+    rng = np.random.default_rng(4242)
+    u = rng.standard_normal(d)
+    u /= np.linalg.norm(u)
+    scale = 1.0 / np.sqrt(d)
+    b = 6.0 * (np.arange(T) // 128) / (scale * 24.0)                 # key row y of tile t scores about 6 t
+    q = 24.0 * u[None, None, :] + 0.3 * rng.standard_normal((T, hq, d))
+    k = b[:, None, None] * u[None, None, :] + 0.3 * rng.standard_normal((T, hkv, d))
+    v = rng.standard_normal((T, hkv, d))
+    inp = {n: torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16) for n, x in (("q", q), ("k", k), ("v", v))}
+    bt = PackedBatch(P, S, hq, hkv, d)
+    o, lse = bt.forward(*(inp[n].cuda() for n in "qkv"))
+    pp_get_status()
+    _compare_full(P, S, inp, o, lse)
+
+
 @pytest.mark.parametrize("name", ["dpo", "grpo", "longprefix", "hetero"])
 def test_fwd_full_workload_sampled_rows(name):
     """Full-size workload in the launch configuration the bench times; the oracle computes sampled rows."""
