@@ -186,10 +186,8 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 umma_ts(tmem + 256 + hs * 128, tmem + hs * 128 + kk * 8,
                         smem_desc(vb + kk * 2048, FwdSmem<D>::CHUNK_BYTES, 1024), IDESC_O, (acc | kk) ? 1u : 0u);
         };
-        FwdItem wn = fwd_decode(meta, hd, blockIdx.x < n_items ? blockIdx.x : 0, hq, hkv);
         for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-            const FwdItem w = wn;                                      // decoded one item ahead
-            if (item + int(gridDim.x) < n_items) wn = fwd_decode(meta, hd, item + gridDim.x, hq, hkv);
+            const FwdItem w = fwd_decode(meta, hd, item, hq, hkv);
             const int n = qtile_nkv(w.t);
             if (!bwait(&sm.q_full, n_it & 1, abort_flag)) goto done;
             ++n_it;
@@ -201,7 +199,6 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 umma_commit(&sm.s_full[hs]);
             }
             umma_commit(&sm.k_empty[st]);
-            if (n == 1) umma_commit(&sm.q_empty);                      // Q feeds S only
             for (int j = 0; j < n; ++j) {
                 st = (kv_it + j) % FWD_STAGES;
                 const int st2 = (kv_it + j + 1) % FWD_STAGES;
@@ -222,8 +219,8 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
                 umma_commit(&sm.v_empty[st]);
                 if (have_next) umma_commit(&sm.k_empty[st2]);
-                if (j + 2 == n) umma_commit(&sm.q_empty);              // the item's last S is issued
             }
+            umma_commit(&sm.q_empty);
             kv_it += n;
             for (int hs = 0; hs < w.nh; ++hs) ++item_cnt[hs];
         }
@@ -235,29 +232,15 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const uint32_t t_s = tmem + (uint32_t(lane_base) << 16) + wg * 128;
         const uint32_t t_o = tmem + (uint32_t(lane_base) << 16) + 256 + wg * 128;
         uint32_t s_cnt = 0, pv_cnt = 0;
-        // The next item's tile is decoded at the start of this one and its rows' segment starts after this item's
-        // first tile, so no global load latency sits on the first step of an item.
-        auto seg_of = [&](const FwdItem &b) {
-            const int rr = b.t.row0 + rt;
-            return rr < b.t.gstart + b.t.glen ? seg_start[rr] : 0;
-        };
-        FwdItem wn = fwd_decode(meta, hd, blockIdx.x < n_items ? blockIdx.x : 0, hq, hkv);
-        int s0n = blockIdx.x < n_items ? seg_of(wn) : 0;
         for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-            const FwdItem w = wn;
-            const int s0 = s0n;
-            const int nxt = item + gridDim.x;
-            if (nxt < n_items) wn = fwd_decode(meta, hd, nxt, hq, hkv);
-            bool next_seg_pending = nxt < n_items;
-            if (wg >= w.nh) {
-                if (next_seg_pending) s0n = seg_of(wn);
-                continue;
-            }
+            const FwdItem w = fwd_decode(meta, hd, item, hq, hkv);
+            if (wg >= w.nh) continue;
             const int h = w.h0 + wg;
             const int n = qtile_nkv(w.t);
             const int row = w.t.row0 + rt;
             const int gend = w.t.gstart + w.t.glen;
             const bool in_group = row < gend;
+            const int s0 = in_group ? seg_start[row] : 0;
             const int pfx_end = w.t.gstart + w.t.plen;
             const int x0 = w.t.row0 - w.t.gstart;
             float m = -INFINITY, l = 0.f;
@@ -342,51 +325,34 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
                 tc_fence_before();
                 mbar_arrive(&sm.p_full[wg]);
-                if (next_seg_pending) {
-                    s0n = seg_of(wn);
-                    next_seg_pending = false;
-                }
             }
-            if (next_seg_pending) s0n = seg_of(wn);
-            // epilogue: O / l, LSE. All of O comes into registers first so the accumulator is released before the
-            // (row-per-thread) stores.
+            // epilogue: O / l, LSE
             if (!bwait(&sm.o_done[wg], (pv_cnt + n - 1) & 1, abort_flag)) goto done;
             pv_cnt += n;
             tc_fence_after();
             {
-                static_assert(D == 64 || D == 128, "head dim");
-                uint32_t r0[32], r1[32], r2[32], r3[32];
-                tmem_ld32(t_o, r0);
-                tmem_ld32(t_o + 32, r1);
-                if constexpr (D == 128) {
-                    tmem_ld32(t_o + 64, r2);
-                    tmem_ld32(t_o + 96, r3);
-                    tmem_wait_ld(r0, r1, r2, r3);
-                } else {
-                    tmem_wait_ld(r0, r1);
-                }
-                tc_fence_before();
-                mbar_arrive(&sm.o_free[wg]);
-                if (in_group) {
-                    const float inv_l = l > 0.f ? 1.f / l : 0.f;
-                    uint4 *dst = reinterpret_cast<uint4 *>(O + (int64_t(row) * hq + h) * D);
-                    auto put = [&](const uint32_t (&rr)[32], int c) {
+                const float inv_l = l > 0.f ? 1.f / l : 0.f;
+                __nv_bfloat16 *orow = O + (int64_t(row) * hq + h) * D;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t rr[32];
+                    tmem_ld32(t_o + c * 32, rr);
+                    tmem_wait_ld(rr);
+                    if (in_group) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            pk[e] = pack_bf16x2(__uint_as_float(rr[2 * e]) * inv_l,
+                                                __uint_as_float(rr[2 * e + 1]) * inv_l);
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            dst[4 * c + e] = make_uint4(
-                                pack_bf16x2(__uint_as_float(rr[8 * e]) * inv_l, __uint_as_float(rr[8 * e + 1]) * inv_l),
-                                pack_bf16x2(__uint_as_float(rr[8 * e + 2]) * inv_l, __uint_as_float(rr[8 * e + 3]) * inv_l),
-                                pack_bf16x2(__uint_as_float(rr[8 * e + 4]) * inv_l, __uint_as_float(rr[8 * e + 5]) * inv_l),
-                                pack_bf16x2(__uint_as_float(rr[8 * e + 6]) * inv_l, __uint_as_float(rr[8 * e + 7]) * inv_l));
-                    };
-                    put(r0, 0);
-                    put(r1, 1);
-                    if constexpr (D == 128) {
-                        put(r2, 2);
-                        put(r3, 3);
+                            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&sm.o_free[wg]);
             if (in_group) LSE[int64_t(h) * T + row] = (m + __log2f(l)) * 0.69314718055994531f;
         }
     }
