@@ -8,7 +8,8 @@ from ``workloads`` only.
 Every function restates the definition it follows; the pages it cites are
   * "Preference Packing: Efficient Preference Optimization for LLMs" (abstract and method digest),
   * "prefix_grouper_utils.py" (verl fork documentation: §1 building position ids, §2 building the grouper,
-    §3 forward, and its prefix-sharing diagram),
+    §3 forward including the split of the logits and the log-probabilities of the responses, and its
+    prefix-sharing diagram),
   * "PackInfer: Compute- and I/O-Efficient Attention for Batched LLM Inference" (abstract).
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py`` (brute force, closed forms, library
@@ -31,4 +32,9 @@ from .packed_attention import (  # noqa: F401
     tile_classes_bruteforce,
     unpacked_backward,
     unpacked_forward,
+)
+from .response_logprobs import (  # noqa: F401
+    response_logprobs,
+    response_logprobs_rows,
+    response_source_rows,
 )

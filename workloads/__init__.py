@@ -162,3 +162,30 @@ def make_inputs(name: str, prefix_lens, suffix_lens, seed: int | None = None, wi
         out[key] = _round_bf16(arr) if dt == "bf16" else torch.from_numpy(arr)
     out["scale_rows"] = scale_rows
     return out
+
+
+# Vocabulary of the response log-probability read-out: the pages name no model; 151,936 is the vocabulary size of
+# the Qwen2-family models that verl-based pipelines like the one on "prefix_grouper_utils.py" commonly train.
+LOGPROB_VOCAB = 151936
+LOGPROB_LOGIT_STD = 4.0
+
+
+def make_logits(prefix_lens, suffix_lens, vocab: int = LOGPROB_VOCAB, seed: int = 2001, dtype: str = "bf16",
+                std: float = LOGPROB_LOGIT_STD):
+    """Synthetic packed logits [T, vocab] ~ N(0, std^2) (rounded to bf16 unless dtype is "fp32") and token ids [T]
+    uniform in [0, vocab), both seeded. Returns (logits, token_ids) as CPU torch tensors (token ids int32).
+
+    Rows are drawn in blocks so that large T x vocab shapes do not need an fp32 copy of the whole array.
+    """
+    import torch
+    T = packed_total(prefix_lens, suffix_lens)
+    rng = np.random.default_rng(seed)
+    ids = torch.from_numpy(rng.integers(0, vocab, size=T).astype(np.int32))
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    logits = torch.empty((T, vocab), dtype=tdt)
+    block = max(1, (1 << 24) // max(vocab, 1))
+    for r0 in range(0, T, block):
+        r1 = min(T, r0 + block)
+        x = rng.standard_normal((r1 - r0, vocab), dtype=np.float32) * np.float32(std)
+        logits[r0:r1] = torch.from_numpy(x).to(tdt)
+    return logits, ids
