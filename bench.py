@@ -389,6 +389,61 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_logprobs(args):
+    """The response log-probability read-out on its own (the row after attention): one pp_response_logprobs call
+    per step over the packed logits of the workload's layout at a 151,936-entry vocabulary. HBM-bound: the
+    algorithmic bytes are one logits row per scored token, plus the token ids and the output."""
+    import torch
+    from shared_prefix_packed_b200 import PackedBatch, _lib
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    name = args.workload
+    P, S = W.group_lengths(name)
+    T = W.packed_total(P, S)
+    V = W.LOGPROB_VOCAB
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2001)
+    logits = (torch.randn(T, V, generator=gen, device=dev, dtype=torch.float32) * W.LOGPROB_LOGIT_STD).to(
+        torch.bfloat16)
+    ids = torch.randint(0, V, (T,), generator=gen, device=dev, dtype=torch.int32)
+    w = W.WORKLOADS[name]
+    batch = PackedBatch(P, S, w.num_heads_q, w.num_heads_kv, w.head_dim, device=dev)
+    out = torch.empty(T, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    # scored rows: every response token, except the first token of each non-empty response of a group with no prefix
+    scored = sum(sum(ss) - (sum(1 for x in ss if x > 0) if p == 0 else 0) for p, ss in zip(P, S))
+    nbytes = scored * V * 2 + T * 4 * 2
+    for _ in range(args.warmup):
+        batch.response_logprobs(logits, ids, 0.9, out=out, stream=stream)
+    _lib.pp_get_status(stream)
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for _ in range(args.steps):
+        batch.response_logprobs(logits, ids, 0.9, out=out, stream=stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    _lib.pp_get_status(stream)
+    ms = t0.elapsed_time(t1) / args.steps
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    peaks = load_peaks()
+    print(json.dumps({
+        "metric": "response log-prob read-out GB/s", "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{name} layout, T={T}, scored rows={scored}, vocab={V}, bf16 logits ~ N(0, 4^2)",
+                   "l2": f"logits {T * V * 2 / 2**30:.1f} GiB, larger than L2, no flush"},
+        "roofline": {"bound": "hbm", "kernel": "k_response_logprobs", "achieved": round(gbs, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                     "traffic": None, "peak_source": peaks["source"] + " hbm_gbs", "bytes_per_launch": nbytes},
+        "gpu_launches": args.steps, "clocks": clocks}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -399,10 +454,14 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--logprobs", action="store_true",
+                    help="time the response log-prob read-out (pp_response_logprobs) instead of the attention step")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.logprobs:
+        run_logprobs(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

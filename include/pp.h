@@ -175,6 +175,23 @@ PP_API pp_status pp_attn_bwd_noalloc(const void *q, const void *k, const void *v
                               float softmax_scale, void *dq, void *dk, void *dv, void *stream);
 
 /* ---------------------------------------------------------------------------------------------------------------
+ * pp_response_logprobs: log-probability of every response token under the packed logits (the read-out of
+ * "prefix_grouper_utils.py" section 3: split_output(logits, include_prefix_last=1) puts the group's last prefix row
+ * in front of each response's rows, the last row of each block is dropped, the rows are divided by the temperature,
+ * and the log-softmax is read at each completion token).
+ *   On the packed layout: the token at response row y is predicted by row y - 1, except a response's first token,
+ *   which is predicted by its group's last prefix row (o_g + P_g - 1). out[y] = x[src, id_y] / temperature -
+ *   ln sum_v exp(x[src, v] / temperature), computed in fp32 with one pass over the row.
+ *   logits: [T, V] row-major, dt PP_BF16 or PP_FP32, aligned to its element size (rows need not be 16-byte
+ *   aligned). token_ids: int32 [T], the packed input ids. meta_d from pp_build_meta for the same groups.
+ *   temperature > 0. out: fp32 [T]; prefix rows, and a response's first token in a group with P_g = 0 (no row
+ *   predicts it), get 0. All pointers are device pointers; nothing is allocated.
+ *   A token id outside [0, V) writes NaN at its row and sets PP_ERR_DEVICE_INPUT (reported by pp_get_status).
+ */
+PP_API pp_status pp_response_logprobs(const void *logits, pp_dtype dt, int64_t V, const int32_t *token_ids,
+                                      const void *meta_d, int64_t T, float temperature, float *out, void *stream);
+
+/* ---------------------------------------------------------------------------------------------------------------
  * pp_get_status: synchronises `stream`, then reads and clears this device's error word. Returns PP_OK,
  * PP_ERR_DEVICE_TIMEOUT, PP_ERR_DEVICE_INPUT or PP_ERR_CUDA (a sticky CUDA error is reported as such).
  */

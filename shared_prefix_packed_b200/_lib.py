@@ -42,6 +42,7 @@ SIGNATURES = {
                            _I64, _VP]),
     "pp_attn_bwd_noalloc": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _I32, _I32, _I32, _F32, _VP, _VP, _VP,
                                    _VP]),
+    "pp_response_logprobs": (_I32, [_VP, _I32, _I64, _VP, _VP, _I64, _F32, _VP, _VP]),
     "pp_get_status": (_I32, [_VP]),
     "pp_last_error": (ctypes.c_char_p, []),
     "pp_version": (ctypes.c_char_p, []),
@@ -146,6 +147,12 @@ def pp_attn_fwd(q, k, v, meta_d, o, lse, workspace, softmax_scale: float = 0.0, 
     _call("pp_attn_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(meta_d), T, hq, hkv, d, float(softmax_scale),
           _dtype_code(q), _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
           _stream(stream))
+
+
+def pp_response_logprobs(logits, token_ids, meta_d, out, temperature: float = 1.0, stream=None):
+    T, V = logits.shape
+    _call("pp_response_logprobs", _ptr(logits), _dtype_code(logits), V, _ptr(token_ids), _ptr(meta_d), T,
+          float(temperature), _ptr(out), _stream(stream))
 
 
 def pp_attn_bwd(q, k, v, o, lse, dout, meta_d, dq, dk, dv, workspace, softmax_scale: float = 0.0, stream=None):

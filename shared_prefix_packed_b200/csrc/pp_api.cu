@@ -18,6 +18,7 @@
 #include "pp_rope.cuh"
 #include "pp_attn_fwd.cuh"
 #include "pp_attn_bwd.cuh"
+#include "pp_logprobs.cuh"
 
 namespace {
 
@@ -257,6 +258,34 @@ pp_status pp_workspace_bytes(int32_t which, int64_t T, int32_t hq, int32_t hkv, 
     return PP_OK;
 }
 
+pp_status pp_response_logprobs(const void *logits, pp_dtype dt, int64_t V, const int32_t *token_ids,
+                               const void *meta_d, int64_t T, float temperature, float *out, void *stream) {
+    if (T < 0 || T >= (int64_t(1) << 31)) return fail(PP_ERR_INVALID_ARG, "T out of range (%lld)", (long long)T);
+    if (V < 1) return fail(PP_ERR_INVALID_ARG, "V must be >= 1 (got %lld)", (long long)V);
+    if (dt != PP_BF16 && dt != PP_FP32) return fail(PP_ERR_INVALID_ARG, "unknown dtype %d", int(dt));
+    if (!(temperature > 0.f) || std::isinf(temperature))
+        return fail(PP_ERR_INVALID_ARG, "temperature must be finite and > 0");
+    if (T == 0) return PP_OK;
+    if (!logits || !token_ids || !meta_d || !out) return fail(PP_ERR_INVALID_ARG, "NULL pointer argument");
+    if (reinterpret_cast<uintptr_t>(logits) % (dt == PP_BF16 ? 2 : 4))
+        return fail(PP_ERR_INVALID_ARG, "logits must be aligned to their element size");
+    DeviceInfo *di;
+    pp_status st;
+    if ((st = device_info(&di)) != PP_OK) return st;
+    const int grid = grid_for(di->sm_count, 8, T);
+    const float inv_temp = 1.f / temperature;
+    const float c2 = float(1.4426950408889634 / double(temperature));
+    cudaStream_t s = as_stream(stream);
+    if (dt == PP_BF16)
+        pp::k_response_logprobs<__nv_bfloat16><<<grid, pp::LP_THREADS, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(logits), V, token_ids, meta_d, c2, inv_temp, out);
+    else
+        pp::k_response_logprobs<float><<<grid, pp::LP_THREADS, 0, s>>>(static_cast<const float *>(logits), V,
+                                                                       token_ids, meta_d, c2, inv_temp, out);
+    PP_CUDA(cudaGetLastError());
+    return PP_OK;
+}
+
 pp_status pp_attn_fwd(const void *q, const void *k, const void *v, const void *meta_d, int64_t T, int32_t hq,
                       int32_t hkv, int32_t d, float softmax_scale, pp_dtype dt, void *o, float *lse,
                       void *workspace, int64_t ws_bytes, void *stream) {
@@ -365,7 +394,7 @@ pp_status pp_get_status(void *stream) {
     e = cudaMemcpyToSymbol(pp::g_dev_err, &zero, sizeof(zero));
     if (e != cudaSuccess) return fail(PP_ERR_CUDA, "clearing the device error word: %s", cudaGetErrorString(e));
     if (word & pp::DEVERR_TIMEOUT) return fail(PP_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait ran out (0x%x)", word);
-    return fail(PP_ERR_DEVICE_INPUT, "inconsistent descriptors or segment boundaries (0x%x)", word);
+    return fail(PP_ERR_DEVICE_INPUT, "inconsistent descriptors, segment boundaries or token ids (0x%x)", word);
 }
 
 }  // extern "C"

@@ -14,6 +14,7 @@ enum DevErr : int32_t {
     DEVERR_TIMEOUT = 1,
     DEVERR_BAD_SEGMENTS = 2,   // cu_seqlens not monotone / not from 0 to T
     DEVERR_BAD_GROUPS = 4,     // descriptors disagree with the segments
+    DEVERR_BAD_TOKEN = 8,      // a token id outside [0, V) given to pp_response_logprobs
 };
 
 __device__ int32_t g_dev_err;  // this device's error word, read and cleared by pp_get_status

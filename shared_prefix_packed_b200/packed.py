@@ -67,6 +67,12 @@ class PackedBatch:
         _lib.pp_attn_bwd(q, k, v, o, lse, dout, self.meta, dq, dk, dv, self.ws_bwd, softmax_scale, stream)
         return dq, dk, dv
 
+    def response_logprobs(self, logits, token_ids, temperature: float = 1.0, out=None, stream=None):
+        """Log-probability of every response token from the packed logits [T, V] (0 where no row predicts it)."""
+        lp = torch.empty(self.T, dtype=torch.float32, device=logits.device) if out is None else out
+        _lib.pp_response_logprobs(logits, token_ids, self.meta, lp, temperature, stream)
+        return lp
+
     def tiles(self, which: int, stream=None):
         """Expanded schedule as a sorted list of (q_row0, kv_row0, class) (test and inspection helper)."""
         count = torch.zeros(1, dtype=torch.int32, device=self.device)
