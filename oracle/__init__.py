@@ -7,7 +7,8 @@ from ``workloads`` only.
 
 Every function restates the definition it follows; the pages it cites are
   * "Preference Packing: Efficient Preference Optimization for LLMs" (abstract and method digest),
-  * "prefix_grouper_utils.py" (verl fork documentation: §1 building position ids, §2 building the grouper,
+  * "prefix_grouper_utils.py" (verl fork documentation: §1 building position ids, §2 building the grouper from a
+    micro-batch,
     §3 forward including the split of the logits and the log-probabilities of the responses, and its
     prefix-sharing diagram),
   * "PackInfer: Compute- and I/O-Efficient Attention for Batched LLM Inference" (abstract).
@@ -33,6 +34,7 @@ from .packed_attention import (  # noqa: F401
     unpacked_backward,
     unpacked_forward,
 )
+from .pack_batch import pack_batch  # noqa: F401
 from .response_logprobs import (  # noqa: F401
     response_logprobs,
     response_logprobs_rows,
