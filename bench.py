@@ -389,6 +389,70 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_pack(args):
+    """Device-side packing of an ungrouped micro-batch (pp_pack_batch, the step before the path) on the workload's
+    groups: every sample carries its group's prompt (left-padded to the longest prompt) and its own response
+    (right-padded), samples of a group share a uid. Tiny and launch-bound; bytes = the masks and ids read plus the
+    packed ids written."""
+    import torch
+    from shared_prefix_packed_b200 import _lib
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    name = args.workload
+    P, S = W.group_lengths(name)
+    rng = np.random.default_rng(4001)
+    samples = [(g, p, s) for g, (p, ss) in enumerate(zip(P, S)) for s in ss]
+    bs = len(samples)
+    Lp, Lr = max(P), max(s for _, _, s in samples)
+    prompts = np.zeros((bs, Lp), np.int32)
+    pm = np.zeros((bs, Lp), np.uint8)
+    responses = np.zeros((bs, Lr), np.int32)
+    rm = np.zeros((bs, Lr), np.uint8)
+    group_prompt = [rng.integers(0, W.LOGPROB_VOCAB, size=p) for p in P]
+    for i, (g, p, s) in enumerate(samples):
+        prompts[i, Lp - p:] = group_prompt[g]
+        pm[i, Lp - p:] = 1
+        responses[i, :s] = rng.integers(0, W.LOGPROB_VOCAB, size=s)
+        rm[i, :s] = 1
+    uids = np.array([g for g, _, _ in samples], np.int64)
+    t = lambda x: torch.from_numpy(x).to(dev)
+    d_p, d_pm, d_r, d_rm, d_u = t(prompts), t(pm), t(responses), t(rm), t(uids)
+    packed = torch.empty(bs * (Lp + Lr), dtype=torch.int32, device=dev)
+    groups = torch.empty(bs, 2, dtype=torch.int32, device=dev)
+    cu = torch.empty(2 * bs + 1, dtype=torch.int32, device=dev)
+    off = torch.empty(bs, 2, dtype=torch.int32, device=dev)
+    counts = torch.empty(3, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call = lambda: _lib.pp_pack_batch(d_p, d_pm, d_r, d_rm, d_u, packed, groups, cu, off, counts, stream)
+    for _ in range(args.warmup):
+        call()
+    _lib.pp_get_status(stream)
+    T = int(counts[2])
+    nbytes = bs * (Lp + Lr) * 5 + bs * 8 + T * 4 + (2 * bs + 1) * 4
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for _ in range(args.steps):
+        call()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / args.steps
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    peaks = load_peaks()
+    print(json.dumps({
+        "metric": "micro-batch packing GB/s", "value": round(gbs, 2), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int32", "data": "synthetic",
+        "config": {"workload": f"{name} groups as an ungrouped micro-batch: bs={bs}, Lp={Lp}, Lr={Lr}, T={T}",
+                   "note": "three launches per call; launch-latency bound at this size"},
+        "roofline": {"bound": "hbm", "kernel": "k_pack_count + k_pack_layout + k_pack_gather",
+                     "achieved": round(gbs, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs / peaks["hbm_gbs"], 5), "traffic": None,
+                     "peak_source": peaks["source"] + " hbm_gbs", "bytes_per_launch": nbytes},
+        "gpu_launches": 3 * args.steps}))
+
+
 def run_logprobs(args):
     """The response log-probability read-out on its own (the row after attention): one pp_response_logprobs call
     per step over the packed logits of the workload's layout at a 151,936-entry vocabulary. HBM-bound: the
@@ -454,12 +518,16 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--pack", action="store_true",
+                    help="time device-side packing of an ungrouped micro-batch (pp_pack_batch)")
     ap.add_argument("--logprobs", action="store_true",
                     help="time the response log-prob read-out (pp_response_logprobs) instead of the attention step")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.logprobs:
+    if args.pack:
+        run_pack(args)
+    elif args.logprobs:
         run_logprobs(args)
     elif args.impl == "reference":
         run_reference(args)

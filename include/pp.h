@@ -175,6 +175,26 @@ PP_API pp_status pp_attn_bwd_noalloc(const void *q, const void *k, const void *v
                               float softmax_scale, void *dq, void *dk, void *dv, void *stream);
 
 /* ---------------------------------------------------------------------------------------------------------------
+ * pp_pack_batch: pack an ungrouped micro-batch on the device ("prefix_grouper_utils.py" section 2, building the
+ * grouper from a micro-batch). Consecutive samples with equal uids form a group (a uid that reappears later starts a
+ * new group); the group's prefix is the valid prompt tokens of its first sample; the packed sequence is, group by
+ * group, the prefix followed by each sample's valid response tokens, in order, without padding.
+ *   prompts int32 [bs, Lp] and prompt_mask uint8 [bs, Lp]; responses int32 [bs, Lr] and response_mask uint8 [bs, Lr]
+ *   (nonzero mask = valid token; padding may be on either side); uids int64 [bs]. 0 <= bs <= 8192.
+ *   Outputs: packed_ids int32 [capacity >= bs * (Lp + Lr)] (first T written); groups pp_group_desc [bs] (first G
+ *   written: prefix_len, num_suffixes = group size); cu_seqlens int32 [2 * bs + 1] (first nseg + 1 written: each
+ *   group's prefix, then each response, empty segments kept; the layout pp_build_meta takes); sample_offsets
+ *   int32 [bs, 2] = (packed offset of the sample's prompt if it heads its group, else -1; packed offset of its
+ *   response); counts int32 [3] = {G, nseg = G + bs, T}. All device pointers; nothing is allocated.
+ *   The counts are device values: a caller reads them (a synchronising copy) to size and call pp_build_meta.
+ *   Errors: PP_ERR_INVALID_ARG (sizes, NULL pointers, capacity), PP_ERR_UNSUPPORTED (bs > 8192).
+ */
+PP_API pp_status pp_pack_batch(const int32_t *prompts, const uint8_t *prompt_mask, int32_t Lp, const int32_t *responses,
+                               const uint8_t *response_mask, int32_t Lr, const int64_t *uids, int32_t bs,
+                               int32_t *packed_ids, int64_t capacity, pp_group_desc *groups, int32_t *cu_seqlens,
+                               int32_t *sample_offsets, int32_t *counts, void *stream);
+
+/* ---------------------------------------------------------------------------------------------------------------
  * pp_response_logprobs: log-probability of every response token under the packed logits (the read-out of
  * "prefix_grouper_utils.py" section 3: split_output(logits, include_prefix_last=1) puts the group's last prefix row
  * in front of each response's rows, the last row of each block is dropped, the rows are divided by the temperature,

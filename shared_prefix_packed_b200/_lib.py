@@ -42,6 +42,7 @@ SIGNATURES = {
                            _I64, _VP]),
     "pp_attn_bwd_noalloc": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _I32, _I32, _I32, _F32, _VP, _VP, _VP,
                                    _VP]),
+    "pp_pack_batch": (_I32, [_VP, _VP, _I32, _VP, _VP, _I32, _VP, _I32, _VP, _I64, _VP, _VP, _VP, _VP, _VP]),
     "pp_response_logprobs": (_I32, [_VP, _I32, _I64, _VP, _VP, _I64, _F32, _VP, _VP]),
     "pp_get_status": (_I32, [_VP]),
     "pp_last_error": (ctypes.c_char_p, []),
@@ -147,6 +148,15 @@ def pp_attn_fwd(q, k, v, meta_d, o, lse, workspace, softmax_scale: float = 0.0, 
     _call("pp_attn_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(meta_d), T, hq, hkv, d, float(softmax_scale),
           _dtype_code(q), _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
           _stream(stream))
+
+
+def pp_pack_batch(prompts, prompt_mask, responses, response_mask, uids, packed_ids, groups, cu_seqlens,
+                  sample_offsets, counts, stream=None):
+    bs, Lp = prompts.shape
+    Lr = responses.shape[1]
+    _call("pp_pack_batch", _ptr(prompts), _ptr(prompt_mask), Lp, _ptr(responses), _ptr(response_mask), Lr, _ptr(uids),
+          bs, _ptr(packed_ids), packed_ids.numel(), _ptr(groups), _ptr(cu_seqlens), _ptr(sample_offsets),
+          _ptr(counts), _stream(stream))
 
 
 def pp_response_logprobs(logits, token_ids, meta_d, out, temperature: float = 1.0, stream=None):

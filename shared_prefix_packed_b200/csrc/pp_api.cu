@@ -19,6 +19,7 @@
 #include "pp_attn_fwd.cuh"
 #include "pp_attn_bwd.cuh"
 #include "pp_logprobs.cuh"
+#include "pp_pack.cuh"
 
 namespace {
 
@@ -255,6 +256,45 @@ pp_status pp_workspace_bytes(int32_t which, int64_t T, int32_t hq, int32_t hkv, 
     } else {
         return fail(PP_ERR_INVALID_ARG, "which must be fwd or bwd");
     }
+    return PP_OK;
+}
+
+pp_status pp_pack_batch(const int32_t *prompts, const uint8_t *prompt_mask, int32_t Lp, const int32_t *responses,
+                        const uint8_t *response_mask, int32_t Lr, const int64_t *uids, int32_t bs,
+                        int32_t *packed_ids, int64_t capacity, pp_group_desc *groups, int32_t *cu_seqlens,
+                        int32_t *sample_offsets, int32_t *counts, void *stream) {
+    if (bs < 0 || bs > pp::PACK_MAX_BATCH)
+        return fail(bs < 0 ? PP_ERR_INVALID_ARG : PP_ERR_UNSUPPORTED, "bs must be in [0, %d] (got %d)",
+                    pp::PACK_MAX_BATCH, bs);
+    if (Lp < 0 || Lr < 0) return fail(PP_ERR_INVALID_ARG, "negative row length");
+    const int64_t worst = int64_t(bs) * (int64_t(Lp) + Lr);
+    if (worst >= (int64_t(1) << 31)) return fail(PP_ERR_INVALID_ARG, "bs * (Lp + Lr) must fit int32");
+    if (capacity < worst) return fail(PP_ERR_INVALID_ARG, "packed_ids capacity %lld < bs * (Lp + Lr) = %lld",
+                                      (long long)capacity, (long long)worst);
+    if (!cu_seqlens || !counts) return fail(PP_ERR_INVALID_ARG, "NULL pointer argument");
+    cudaStream_t s = as_stream(stream);
+    if (bs == 0) {
+        PP_CUDA(cudaMemsetAsync(counts, 0, 3 * sizeof(int32_t), s));
+        PP_CUDA(cudaMemsetAsync(cu_seqlens, 0, sizeof(int32_t), s));
+        return PP_OK;
+    }
+    if (!uids || !groups || !sample_offsets || (worst > 0 && !packed_ids) || (Lp > 0 && (!prompts || !prompt_mask)) ||
+        (Lr > 0 && (!responses || !response_mask)))
+        return fail(PP_ERR_INVALID_ARG, "NULL pointer argument");
+    DeviceInfo *di;
+    pp_status st;
+    if ((st = device_info(&di)) != PP_OK) return st;
+    pp::k_pack_count<<<bs, pp::PACK_THREADS, 0, s>>>(prompt_mask, Lp, response_mask, Lr, sample_offsets);
+    PP_CUDA(cudaGetLastError());
+    const int smem = 4 * bs * int(sizeof(int32_t));
+    PP_CUDA(cudaFuncSetAttribute(pp::k_pack_layout, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    pp::k_pack_layout<<<1, pp::PACK_LAYOUT_THREADS, smem, s>>>(uids, bs, sample_offsets,
+                                                               reinterpret_cast<int32_t *>(groups), cu_seqlens,
+                                                               counts);
+    PP_CUDA(cudaGetLastError());
+    pp::k_pack_gather<<<bs, pp::PACK_THREADS, 0, s>>>(prompts, prompt_mask, Lp, responses, response_mask, Lr,
+                                                      sample_offsets, packed_ids);
+    PP_CUDA(cudaGetLastError());
     return PP_OK;
 }
 

@@ -82,3 +82,31 @@ class PackedBatch:
         _lib.pp_meta_tiles(self.meta, which, buf, count, stream)
         rows = buf[: 3 * n].view(-1, 3).cpu().tolist()
         return sorted(tuple(r) for r in rows)
+
+
+def pack_batch(prompts, prompt_mask, responses, response_mask, uids, stream=None):
+    """Pack an ungrouped micro-batch on the device (pp_pack_batch): returns (packed_ids [T], prefix_lens,
+    suffix_lens, cu_seqlens [nseg + 1], sample_offsets [bs, 2]). The lengths come back to the host with one small
+    synchronising copy, so they can be handed to PackedBatch."""
+    dev = prompts.device
+    bs, Lp = prompts.shape
+    Lr = responses.shape[1]
+    packed = torch.empty(max(1, bs * (Lp + Lr)), dtype=torch.int32, device=dev)
+    groups = torch.empty(max(1, bs), 2, dtype=torch.int32, device=dev)
+    cu = torch.empty(2 * bs + 1, dtype=torch.int32, device=dev)
+    offsets = torch.empty(max(1, bs), 2, dtype=torch.int32, device=dev)
+    counts = torch.zeros(3, dtype=torch.int32, device=dev)
+    _lib.pp_pack_batch(prompts.to(torch.int32), prompt_mask.to(torch.uint8), responses.to(torch.int32),
+                       response_mask.to(torch.uint8), uids.to(torch.int64), packed, groups, cu, offsets, counts,
+                       stream)
+    G, nseg, T = (int(x) for x in counts.cpu())
+    g = groups[:G].cpu().tolist()
+    P = [int(p) for p, _ in g]
+    sizes = [int(k) for _, k in g]
+    cu_h = cu[:nseg + 1]
+    lens = (cu_h[1:] - cu_h[:-1]).cpu().tolist()
+    S, seg = [], 0
+    for k in sizes:
+        S.append([int(x) for x in lens[seg + 1:seg + 1 + k]])
+        seg += 1 + k
+    return packed[:T], P, S, cu_h, offsets[:bs]
