@@ -465,7 +465,7 @@ def run_logprobs(args):
     name = args.workload
     P, S = W.group_lengths(name)
     T = W.packed_total(P, S)
-    V = W.LOGPROB_VOCAB
+    V = args.vocab
     gen = torch.Generator(device=dev)
     gen.manual_seed(2001)
     logits = (torch.randn(T, V, generator=gen, device=dev, dtype=torch.float32) * W.LOGPROB_LOGIT_STD).to(
@@ -518,6 +518,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--vocab", type=int, default=W.LOGPROB_VOCAB, help="vocabulary of the --logprobs read-out")
     ap.add_argument("--pack", action="store_true",
                     help="time device-side packing of an ungrouped micro-batch (pp_pack_batch)")
     ap.add_argument("--logprobs", action="store_true",
