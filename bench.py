@@ -504,7 +504,9 @@ def run_logprobs(args):
                    "l2": f"logits {T * V * 2 / 2**30:.1f} GiB, larger than L2, no flush"},
         "roofline": {"bound": "hbm", "kernel": "k_response_logprobs", "achieved": round(gbs, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                     "traffic": None, "peak_source": peaks["source"] + " hbm_gbs", "bytes_per_launch": nbytes},
+                     "traffic": recorded_traffic(["k_response_logprobs"]) if V == W.LOGPROB_VOCAB and
+                     name == "dpo" else None,
+                     "peak_source": peaks["source"] + " hbm_gbs", "bytes_per_launch": nbytes},
         "gpu_launches": args.steps, "clocks": clocks}))
 
 
