@@ -494,10 +494,13 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     for (int e = 0; e < 32; ++e) { sr[e] = a0[e]; sr[32 + e] = a1[e]; }
                 }
                 if (all_in) {
+                    const float2 sl2v = make_float2(sl2, sl2);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        pk[e] = pack_bf16x2(ex2_approx(__uint_as_float(sr[2 * e]) * sl2),
-                                            ex2_approx(__uint_as_float(sr[2 * e + 1]) * sl2));
+                    for (int e = 0; e < 32; ++e) {
+                        const float2 x = fmul2(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
+                                               sl2v);
+                        pk[e] = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
+                    }
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
@@ -538,11 +541,13 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         for (int e = 0; e < 32; ++e) { pr[e] = a0[e]; pr[32 + e] = a1[e]; }
                     }
                     uint32_t t0[16], t1[16];
+                    const float2 sc = make_float2(scale, scale);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const uint32_t p = pk[e];
-                        const uint32_t dd = pack_bf16x2(bf16lo(p) * __uint_as_float(pr[2 * e]) * scale,
-                                                        bf16hi(p) * __uint_as_float(pr[2 * e + 1]) * scale);
+                        const float2 ds = fmul2(fmul2(make_float2(bf16lo(p), bf16hi(p)), sc),
+                                                make_float2(__uint_as_float(pr[2 * e]), __uint_as_float(pr[2 * e + 1])));
+                        const uint32_t dd = pack_bf16x2(ds.x, ds.y);
                         if (e < 16) t0[e] = dd; else t1[e - 16] = dd;
                     }
                     tmem_st16(tmem + lane_off + COL_DP + cb, t0);

@@ -300,11 +300,14 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     tmem_wait_ld(a0);
                     tc_fence_before();
                     mbar_arrive(&sm.s_free);
+                    const float2 sl2v = make_float2(sl2, sl2), c0v = make_float2(c0, c0);
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const int c = 2 * e;
-                        float p0 = ex2_approx(fmaf(__uint_as_float(a0[c]), sl2, c0));
-                        float p1 = ex2_approx(fmaf(__uint_as_float(a0[c + 1]), sl2, c0));
+                        const float2 x = ffma2(make_float2(__uint_as_float(a0[c]), __uint_as_float(a0[c + 1])), sl2v,
+                                               c0v);
+                        float p0 = ex2_approx(x.x);
+                        float p1 = ex2_approx(x.y);
                         if (cls != TILE_FULL) {
                             if (!(c <= lim_diag && (c < lim_pfx || c >= lim_seg))) p0 = 0.f;
                             if (!(c + 1 <= lim_diag && (c + 1 < lim_pfx || c + 1 >= lim_seg))) p1 = 0.f;
@@ -327,11 +330,15 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     tmem_ld32(tmem + lane_off + cdp + cb, a0);
                     tmem_wait_ld(a0);
                     uint32_t d0[16];
+                    const float2 dv = make_float2(lv.y, lv.y), sc = make_float2(scale, scale);
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const uint32_t p = pk[e];
-                        d0[e] = pack_bf16x2(bf16lo(p) * (__uint_as_float(a0[2 * e]) + lv.y) * scale,
-                                            bf16hi(p) * (__uint_as_float(a0[2 * e + 1]) + lv.y) * scale);
+                        const float2 ps = fmul2(make_float2(bf16lo(p), bf16hi(p)), sc);
+                        const float2 dp = fadd2(make_float2(__uint_as_float(a0[2 * e]), __uint_as_float(a0[2 * e + 1])),
+                                                dv);
+                        const float2 ds = fmul2(ps, dp);
+                        d0[e] = pack_bf16x2(ds.x, ds.y);
                     }
                     tmem_st16(tmem + lane_off + cdp + cb, d0);
                     tmem_wait_st();

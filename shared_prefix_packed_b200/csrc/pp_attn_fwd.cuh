@@ -278,7 +278,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
                 float m4[4] = {s[0], s[1], s[2], s[3]};                 // four independent max chains
 #pragma unroll
-                for (int c = 4; c < FWD_BN; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+                for (int c = 4; c < FWD_BN; c += 2) m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], s[c], s[c + 1]);
                 const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
                 const float mt = mx * sl2;
                 bool rescale = false;
@@ -292,20 +292,23 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     m = mt;
                 }
                 const float mu = (m == -INFINITY) ? 0.f : m;
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};                      // four independent sum chains
+                // scale/shift and row sum on packed fp32 pairs (one instruction per pair)
+                float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // two independent pair chains
+                const float2 sl2v = make_float2(sl2, sl2), nmu = make_float2(-mu, -mu);
 #pragma unroll
                 for (int c = 0; c < FWD_BN / 32; ++c) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * e], sl2, -mu));
-                        const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * e + 1], sl2, -mu));
-                        ls[e & 3] += p0 + p1;
+                        const float2 x = ffma2(make_float2(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]), sl2v, nmu);
+                        const float p0 = ex2_approx(x.x);
+                        const float p1 = ex2_approx(x.y);
+                        ls[e & 1] = fadd2(ls[e & 1], make_float2(p0, p1));
                         pk[e] = pack_bf16x2(p0, p1);
                     }
                     tmem_st16(t_s + c * 16, pk);
                 }
-                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+                l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
                 tmem_wait_st();
                 // tcgen05.ld/st are warp-collective: the whole warp takes the rescale path if any row needs it
                 if (__any_sync(0xffffffffu, rescale)) {
