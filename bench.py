@@ -424,6 +424,59 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_decode(args):
+    """One decoding step of every response over the workload's layout as a group-contiguous KV cache
+    (pp_decode_attn): one query per response (its newest token), 32/8 heads, d = 128. HBM-bound; the algorithmic
+    bytes are the cache read once (a prefix serves all responses of its group) plus the queries and outputs."""
+    import torch
+    from shared_prefix_packed_b200 import PackedBatch, _lib
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    name = args.workload
+    P, S = W.group_lengths(name)
+    w = W.WORKLOADS[name]
+    hq, hkv, d = w.num_heads_q, w.num_heads_kv, w.head_dim
+    T = W.packed_total(P, S)
+    n_resp = sum(len(ss) for ss in S)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(3001)
+    k = torch.randn(T, hkv, d, generator=gen, device=dev).to(torch.bfloat16)
+    v = torch.randn(T, hkv, d, generator=gen, device=dev).to(torch.bfloat16)
+    q = torch.randn(n_resp, hq, d, generator=gen, device=dev).to(torch.bfloat16)
+    batch = PackedBatch(P, S, hq, hkv, d, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(hq, n_resp, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    nbytes = 2 * T * hkv * d * 2 + 2 * n_resp * hq * d * 2 + n_resp * hq * 4
+    unpacked = sum((p + s) * hkv * d * 2 * 2 for p, ss in zip(P, S) for s in ss)
+    for _ in range(args.warmup):
+        batch.decode(q, k, v, out=o, lse=lse, stream=stream)
+    _lib.pp_get_status(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for _ in range(args.steps):
+        batch.decode(q, k, v, out=o, lse=lse, stream=stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / args.steps
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    peaks = load_peaks()
+    print(json.dumps({
+        "metric": "decode step over a group-contiguous KV cache GB/s", "value": round(gbs, 1), "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{name} layout as the KV cache: T={T}, {n_resp} responses, {hq}/{hkv} heads, d={d}",
+                   "cache_bytes_read_once": 2 * T * hkv * d * 2,
+                   "cache_bytes_if_unpacked": unpacked,
+                   "l2": f"K/V cache {2 * T * hkv * d * 2 / 2**20:.0f} MiB, larger than L2, no flush"},
+        "roofline": {"bound": "hbm", "kernel": "k_dec_plan + k_dec_partial + k_dec_combine", "achieved": round(gbs, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                     "traffic": None, "peak_source": peaks["source"] + " hbm_gbs", "bytes_per_launch": nbytes},
+        "gpu_launches": 3 * args.steps}))
+
+
 def run_pack(args):
     """Device-side packing of an ungrouped micro-batch (pp_pack_batch, the step before the path) on the workload's
     groups: every sample carries its group's prompt (left-padded to the longest prompt) and its own response
@@ -556,6 +609,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--vocab", type=int, default=W.LOGPROB_VOCAB, help="vocabulary of the --logprobs read-out")
+    ap.add_argument("--decode", action="store_true",
+                    help="time one decoding step over the workload's layout as a KV cache (pp_decode_attn)")
     ap.add_argument("--pack", action="store_true",
                     help="time device-side packing of an ungrouped micro-batch (pp_pack_batch)")
     ap.add_argument("--logprobs", action="store_true",
@@ -563,7 +618,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.pack:
+    if args.decode:
+        run_decode(args)
+    elif args.pack:
         run_pack(args)
     elif args.logprobs:
         run_logprobs(args)

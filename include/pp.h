@@ -175,6 +175,29 @@ PP_API pp_status pp_attn_bwd_noalloc(const void *q, const void *k, const void *v
                               float softmax_scale, void *dq, void *dk, void *dv, void *stream);
 
 /* ---------------------------------------------------------------------------------------------------------------
+ * pp_decode_attn: one decoding step of every response over a group-contiguous KV cache.
+ * The cache holds the packed layout of pp_build_meta (each group's prefix rows, then each response's rows), the
+ * newest token of each response last. Each response has one query (its newest token), which attends to its group's
+ * prefix and its own rows, the packed mask at the response's last row ("PackInfer" abstract: group-contiguous KV
+ * and attention over packed query-key regions; "Preference Packing": the prompt is shared by its responses).
+ * A prefix chunk is read from HBM once per group and serves all of the group's responses (flash-decoding in
+ * 64-key chunks, fp32 partials combined per query).
+ *   q: [n_resp, hq, d] bf16, n_resp = num_segments - num_groups (responses in packed order). k_cache, v_cache:
+ *   [T, hkv, d] bf16. groups_d, cu_d: the device descriptors and segment bounds of the cache (as for
+ *   pp_build_meta; every response of nonzero length has its query's K/V as its last row). d = 128.
+ *   o: [n_resp, hq, d] bf16; lse: [hq, n_resp] fp32 (natural log); a response with no keys gets 0 and -inf.
+ *   workspace: ws_bytes >= pp_decode_workspace_bytes for the same descriptors, 256-byte aligned. Descriptors that
+ *   disagree with T, num_segments or the sized workspace set PP_ERR_DEVICE_INPUT and yield NaN outputs.
+ */
+PP_API pp_status pp_decode_workspace_bytes(const pp_group_desc *groups_host, int32_t num_groups,
+                                           const int32_t *cu_seqlens_host, int32_t num_segments, int32_t num_heads_q,
+                                           int64_t *bytes);
+PP_API pp_status pp_decode_attn(const void *q, const void *k_cache, const void *v_cache, const pp_group_desc *groups_d,
+                                int32_t num_groups, const int32_t *cu_seqlens_d, int32_t num_segments, int64_t T,
+                                int32_t hq, int32_t hkv, int32_t d, float softmax_scale, void *o, float *lse,
+                                void *workspace, int64_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------------------------------------------
  * pp_pack_batch: pack an ungrouped micro-batch on the device ("prefix_grouper_utils.py" section 2, building the
  * grouper from a micro-batch). Consecutive samples with equal uids form a group (a uid that reappears later starts a
  * new group); the group's prefix is the valid prompt tokens of its first sample; the packed sequence is, group by

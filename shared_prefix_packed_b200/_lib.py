@@ -42,6 +42,9 @@ SIGNATURES = {
                            _I64, _VP]),
     "pp_attn_bwd_noalloc": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _I32, _I32, _I32, _F32, _VP, _VP, _VP,
                                    _VP]),
+    "pp_decode_workspace_bytes": (_I32, [_VP, _I32, _VP, _I32, _I32, _I64P]),
+    "pp_decode_attn": (_I32, [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _I64, _I32, _I32, _I32, _F32, _VP, _VP, _VP, _I64,
+                              _VP]),
     "pp_pack_batch": (_I32, [_VP, _VP, _I32, _VP, _VP, _I32, _VP, _I32, _VP, _I64, _VP, _VP, _VP, _VP, _VP]),
     "pp_response_logprobs": (_I32, [_VP, _I32, _I64, _VP, _VP, _I64, _F32, _VP, _VP]),
     "pp_get_status": (_I32, [_VP]),
@@ -148,6 +151,24 @@ def pp_attn_fwd(q, k, v, meta_d, o, lse, workspace, softmax_scale: float = 0.0, 
     _call("pp_attn_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(meta_d), T, hq, hkv, d, float(softmax_scale),
           _dtype_code(q), _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
           _stream(stream))
+
+
+def pp_decode_workspace_bytes(groups_host, cu_host, hq: int) -> int:
+    """groups_host: int32 [G, 2] CPU tensor; cu_host: int32 [nseg + 1] CPU tensor."""
+    out = ctypes.c_int64(0)
+    g = groups_host.contiguous()
+    c = cu_host.contiguous()
+    _call("pp_decode_workspace_bytes", ctypes.c_void_p(g.data_ptr()), g.shape[0], ctypes.c_void_p(c.data_ptr()),
+          c.numel() - 1, hq, ctypes.byref(out))
+    return out.value
+
+
+def pp_decode_attn(q, k_cache, v_cache, groups_d, cu_d, o, lse, workspace, softmax_scale: float = 0.0, stream=None):
+    T, hkv, d = k_cache.shape
+    hq = q.shape[1]
+    _call("pp_decode_attn", _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(groups_d), groups_d.shape[0], _ptr(cu_d),
+          cu_d.numel() - 1, T, hq, hkv, d, float(softmax_scale), _ptr(o), _ptr(lse), _ptr(workspace),
+          workspace.numel() * workspace.element_size(), _stream(stream))
 
 
 def pp_pack_batch(prompts, prompt_mask, responses, response_mask, uids, packed_ids, groups, cu_seqlens,

@@ -20,6 +20,7 @@
 #include "pp_attn_bwd.cuh"
 #include "pp_logprobs.cuh"
 #include "pp_pack.cuh"
+#include "pp_decode.cuh"
 
 namespace {
 
@@ -256,6 +257,75 @@ pp_status pp_workspace_bytes(int32_t which, int64_t T, int32_t hq, int32_t hkv, 
     } else {
         return fail(PP_ERR_INVALID_ARG, "which must be fwd or bwd");
     }
+    return PP_OK;
+}
+
+// Exact (chunk, query) pair count of the decode plan, from host copies of the descriptors and segment bounds.
+static pp_status decode_pairs(const pp_group_desc *groups, int32_t G, const int32_t *cu, int32_t nseg, int64_t *pairs) {
+    int64_t np = 0;
+    int32_t s = 0;
+    auto nch = [&](int32_t seg) -> int64_t {
+        const int64_t len = int64_t(cu[seg + 1]) - cu[seg];
+        return len > 0 ? (len + pp::DEC_CH - 1) / pp::DEC_CH : 0;
+    };
+    for (int32_t g = 0; g < G; ++g) {
+        const int32_t k = groups[g].num_suffixes;
+        if (k < 0 || s + 1 + int64_t(k) > nseg) return fail(PP_ERR_INVALID_ARG, "descriptors exceed num_segments");
+        np += nch(s) * k;
+        for (int32_t i = 0; i < k; ++i) np += nch(s + 1 + i);
+        s += 1 + k;
+    }
+    if (s != nseg) return fail(PP_ERR_INVALID_ARG, "num_segments must equal sum_g (1 + k_g)");
+    *pairs = np;
+    return PP_OK;
+}
+
+pp_status pp_decode_workspace_bytes(const pp_group_desc *groups_host, int32_t G, const int32_t *cu_host, int32_t nseg,
+                                    int32_t hq, int64_t *bytes) {
+    if (!groups_host || !cu_host || !bytes) return fail(PP_ERR_INVALID_ARG, "NULL pointer argument");
+    if (G < 1 || nseg < G || hq < 1) return fail(PP_ERR_INVALID_ARG, "need G >= 1, num_segments >= G, hq >= 1");
+    int64_t np;
+    pp_status st = decode_pairs(groups_host, G, cu_host, nseg, &np);
+    if (st != PP_OK) return st;
+    *bytes = pp::dec_plan_layout(cu_host[nseg], G, nseg, hq, np).total;
+    return PP_OK;
+}
+
+pp_status pp_decode_attn(const void *q, const void *k_cache, const void *v_cache, const pp_group_desc *groups_d,
+                         int32_t G, const int32_t *cu_d, int32_t nseg, int64_t T, int32_t hq, int32_t hkv, int32_t d,
+                         float softmax_scale, void *o, float *lse, void *workspace, int64_t ws_bytes, void *stream) {
+    pp_status st = check_heads(T, hq, hkv, d);
+    if (st != PP_OK) return st;
+    if (d != pp::DEC_D) return fail(PP_ERR_UNSUPPORTED, "decode supports head dim 128 only (got %d)", d);
+    if (G < 1 || nseg < G) return fail(PP_ERR_INVALID_ARG, "need G >= 1 and num_segments >= G");
+    const int32_t n_resp = nseg - G;
+    if (n_resp == 0) return PP_OK;
+    if (!q || !k_cache || !v_cache || !groups_d || !cu_d || !o || !lse || !workspace)
+        return fail(PP_ERR_INVALID_ARG, "NULL pointer argument");
+    const void *ptrs[4] = {q, k_cache, v_cache, o};
+    for (const void *ptr : ptrs)
+        if (reinterpret_cast<uintptr_t>(ptr) % 16) return fail(PP_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(PP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const pp::DecPlan base = pp::dec_plan_layout(T, G, nseg, hq, 0);
+    const int64_t rec = 4 * int64_t(hq) * (pp::DEC_D + 2);
+    if (ws_bytes < base.off_part + rec) return fail(PP_ERR_WORKSPACE, "workspace too small for the decode plan");
+    const pp::DecPlan p = pp::dec_plan_layout(T, G, nseg, hq, (ws_bytes - base.off_part) / rec);
+    DeviceInfo *di;
+    if ((st = device_info(&di)) != PP_OK) return st;
+    const float scale = softmax_scale == 0.f ? 1.f / std::sqrt(float(d)) : softmax_scale;
+    cudaStream_t s = as_stream(stream);
+    const int32_t *gd = reinterpret_cast<const int32_t *>(groups_d);
+    pp::k_dec_plan<<<1, 1024, 0, s>>>(gd, G, cu_d, nseg, T, workspace, p);
+    PP_CUDA(cudaGetLastError());
+    PP_CUDA(cudaFuncSetAttribute(pp::k_dec_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, pp::DEC_SMEM));
+    pp::k_dec_partial<<<di->sm_count, pp::DEC_THREADS, pp::DEC_SMEM, s>>>(
+        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k_cache),
+        static_cast<const __nv_bfloat16 *>(v_cache), gd, G, cu_d, nseg, hq, hkv, scale * 1.4426950408889634f,
+        workspace, p);
+    PP_CUDA(cudaGetLastError());
+    pp::k_dec_combine<<<grid_for(di->sm_count, 16, int64_t(n_resp) * hq), pp::DEC_D, 0, s>>>(
+        gd, G, cu_d, nseg, hq, n_resp, workspace, p, static_cast<__nv_bfloat16 *>(o), lse);
+    PP_CUDA(cudaGetLastError());
     return PP_OK;
 }
 
