@@ -34,6 +34,7 @@ from .packed_attention import (  # noqa: F401
     unpacked_backward,
     unpacked_forward,
 )
+from .batcher import plan_batches  # noqa: F401
 from .pack_batch import pack_batch  # noqa: F401
 from .response_logprobs import (  # noqa: F401
     response_logprobs,
