@@ -424,6 +424,66 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_batcher(args):
+    """The host batch planner (pp_plan_batches) and the work model behind "packing combines with batch sorting".
+
+    Throughput: plans per second over one million synthetic groups (host code, host clock). Work model, on 20,000
+    synthetic groups with the dpo length distribution (P ~ U[512, 2048], two responses ~ U[128, 1024]): the tokens
+    and causal attention pairs a padded implementation processes with 8 groups per batch, for
+      baseline   one sequence per (prompt, response), dataset order, padded to the batch's longest;
+      sorted     the same with the groups sorted by length first;
+      packed     one sequence per group (prompt once, then its responses), dataset order, padded;
+      packed+sorted,
+    and the pad-free packed form these kernels run (capacity batches from pp_plan_batches, no padding, only the
+    allowed pairs of the packed mask)."""
+    from shared_prefix_packed_b200 import pp_plan_batches
+
+    rng = np.random.default_rng(5001)
+    n_big = 1_000_000
+    toks = rng.integers(512, 2049, size=n_big) + rng.integers(128, 1025, size=(n_big, 2)).sum(axis=1)
+    pp_plan_batches(toks[:1000], 65536, True)
+    t0 = time.perf_counter()
+    for _ in range(3):
+        pp_plan_batches(toks, 65536, True)
+    plan_s = (time.perf_counter() - t0) / 3
+
+    n = 20000
+    P = rng.integers(512, 2049, size=n)
+    Sr = rng.integers(128, 1025, size=(n, 2))
+    B = 8                                                     # groups per padded batch
+
+    def padded(lengths_per_group, order):
+        tok = pairs = 0
+        for b0 in range(0, n, B):
+            seqs = [L for g in order[b0:b0 + B] for L in lengths_per_group[g]]
+            mx = max(seqs)
+            tok += len(seqs) * mx
+            pairs += len(seqs) * mx * (mx + 1) // 2
+        return tok, pairs
+
+    unpacked = [[int(P[g] + Sr[g, 0]), int(P[g] + Sr[g, 1])] for g in range(n)]
+    packed = [[int(P[g] + Sr[g].sum())] for g in range(n)]
+    ident = list(range(n))
+    by_unp = sorted(ident, key=lambda g: -max(unpacked[g]))
+    by_pk = sorted(ident, key=lambda g: -packed[g][0])
+    rows = {"baseline": padded(unpacked, ident), "sorted": padded(unpacked, by_unp),
+            "packed": padded(packed, ident), "packed+sorted": padded(packed, by_pk)}
+    useful_tok = int(P.sum() + Sr.sum())
+    useful_pairs = int(sum(p * (p + 1) // 2 + sum(s * p + s * (s + 1) // 2 for s in Sr[g]) for g, p in enumerate(P)))
+    order, batch, nb = pp_plan_batches([packed[g][0] for g in range(n)], 65536, True)
+    rows["pad-free packed (these kernels)"] = (useful_tok, useful_pairs)
+    base_tok, base_pairs = rows["baseline"]
+    model = {k: {"tokens": v[0], "attention_pairs": v[1], "token_speedup": round(base_tok / v[0], 3),
+                 "attention_speedup": round(base_pairs / v[1], 3)} for k, v in rows.items()}
+    print(json.dumps({
+        "metric": "host batch planning groups/s", "value": round(n_big / plan_s, 1), "unit": "groups/s",
+        "n_gpus": 0, "steps": 3, "warmup": 1, "ms_per_step": round(plan_s * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int64", "data": "synthetic",
+        "config": {"workload": f"{n_big} groups of the dpo length mix, capacity 65,536 tokens, sorted",
+                   "model_groups": n, "model_batch_groups": B, "pad_free_batches": nb},
+        "modeled_work": model}))
+
+
 def run_decode(args):
     """One decoding step of every response over the workload's layout as a group-contiguous KV cache
     (pp_decode_attn): one query per response (its newest token), 32/8 heads, d = 128. HBM-bound; the algorithmic
@@ -609,6 +669,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--vocab", type=int, default=W.LOGPROB_VOCAB, help="vocabulary of the --logprobs read-out")
+    ap.add_argument("--batcher", action="store_true",
+                    help="host batch planner throughput and the modeled work of packing with batch sorting")
     ap.add_argument("--decode", action="store_true",
                     help="time one decoding step over the workload's layout as a KV cache (pp_decode_attn)")
     ap.add_argument("--pack", action="store_true",
@@ -618,7 +680,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.decode:
+    if args.batcher:
+        run_batcher(args)
+    elif args.decode:
         run_decode(args)
     elif args.pack:
         run_pack(args)

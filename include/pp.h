@@ -235,6 +235,19 @@ PP_API pp_status pp_response_logprobs(const void *logits, pp_dtype dt, int64_t V
                                       const void *meta_d, int64_t T, float temperature, float *out, void *stream);
 
 /* ---------------------------------------------------------------------------------------------------------------
+ * pp_plan_batches (host only): plan training batches of packed preference groups ("Preference Packing" abstract and
+ * method digest: packing combined with batch sorting, batch size following the lengths). A group costs its packed
+ * length group_tokens[g] (P_g + sum of its response lengths). With sort_by_length != 0 the groups are taken longest
+ * first (stable: ties keep their input order), otherwise in input order; batches are filled greedily in that order
+ * up to token_capacity tokens; a group longer than the capacity forms a batch of its own.
+ *   group_tokens: int64 [num_groups] (host, >= 0). order: int32 [num_groups] out, the groups in batch order.
+ *   batch_of_group: int32 [num_groups] out. *num_batches out. token_capacity >= 1.
+ *   Errors: PP_ERR_INVALID_ARG (no message is recorded for this call; it touches no device state).
+ */
+PP_API pp_status pp_plan_batches(const int64_t *group_tokens, int32_t num_groups, int64_t token_capacity,
+                                 int32_t sort_by_length, int32_t *order, int32_t *batch_of_group, int32_t *num_batches);
+
+/* ---------------------------------------------------------------------------------------------------------------
  * pp_get_status: synchronises `stream`, then reads and clears this device's error word. Returns PP_OK,
  * PP_ERR_DEVICE_TIMEOUT, PP_ERR_DEVICE_INPUT or PP_ERR_CUDA (a sticky CUDA error is reported as such).
  */

@@ -42,6 +42,7 @@ SIGNATURES = {
                            _I64, _VP]),
     "pp_attn_bwd_noalloc": (_I32, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _I32, _I32, _I32, _F32, _VP, _VP, _VP,
                                    _VP]),
+    "pp_plan_batches": (_I32, [_VP, _I32, _I64, _I32, _VP, _VP, _VP]),
     "pp_decode_workspace_bytes": (_I32, [_VP, _I32, _VP, _I32, _I32, _I64P]),
     "pp_decode_attn": (_I32, [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _I64, _I32, _I32, _I32, _F32, _VP, _VP, _VP, _I64,
                               _VP]),
@@ -151,6 +152,24 @@ def pp_attn_fwd(q, k, v, meta_d, o, lse, workspace, softmax_scale: float = 0.0, 
     _call("pp_attn_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(meta_d), T, hq, hkv, d, float(softmax_scale),
           _dtype_code(q), _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
           _stream(stream))
+
+
+def pp_plan_batches(group_tokens, capacity: int, sort_by_length: bool = True):
+    """Host-side batch plan (see pp.h): returns (order, batch_of_group, n_batches) as a list, a list and an int."""
+    import numpy as np
+    toks = np.ascontiguousarray(np.asarray(group_tokens, dtype=np.int64))
+    if toks.ndim != 1 or (toks.size and toks.min() < 0) or int(capacity) < 1:
+        raise ValueError("group_tokens must be a 1-D array of non-negative counts and capacity >= 1")
+    G = toks.size
+    order = np.zeros(max(G, 1), dtype=np.int32)
+    batch = np.zeros(max(G, 1), dtype=np.int32)
+    nb = ctypes.c_int32(0)
+    st = lib().pp_plan_batches(toks.ctypes.data_as(ctypes.c_void_p), G, int(capacity), 1 if sort_by_length else 0,
+                               order.ctypes.data_as(ctypes.c_void_p), batch.ctypes.data_as(ctypes.c_void_p),
+                               ctypes.byref(nb))
+    if st != 0:
+        raise PPError("pp_plan_batches", st, "invalid arguments")
+    return order[:G].tolist(), batch[:G].tolist(), int(nb.value)
 
 
 def pp_decode_workspace_bytes(groups_host, cu_host, hq: int) -> int:

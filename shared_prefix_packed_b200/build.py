@@ -1,7 +1,8 @@
 """Build libpp.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
 
-The library is one translation unit, ``csrc/pp_api.cu``, which includes every kernel header. The output lands next
-to this file so it travels with the source tree; ``python -m shared_prefix_packed_b200.build`` rebuilds it.
+The device code is one translation unit, ``csrc/pp_api.cu``, which includes every kernel header; plain host code
+(the batch planner) lives in ``host/*.cpp`` and is linked into the same library. The output lands next to this file
+so it travels with the source tree; ``python -m shared_prefix_packed_b200.build`` rebuilds it.
 """
 from __future__ import annotations
 
@@ -15,6 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libpp.so")
 SRC = os.path.join(HERE, "csrc", "pp_api.cu")
+HOST_SRC = sorted(glob.glob(os.path.join(HERE, "host", "*.cpp")))
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -26,7 +28,7 @@ def _nvcc() -> str:
 
 
 def _sources():
-    return [SRC] + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + [os.path.join(ROOT, "include", "pp.h")]
+    return [SRC] + HOST_SRC + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + [os.path.join(ROOT, "include", "pp.h")]
 
 
 def up_to_date() -> bool:
@@ -41,7 +43,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
     cmd = [_nvcc(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
-           "-Xcompiler", "-fvisibility=hidden", "-o", LIB + ".tmp", SRC]
+           "-Xcompiler", "-fvisibility=hidden", "-o", LIB + ".tmp", SRC, *HOST_SRC]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)
