@@ -8,6 +8,18 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+@pytest.fixture(scope="session", autouse=True)
+def _built_library():
+    """Build libpp.so once if it is missing or older than its sources (a no-op otherwise). Without nvcc the
+    oracle-only tests still run; tests that need the library then fail loudly when they load it."""
+    try:
+        from shared_prefix_packed_b200 import build as B
+        B.build()
+    except (RuntimeError, OSError):
+        pass
+    yield
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a) and the built library")
     config.addinivalue_line("markers", "slow: long-running CPU test")
