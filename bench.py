@@ -47,6 +47,26 @@ def unpacked_pairs(P, S):
         p * (p + 1) // 2 for p, ss in zip(P, S) if not ss)
 
 
+# Datasheet dense bf16 tensor peak of one B200: NVIDIA's HGX B200 datasheet lists 36 PFLOPS FP16/BF16 for 8 GPUs
+# with 2:4 sparsity, i.e. 18 PFLOPS dense for 8 GPUs, 2.25 PFLOPS dense per GPU.
+DATASHEET_BF16_TFLOPS = 2250.0
+DATASHEET_SOURCE = "NVIDIA HGX B200 datasheet: 36 PFLOPS FP16/BF16 per 8 GPUs with 2:4 sparsity = 2.25 dense per GPU"
+
+
+def unpacked_layout(P, S):
+    """The same preference samples without packing: every response becomes its own sequence P || S_i (a group with
+    P' = P and one response); a group without responses keeps its prefix alone."""
+    Pu, Su = [], []
+    for p, ss in zip(P, S):
+        if not ss:
+            Pu.append(p)
+            Su.append([])
+        for s_ in ss:
+            Pu.append(p)
+            Su.append([s_])
+    return Pu, Su
+
+
 def flops_of(name, P, S):
     w = W.WORKLOADS[name]
     pairs = pair_count(P, S)
@@ -249,7 +269,13 @@ def run_gpu(args):
     for m in marks:
         for key, a, b in (("build_meta", 0, 1), ("rope", 1, 2), ("attn_fwd", 2, 3), ("attn_bwd", 3, 4)):
             parts[key] += m[a].elapsed_time(m[b]) / args.steps
+    step_ms = [m[0].elapsed_time(m[4]) for m in marks]
+    median_ms = max_over_ranks(statistics.median(step_ms), dev, dist)
     ms_per_step = max_over_ranks(ms, dev, dist) / args.steps
+
+    extras = {}
+    if not args.no_extras:
+        extras = measure_extras(args, name, P, S, batch, q, k, v, dout, stream, dev)
     total_flops = (f_fwd + f_bwd) * world
     value = aggregate_tflops(f_fwd + f_bwd, world, ms_per_step)
 
@@ -359,11 +385,116 @@ def run_gpu(args):
                    "l2": f"inputs larger than L2 ({(q.numel() + k.numel() + v.numel()) * 2 / 2**20:.0f} MiB of Q/K/V "
                          f"per rank vs 126 MiB), no flush", "parallelism": f"weak-scaled replicas x{world}"},
         "frac_of_peak": round(value / world / peaks["bf16_tflops"], 4),
+        "frac_of_peak_sustained": round(value / world / peaks["bf16_tflops_sustained"], 4)
+        if peaks.get("bf16_tflops_sustained") else None,
+        "frac_of_datasheet": round(value / world / DATASHEET_BF16_TFLOPS, 4),
+        "datasheet": {"bf16_dense_tflops": DATASHEET_BF16_TFLOPS, "source": DATASHEET_SOURCE},
+        "step_ms_median": round(median_ms, 4), "step_ms_mean": round(ms_per_step, 4),
         "ms_per_call": {k_: round(v_, 4) for k_, v_ in parts.items()},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    line.update(extras)
     print(json.dumps(line), flush=True)
+
+
+def _timed(fn, reps, stream, flush=None):
+    """Median device time (ms) of fn() over reps calls, each timed alone with CUDA events on `stream`; flush() (an
+    L2-sized write) runs before every call, outside the timed span."""
+    import torch
+    out = []
+    for _ in range(reps):
+        if flush is not None:
+            flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        out.append(a.elapsed_time(b))
+    return statistics.median(out)
+
+
+def measure_extras(args, name, P, S, batch, q, k, v, dout, stream, dev, reps=20):
+    """Measurements beside the headline step (same rank, after its timed region):
+      * pp_rope and pp_build_meta alone, each after an L2 flush (a 256 MiB write), as GB/s of their algorithmic
+        bytes: RoPE reads and writes Q and K once and reads the position ids; the builder reads the descriptors and
+        segment bounds and writes the position ids, the two per-token tables and the tile lists;
+      * the unpacked comparison: the same four calls on the same preference samples laid out without packing (every
+        response its own sequence P || S_i), with its allowed pairs, K/V bytes and step time."""
+    import torch
+    from shared_prefix_packed_b200 import PackedBatch, _lib
+    w = W.WORKLOADS[name]
+    hq, hkv, d = w.num_heads_q, w.num_heads_kv, w.head_dim
+    T = W.packed_total(P, S)
+    flush_buf = torch.empty(64 * 2 ** 20, dtype=torch.float32, device=dev)
+    flush = lambda: flush_buf.fill_(1.0)  # noqa: E731
+    peaks = load_peaks()
+    res = {}
+    hdr = batch.meta[:64].view(torch.int32).cpu().tolist()
+    n_qt, n_kt, n_bw = hdr[6], hdr[7], hdr[8]
+    G, nseg = len(P), sum(1 + len(ss) for ss in S)
+    meta_bytes = 8 * G + 4 * (nseg + 1) + 4 * T + 8 * T + 2 * 48 * n_qt + 32 * n_kt + 32 * n_bw
+    ms_meta = _timed(lambda: batch.build(stream), reps, stream, flush)
+    res["meta"] = {"ms": round(ms_meta, 4), "bytes": meta_bytes, "gbs": round(meta_bytes / (ms_meta * 1e-3) / 1e9, 1),
+                   "launches": 5, "note": "five launches of a few us each: launch-latency bound at this size"}
+    if w.rope:
+        rope_bytes = T * (hq + hkv) * d * 2 * 2 + 4 * T
+        ms_rope = _timed(lambda: batch.rope(q, k, stream=stream), reps, stream, flush)
+        gbs = rope_bytes / (ms_rope * 1e-3) / 1e9
+        res["rope"] = {"ms": round(ms_rope, 4), "bytes": rope_bytes, "gbs": round(gbs, 1),
+                       "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4), "l2": "flushed (256 MiB write) before each call"}
+    # unpacked comparison
+    Pu, Su = unpacked_layout(P, S)
+    Tu = W.packed_total(Pu, Su)
+    inp = W.make_inputs(name, Pu, Su, seed=w.tensor_seed + 17)
+    qu, ku, vu = (inp[x].to(dev) for x in "qkv")
+    bu = PackedBatch(Pu, Su, hq, hkv, d, device=dev)
+    ou = torch.empty_like(qu)
+    lu = torch.empty(hq, Tu, dtype=torch.float32, device=dev)
+    if w.backward:
+        du = inp["dout"].to(dev)
+        gq, gk, gv = torch.empty_like(qu), torch.empty_like(ku), torch.empty_like(vu)
+
+    def ustep():
+        bu.build(stream)
+        if w.rope:
+            bu.rope(qu, ku, stream=stream)
+        bu.forward(qu, ku, vu, out=ou, lse=lu, stream=stream)
+        if w.backward:
+            bu.backward(qu, ku, vu, ou, lu, du, dq=gq, dk=gk, dv=gv, stream=stream)
+
+    o_ = torch.empty_like(q)
+    l_ = torch.empty(hq, T, dtype=torch.float32, device=dev)
+    if w.backward:
+        g_ = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+
+    def pstep():
+        batch.build(stream)
+        if w.rope:
+            batch.rope(q, k, stream=stream)
+        batch.forward(q, k, v, out=o_, lse=l_, stream=stream)
+        if w.backward:
+            batch.backward(q, k, v, o_, l_, dout, dq=g_[0], dk=g_[1], dv=g_[2], stream=stream)
+
+    for _ in range(3):
+        ustep()
+    _lib.pp_get_status(stream)
+    ms_u = _timed(ustep, reps, stream)
+    ms_p = _timed(pstep, reps, stream)
+    pairs_p, pairs_u = pair_count(P, S), pair_count(Pu, Su)
+    kv_p, kv_u = 2 * T * hkv * d * 2, 2 * Tu * hkv * d * 2
+    fl = (4 + (10 if w.backward else 0)) * d * hq
+    res["unpacked"] = {
+        "layout": "every response its own sequence P || S_i (same samples, no packing)",
+        "T": Tu, "allowed_pairs_per_head": pairs_u, "kv_bytes": kv_u, "ms_per_step": round(ms_u, 4),
+        "tflops_on_its_own_pairs": round(fl * pairs_u / (ms_u * 1e-3) / 1e12, 1),
+        "packed_ms_per_step_same_timing": round(ms_p, 4),
+        "speedup_packed_over_unpacked": round(ms_u / ms_p, 3),
+        "pairs_saved": round(1 - pairs_p / pairs_u, 4), "kv_bytes_saved": round(1 - kv_p / kv_u, 4),
+        "timing": f"median of {reps} single steps each (CUDA events), both layouts timed the same way"}
+    del qu, ku, vu, ou, lu, bu
+    return res
 
 
 # ---------------------------------------------------------------------------------------------------- CPU oracle
@@ -668,6 +799,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the rope/meta GB/s and the unpacked comparison measured after the timed region")
     ap.add_argument("--vocab", type=int, default=W.LOGPROB_VOCAB, help="vocabulary of the --logprobs read-out")
     ap.add_argument("--batcher", action="store_true",
                     help="host batch planner throughput and the modeled work of packing with batch sorting")

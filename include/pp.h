@@ -103,6 +103,21 @@ PP_API pp_status pp_meta_tiles(const void *meta_d, int32_t which, int32_t *tiles
                         void *stream);
 
 /* ---------------------------------------------------------------------------------------------------------------
+ * pp_meta_schedule: the work lists the attention kernels execute, in their stored order, for checking.
+ * ("PackInfer" abstract: attention work over the packed query-key regions, ordered to balance the thread blocks.)
+ *   which = PP_PASS_FWD: the forward query tiles in cost order (the order pp_attn_fwd and the dQ half of
+ *   pp_attn_bwd walk them); one record per key tile a query tile visits. which = PP_PASS_BWD: the backward work
+ *   chunks (key tile x a range of its query tiles) in their stored order; one record per query tile of a chunk.
+ *   Each record is five int32 (item, q_row0, kv_row0, class, split): item = position of the query tile (fwd) or of
+ *   the chunk (bwd) in its list; class 1 = FULL, 2 = PARTIAL; split = 1 if the chunk's key tile is split over
+ *   several chunks (its dK/dV partials are added in fp32), else 0 (always 0 for fwd). records_d: device
+ *   int32[5 * capacity]; *count_d (device int32) receives the number of records (only the first `capacity` are
+ *   written). The order of the records is unspecified; their item fields give the stored order.
+ */
+PP_API pp_status pp_meta_schedule(const void *meta_d, int32_t which, int32_t *records_d, int64_t capacity,
+                                  int32_t *count_d, void *stream);
+
+/* ---------------------------------------------------------------------------------------------------------------
  * pp_rope: rotary embedding at the grouped position ids, in place on q and k (v untouched).
  * Rotate-half form with base theta: for m < d/2, w_m = theta^(-2m/d), a = pos * w_m,
  *   y_m = x_m cos a - x_{m+d/2} sin a,  y_{m+d/2} = x_{m+d/2} cos a + x_m sin a
@@ -246,6 +261,19 @@ PP_API pp_status pp_response_logprobs(const void *logits, pp_dtype dt, int64_t V
  */
 PP_API pp_status pp_plan_batches(const int64_t *group_tokens, int32_t num_groups, int64_t token_capacity,
                                  int32_t sort_by_length, int32_t *order, int32_t *batch_of_group, int32_t *num_batches);
+
+/* ---------------------------------------------------------------------------------------------------------------
+ * pp_selftest_bounded_wait: exercise the error channel of the kernels' bounded waits without a fault.
+ * (The pages have no counterpart; this checks the library's failure detection.) Every mbarrier wait in the attention
+ * kernels gives up after a time limit (2 s), records PP_ERR_DEVICE_TIMEOUT in the device error word and returns, so
+ * a stuck pipeline ends with an error status instead of a hung GPU. This call launches one small kernel whose single
+ * wait, with the same wait code and the given limit, is on an mbarrier that nothing arrives on; it issues no copy and
+ * no MMA, so nothing is in flight when the wait gives up. The next pp_get_status() returns PP_ERR_DEVICE_TIMEOUT
+ * (and clears the word); the context stays usable.
+ *   limit_ns in [1e3, 2e9]. waited_ns_d: device uint64 out, the time the wait took before it gave up (0 if it
+ *   completed, which cannot happen here). Errors: PP_ERR_INVALID_ARG.
+ */
+PP_API pp_status pp_selftest_bounded_wait(int64_t limit_ns, unsigned long long *waited_ns_d, void *stream);
 
 /* ---------------------------------------------------------------------------------------------------------------
  * pp_get_status: synchronises `stream`, then reads and clears this device's error word. Returns PP_OK,

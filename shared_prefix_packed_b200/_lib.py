@@ -35,6 +35,7 @@ SIGNATURES = {
     "pp_meta_bounds": (_I32, [_I32, _I32, _I64, _I32, _I32, _I64P]),
     "pp_build_meta": (_I32, [_VP, _I32, _VP, _I32, _I64, _I32, _I32, _VP, _VP, _I64, _VP]),
     "pp_meta_tiles": (_I32, [_VP, _I32, _VP, _I64, _VP, _VP]),
+    "pp_meta_schedule": (_I32, [_VP, _I32, _VP, _I64, _VP, _VP]),
     "pp_rope": (_I32, [_VP, _VP, _VP, _I64, _I32, _I32, _I32, _F32, _I32, _I32, _VP]),
     "pp_workspace_bytes": (_I32, [_I32, _I64, _I32, _I32, _I32, _I64P]),
     "pp_attn_fwd": (_I32, [_VP, _VP, _VP, _VP, _I64, _I32, _I32, _I32, _F32, _I32, _VP, _VP, _VP, _I64, _VP]),
@@ -48,6 +49,7 @@ SIGNATURES = {
                               _VP]),
     "pp_pack_batch": (_I32, [_VP, _VP, _I32, _VP, _VP, _I32, _VP, _I32, _VP, _I64, _VP, _VP, _VP, _VP, _VP]),
     "pp_response_logprobs": (_I32, [_VP, _I32, _I64, _VP, _VP, _I64, _F32, _VP, _VP]),
+    "pp_selftest_bounded_wait": (_I32, [_I64, _VP, _VP]),
     "pp_get_status": (_I32, [_VP]),
     "pp_last_error": (ctypes.c_char_p, []),
     "pp_version": (ctypes.c_char_p, []),
@@ -130,6 +132,11 @@ def pp_build_meta(groups_d, cu_seqlens_d, total_tokens: int, hq: int, hkv: int, 
 def pp_meta_tiles(meta_d, which: int, tiles_d, count_d, stream=None):
     cap = tiles_d.numel() // 3
     _call("pp_meta_tiles", _ptr(meta_d), which, _ptr(tiles_d), cap, _ptr(count_d), _stream(stream))
+
+
+def pp_meta_schedule(meta_d, which: int, records_d, count_d, stream=None):
+    cap = records_d.numel() // 5
+    _call("pp_meta_schedule", _ptr(meta_d), which, _ptr(records_d), cap, _ptr(count_d), _stream(stream))
 
 
 def pp_rope(q, k, pos_ids_d, hq: int, hkv: int, d: int, theta: float = 10000.0, inverse: bool = False,
@@ -222,6 +229,11 @@ def pp_attn_bwd_noalloc(q, k, v, o, lse, dout, meta_d, dq, dk, dv, softmax_scale
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def pp_selftest_bounded_wait(limit_ns: int, waited_ns_d, stream=None):
+    """Launch the bounded-wait self-test (a wait on an mbarrier nothing arrives on); waited_ns_d: int64 [1] device."""
+    _call("pp_selftest_bounded_wait", int(limit_ns), _ptr(waited_ns_d), _stream(stream))
 
 
 def pp_get_status(stream=None) -> int:

@@ -220,6 +220,20 @@ pp_status pp_meta_tiles(const void *meta_d, int32_t which, int32_t *tiles_d, int
     return PP_OK;
 }
 
+pp_status pp_meta_schedule(const void *meta_d, int32_t which, int32_t *records_d, int64_t capacity, int32_t *count_d,
+                           void *stream) {
+    if (!meta_d || !count_d || (capacity > 0 && !records_d)) return fail(PP_ERR_INVALID_ARG, "NULL pointer");
+    if (which != PP_PASS_FWD && which != PP_PASS_BWD) return fail(PP_ERR_INVALID_ARG, "which must be fwd or bwd");
+    DeviceInfo *di;
+    pp_status st = device_info(&di);
+    if (st != PP_OK) return st;
+    cudaStream_t s = as_stream(stream);
+    PP_CUDA(cudaMemsetAsync(count_d, 0, sizeof(int32_t), s));
+    pp::k_meta_schedule<<<di->sm_count, 128, 0, s>>>(meta_d, which, records_d, capacity, count_d);
+    PP_CUDA(cudaGetLastError());
+    return PP_OK;
+}
+
 pp_status pp_rope(void *q, void *k, const int32_t *pos_ids_d, int64_t T, int32_t hq, int32_t hkv, int32_t d,
                   float theta, pp_dtype dt, int32_t inverse, void *stream) {
     pp_status st = check_heads(T, hq, hkv, d);
@@ -306,6 +320,7 @@ pp_status pp_decode_attn(const void *q, const void *k_cache, const void *v_cache
     for (const void *ptr : ptrs)
         if (reinterpret_cast<uintptr_t>(ptr) % 16) return fail(PP_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
     if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(PP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (!(softmax_scale >= 0.f) || std::isinf(softmax_scale)) return fail(PP_ERR_INVALID_ARG, "bad softmax_scale");
     const pp::DecPlan base = pp::dec_plan_layout(T, G, nseg, hq, 0);
     const int64_t rec = 4 * int64_t(hq) * (pp::DEC_D + 2);
     if (ws_bytes < base.off_part + rec) return fail(PP_ERR_WORKSPACE, "workspace too small for the decode plan");
@@ -492,6 +507,18 @@ pp_status pp_attn_bwd_noalloc(const void *q, const void *k, const void *v, const
     if ((st = noalloc_scratch(&scratch)) != PP_OK) return st;
     return pp_attn_bwd(q, k, v, o, lse, dout, meta_d, T, hq, hkv, d, softmax_scale, dq, dk, dv, scratch,
                        PP_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+pp_status pp_selftest_bounded_wait(int64_t limit_ns, unsigned long long *waited_ns_d, void *stream) {
+    if (limit_ns < 1000 || limit_ns > 2000000000ll)
+        return fail(PP_ERR_INVALID_ARG, "limit_ns must be in [1e3, 2e9] (got %lld)", (long long)limit_ns);
+    if (!waited_ns_d) return fail(PP_ERR_INVALID_ARG, "waited_ns_d is NULL");
+    DeviceInfo *di;
+    pp_status st = device_info(&di);
+    if (st != PP_OK) return st;
+    pp::k_selftest_wait<<<1, 32, 0, as_stream(stream)>>>(uint64_t(limit_ns), waited_ns_d);
+    PP_CUDA(cudaGetLastError());
+    return PP_OK;
 }
 
 pp_status pp_get_status(void *stream) {

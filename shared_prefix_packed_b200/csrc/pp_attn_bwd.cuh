@@ -74,10 +74,33 @@ inline BwdWorkspace bwd_workspace_layout(int64_t T, int hq, int hkv, int d) {
 // D = sum_d dO * O in fp32 per (row, head), stored with the lse as (-lse / scale, -D), the values the query side of
 // the extra MMA slice carries; padding rows get zeros. (row, head) pairs are contiguous 256-byte rows of O and dO,
 // so a warp takes eight consecutive pairs: half-warps of 16 lanes x 16 bytes, four loads of each tensor in flight
-// per lane (HBM-bound).
+// per lane (HBM-bound). The same grid also zeroes the fp32 dK/dV accumulator rows of the split key tiles (the
+// only rows the key-side kernel adds partials into); no other row of the accumulators is ever read.
 __global__ void k_bwd_pre(const __nv_bfloat16 *__restrict__ O, const __nv_bfloat16 *__restrict__ dO,
                           const float *__restrict__ lse, float2 *__restrict__ ld, int64_t T, int64_t rows_pad,
-                          int hq, float inv_scale) {
+                          int hq, float inv_scale, const void *__restrict__ meta, float *__restrict__ dk_acc,
+                          float *__restrict__ dv_acc, int hkv) {
+    {
+        const MetaHeader hd = *meta_ptr<MetaHeader>(meta, 0);
+        if (hd.dev_err == 0 && hd.n_split > 0) {
+            const KTile *kts = meta_ptr<KTile>(meta, hd.off_kt);
+            const int64_t per_row = int64_t(hkv) * (BWD_D / 4);       // float4 per row
+            const int64_t per_tile = 128 * per_row;
+            const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < int64_t(hd.n_kt) * per_tile;
+                 e += stride) {
+                const KTile t = kts[e / per_tile];
+                if (t.nch <= 1) continue;
+                const int64_t rem = e % per_tile;
+                const int64_t row = t.row0 + rem / per_row;
+                if (row >= t.gstart + t.glen) continue;
+                const int64_t off = row * hkv * BWD_D + (rem % per_row) * 4;
+                *reinterpret_cast<float4 *>(dk_acc + off) = z;
+                *reinterpret_cast<float4 *>(dv_acc + off) = z;
+            }
+        }
+    }
     const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
     const int64_t n_pairs = rows_pad * hq, n_real = T * hq;
     const int64_t nwarps = int64_t(gridDim.x) * (blockDim.x >> 5);
@@ -623,11 +646,9 @@ inline pp_status launch_bwd(const void *q, const void *k, const void *v, const v
     if ((st = make_map(&mv, v, T, hkv, d, BWD_BN)) != PP_OK) return st;
     if ((st = make_map(&mdo, dout, T, hq, d, BWD_BM)) != PP_OK) return st;
     cudaError_t e;
-    if ((e = cudaMemsetAsync(ws + L.off_dk, 0, L.total - L.off_dk, s)) != cudaSuccess)
-        return fail(PP_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
     k_bwd_pre<<<sm_count * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(o),
                                            static_cast<const __nv_bfloat16 *>(dout), lse, ldg, T, L.rows_pad, hq,
-                                           1.f / scale);
+                                           1.f / scale, meta, dk_acc, dv_acc, hkv);
     if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_pre: %s", cudaGetErrorString(e));
     const size_t smem = sizeof(BwdSmem) + 1024;
     if ((e = cudaFuncSetAttribute(k_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem))) != cudaSuccess)

@@ -38,21 +38,41 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
-// Bounded mbarrier wait. On timeout it records DEVERR_TIMEOUT, raises the CTA's abort flag and returns false;
-// every other waiter of the CTA then gives up at its next poll.
-__device__ __forceinline__ bool bwait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+// Bounded mbarrier wait. On timeout (limit_ns) it records DEVERR_TIMEOUT, raises the CTA's abort flag and returns
+// false; every other waiter of the CTA then gives up at its next poll.
+__device__ __forceinline__ bool bwait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                      uint64_t limit_ns = WAIT_TIMEOUT_NS) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
         if ((it & 7) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > WAIT_TIMEOUT_NS) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 *abort_flag = 1;
                 atomicOr(&g_dev_err, DEVERR_TIMEOUT);
                 return false;
             }
         }
+    }
+}
+
+// Self-test of the bounded wait: one CTA waits, with the kernels' own bwait and the given limit, on an mbarrier that
+// nothing ever arrives on. It issues no copy and no MMA, so nothing is in flight when the wait gives up; the
+// timeout is reported through the device error word like any other. waited_ns receives the time the wait took.
+__global__ void k_selftest_wait(uint64_t limit_ns, unsigned long long *waited_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        const bool ok = bwait(&bar, 0, &abort_flag, limit_ns);
+        *waited_ns = ok ? 0ull : static_cast<unsigned long long>(globaltimer_ns() - t0);
     }
 }
 

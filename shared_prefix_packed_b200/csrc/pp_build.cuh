@@ -328,4 +328,50 @@ __global__ void k_meta_expand(const void *meta, int which, int32_t *__restrict__
     }
 }
 
+// pp_meta_schedule: expand the work lists the kernels execute, in their stored order, into records
+// (item, q_row0, kv_row0, class, split). Forward: item = position of the query tile in the cost order (qts), one
+// record per key tile it visits, split = 0. Backward: item = index of the work chunk (BWork) in its stored order, one
+// record per query tile of its range, split = the chunk's flag.
+__global__ void k_meta_schedule(const void *meta, int which, int32_t *__restrict__ out, int64_t cap,
+                                int32_t *__restrict__ count) {
+    const MetaHeader *h = meta_ptr<MetaHeader>(meta, 0);
+    if (h->dev_err) return;
+    const int32_t *seg_start = meta_ptr<int32_t>(meta, h->off_seg_start);
+    auto emit = [&](int item, int q0, int k0, int c, int split) {
+        const int p = atomicAdd(count, 1);
+        if (p < cap) {
+            int32_t *o = out + 5 * int64_t(p);
+            o[0] = item; o[1] = q0; o[2] = k0; o[3] = c; o[4] = split;
+        }
+    };
+    if (which == 0) {
+        const QTile *qts = meta_ptr<QTile>(meta, h->off_qts);
+        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < h->n_qt; i += gridDim.x * blockDim.x) {
+            const QTile t = qts[i];
+            const int n = qtile_nkv(t);
+            const int x0 = t.row0 - t.gstart;
+            for (int j = 0; j < n; ++j) {
+                const int y0 = qtile_kv(t, j) * FWD_BN;
+                emit(i, t.row0, t.gstart + y0,
+                     tile_class(x0, FWD_BM, y0, FWD_BN, t.glen, t.plen, t.s0first, t.s0last), 0);
+            }
+        }
+    } else {
+        const BWork *bw = meta_ptr<BWork>(meta, h->off_bw);
+        const KTile *kt = meta_ptr<KTile>(meta, h->off_kt);
+        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < h->n_bw; i += gridDim.x * blockDim.x) {
+            const BWork w = bw[i];
+            const KTile t = kt[w.kt];
+            const int y0 = w.row0 - w.gstart;
+            for (int a = w.qa; a < w.qb; ++a) {
+                const int x0 = a * BWD_BM;
+                const int xm = min(x0 + BWD_BM, w.glen) - 1;
+                const int s0f = x0 >= t.plen ? seg_start[w.gstart + x0] - w.gstart : t.plen;
+                const int s0l = xm >= t.plen ? seg_start[w.gstart + xm] - w.gstart : 0;
+                emit(i, w.gstart + x0, w.row0, tile_class(x0, BWD_BM, y0, BWD_BN, w.glen, t.plen, s0f, s0l), w.split);
+            }
+        }
+    }
+}
+
 }  // namespace pp

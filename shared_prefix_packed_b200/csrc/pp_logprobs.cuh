@@ -52,6 +52,7 @@ __device__ __forceinline__ void lse2_add(float &m, float &s, const float (&x)[N]
     float vm = x[0];
 #pragma unroll
     for (int i = 1; i < N; ++i) vm = fmaxf(vm, x[i]);
+    if (vm == -INFINITY) return;                               // all masked: adds nothing (and -inf - -inf is NaN)
     if (vm > m) {
         s *= ex2_approx(m - vm);                               // m = -inf: s is 0 and stays 0
         m = vm;

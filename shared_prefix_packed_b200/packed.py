@@ -96,6 +96,17 @@ class PackedBatch:
         rows = buf[: 3 * n].view(-1, 3).cpu().tolist()
         return sorted(tuple(r) for r in rows)
 
+    def schedule(self, which: int, stream=None):
+        """The executed work list as rows (item, q_row0, kv_row0, class, split), sorted by item (test helper)."""
+        count = torch.zeros(1, dtype=torch.int32, device=self.device)
+        _lib.pp_meta_schedule(self.meta, which, torch.empty(5, dtype=torch.int32, device=self.device), count,
+                              stream)
+        n = int(count.item())
+        buf = torch.empty(5 * max(n, 1), dtype=torch.int32, device=self.device)
+        _lib.pp_meta_schedule(self.meta, which, buf, count, stream)
+        rows = buf[: 5 * n].view(-1, 5).cpu().tolist()
+        return sorted(tuple(r) for r in rows)
+
 
 def pack_batch(prompts, prompt_mask, responses, response_mask, uids, stream=None):
     """Pack an ungrouped micro-batch on the device (pp_pack_batch): returns (packed_ids [T], prefix_lens,

@@ -70,6 +70,35 @@ def test_logprobs_full_layout_sampled_rows():
     assert np.all(np.isfinite(lp)) and np.all(lp[src >= 0] < 0)
 
 
+@pytest.mark.parametrize("V,dtype", [(1000, "bf16"), (4099, "fp32"), (32771, "bf16")])
+def test_logprobs_negative_infinity_entries(V, dtype):
+    """Masked vocabulary entries (-inf logits): a padded tail of every row, scattered entries, whole 16-byte vectors
+    and the scalar head and tail. They add nothing to the sum; a token whose own logit is -inf gets -inf."""
+    from shared_prefix_packed_b200 import PackedBatch, pp_get_status
+    P, S = [130], [[129, 1, 300]]
+    logits, ids = W.make_logits(P, S, vocab=V, seed=77, dtype=dtype)
+    rng = np.random.default_rng(78)
+    ninf = float("-inf")
+    logits[:, V - 37:] = ninf                                   # padded tail of every row
+    logits[torch.from_numpy(rng.random(logits.shape) < 0.3)] = ninf   # 30 % scattered
+    logits[:, 8:64] = ninf                                      # whole vectors in a row
+    logits[:, :3] = ninf                                        # part of the head
+    src = oracle.response_source_rows(P, S)
+    resp = np.nonzero(src >= 0)[0]
+    ids[int(resp[5])] = V - 1                                   # a token whose logit is -inf
+    ids[int(resp[9])] = 10
+    b = PackedBatch(P, S, 4, 2, 128)
+    got = b.response_logprobs(logits.cuda(), ids.cuda(), temperature=0.8).cpu().double().numpy()
+    pp_get_status()
+    want, valid = oracle.response_logprobs(logits, ids, P, S, temperature=0.8)
+    assert not np.isnan(got).any()
+    assert np.all(got[~valid] == 0.0)
+    inf_rows = valid & np.isneginf(want)
+    assert inf_rows.sum() >= 2 and np.all(np.isneginf(got[inf_rows]))
+    fin = valid & np.isfinite(want)
+    assert np.max(np.abs(got[fin] - want[fin])) <= TOL
+
+
 def test_logprobs_bad_token_is_reported():
     from shared_prefix_packed_b200 import PackedBatch, PPError, pp_get_status
     P, S = [3], [[4]]

@@ -6,6 +6,7 @@ import torch
 import oracle
 import workloads as W
 from tests.gpu_util import random_case
+from tests.schedule_checks import check_backward_schedule, check_forward_schedule
 
 pytestmark = pytest.mark.gpu
 
@@ -58,15 +59,35 @@ def test_meta_full_workloads(name):
     assert b.tiles(PP_PASS_BWD) == oracle.tile_classes(P, S, 128, 128)
 
 
-def test_schedule_invariants():
-    """The forward order is a permutation of the query tiles by non-increasing cost; the backward chunks of each key
-    tile partition its query range exactly (read back from the metadata's documented structure via the tiles)."""
-    P, S = W.group_lengths("grpo")
-    b = _batch(P, S, 32, 8, 128)
-    from shared_prefix_packed_b200 import PP_PASS_FWD
-    tiles = b.tiles(PP_PASS_FWD)
-    # every non-empty forward tile appears exactly once
-    assert len(tiles) == len(set(tiles))
+SCHED_CASES = CASES + [([2100], [[700, 900]]), ([4000, 10], [[3000, 3000, 3000], [5]])]
+
+
+@pytest.mark.parametrize("P,S", SCHED_CASES)
+def test_schedule_small_cases(P, S):
+    from shared_prefix_packed_b200 import PP_PASS_BWD, PP_PASS_FWD
+    b = _batch(P, S)
+    check_forward_schedule(P, S, b.schedule(PP_PASS_FWD))
+    check_backward_schedule(P, S, b.schedule(PP_PASS_BWD))
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_schedule_random_groups(seed):
+    from shared_prefix_packed_b200 import PP_PASS_BWD, PP_PASS_FWD
+    P, S = random_case(500 + seed, 1 + seed % 5, 3000, 1500, 6)
+    b = _batch(P, S)
+    check_forward_schedule(P, S, b.schedule(PP_PASS_FWD))
+    check_backward_schedule(P, S, b.schedule(PP_PASS_BWD))
+
+
+@pytest.mark.parametrize("name", ["tiny", "dpo", "grpo", "longprefix", "hetero"])
+def test_schedule_full_workloads(name):
+    """The executed schedule of every workload, in the launch configuration the bench times."""
+    from shared_prefix_packed_b200 import PP_PASS_BWD, PP_PASS_FWD
+    P, S = W.group_lengths(name)
+    w = W.WORKLOADS[name]
+    b = _batch(P, S, w.num_heads_q, w.num_heads_kv, w.head_dim)
+    check_forward_schedule(P, S, b.schedule(PP_PASS_FWD))
+    check_backward_schedule(P, S, b.schedule(PP_PASS_BWD))
 
 
 def test_device_detects_inconsistent_descriptors():

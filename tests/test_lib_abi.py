@@ -55,3 +55,13 @@ def test_host_only_calls_and_validation():
         _lib.pp_workspace_bytes(_lib.PP_PASS_FWD, 100, 32, 8, 96)       # unsupported head dim
     with pytest.raises(_lib.PPError, match="INVALID_ARG"):
         _lib.pp_workspace_bytes(_lib.PP_PASS_FWD, -1, 32, 8, 128)
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    """The binding's copy of PP_NOALLOC_SCRATCH_BYTES must equal the header's value (the no-allocation test sizes
+    its case against it)."""
+    with open(os.path.join(ROOT, "include", "pp.h")) as f:
+        m = re.search(r"#define\s+PP_NOALLOC_SCRATCH_BYTES\s+\((\d+)ll\s*<<\s*(\d+)\)", f.read())
+    assert m, "PP_NOALLOC_SCRATCH_BYTES not found in pp.h"
+    from shared_prefix_packed_b200 import _lib
+    assert _lib.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
