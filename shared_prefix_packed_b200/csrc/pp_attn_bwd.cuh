@@ -150,7 +150,7 @@ __device__ __forceinline__ uint2 split3_bf16(float x) {
 
 // ------------------------------------------------------------------------------------------------- main kernel
 struct BwdSmem {
-    static constexpr int TILE = 128 * BWD_D * 2;         // 128 rows x d, bf16 (K, V, Q, dO; dS^T has the same size)
+    static constexpr int TILE = 128 * BWD_D * 2;         // 128 rows x d, bf16 (K, V, Q, dO)
     static constexpr int CHUNK = 128 * 64 * 2;           // one 64-column 128-byte-swizzled chunk of such a tile
     static constexpr int QSTAGES = 2;
     static constexpr int AUG = 128 * 16 * 2;             // 128 rows x 16 bf16, no-swizzle core-matrix layout
@@ -162,12 +162,13 @@ struct BwdSmem {
     alignas(1024) uint8_t aug_ones[AUG];                 // key side of the extra slice: (1, 1, 1, 0, ...)
     alignas(1024) uint8_t aug_q[QSTAGES][AUG];           // query side for S^T: split(-lse / scale)
     alignas(1024) uint8_t aug_do[QSTAGES][AUG];          // query side for dP^T: split(-D)
-    uint64_t kv_full, kv_empty, dkv_full, dkv_free;
-    uint64_t q_full[QSTAGES], q_empty[QSTAGES];
-    uint64_t s_full, dp_full, p_ready, ds_ready;
+    uint64_t k_full, k_empty, v_full, v_empty, dkv_full, dkv_free;
+    uint64_t q_full[QSTAGES], q_empty[QSTAGES], do_full[QSTAGES], do_empty[QSTAGES];
+    uint64_t s_full, s_free, dp_full, pds_ready;
     uint32_t tmem_base;
     int abort_flag;
 };
+static_assert(sizeof(BwdSmem) + 1024 <= 232448, "dK/dV kernel shared memory exceeds 227 KB");
 
 struct BwdItem {
     KTile t;
@@ -202,9 +203,6 @@ __device__ __forceinline__ BwdItem bwd_decode(const void *meta, const MetaHeader
 // Byte offset of row r, column 0 in a 128 x 16 bf16 no-swizzle K-major tile (8-row x 16-byte core matrices).
 __device__ __forceinline__ uint32_t aug_row_off(int r) { return (r >> 3) * 256 + (r & 7) * 16; }
 
-__device__ __forceinline__ void red_add_f32(float *addr, float a) {
-    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
-}
 __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
@@ -256,18 +254,22 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     volatile int *abort_flag = &sm.abort_flag;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sm.kv_full, 1);
-        mbar_init(&sm.kv_empty, 1);
+        mbar_init(&sm.k_full, 1);
+        mbar_init(&sm.k_empty, 1);
+        mbar_init(&sm.v_full, 1);
+        mbar_init(&sm.v_empty, 1);
         mbar_init(&sm.dkv_full, 1);
         mbar_init(&sm.dkv_free, 256);
         for (int b = 0; b < BwdSmem::QSTAGES; ++b) {
             mbar_init(&sm.q_full[b], 32);
             mbar_init(&sm.q_empty[b], 1);
+            mbar_init(&sm.do_full[b], 32);
+            mbar_init(&sm.do_empty[b], 1);
         }
         mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.s_free, 256);
         mbar_init(&sm.dp_full, 1);
-        mbar_init(&sm.p_ready, 256);
-        mbar_init(&sm.ds_ready, 256);
+        mbar_init(&sm.pds_ready, 256);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -303,31 +305,40 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         // nothing to do: the metadata builder rejected its input
     } else if (warp == 8) {
         // ------------------------------------------------------------------ producer warp
+        // Loads in the order the MMAs need them: K of the item, then per step Q (with its extra-slice tile), V (on
+        // the item's first step) and dO (with its extra-slice tile). Q and dO have separate stages, so each is
+        // reloaded as soon as its own last MMA (dK, dV) has read it.
         uint32_t g = 0, it_n = 0;
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
             const BwdItem w = bwd_decode(meta, hd, item, hkv);
-            if (lane == 0) {
-                if (!bwait(&sm.kv_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
-                mbar_arrive_expect_tx(&sm.kv_full, 2 * BwdSmem::TILE);
-                for (int c = 0; c < BWD_D / 64; ++c) {
-                    tma_load_3d(sm.k + c * BwdSmem::CHUNK, &tmK, c * 64, w.kh, w.t.row0, &sm.kv_full);
-                    tma_load_3d(sm.v + c * BwdSmem::CHUNK, &tmV, c * 64, w.kh, w.t.row0, &sm.kv_full);
-                }
-            }
             const int n = (w.qb - w.qa) * r;
             auto step_h = [&](int t) { return w.kh * r + t % r; };
             auto step_x0 = [&](int t) { return w.t.gstart + (w.qa + t / r) * BWD_BM; };
-            float2 lv[4];                                              // rows lane + 32u of the current step
-#pragma unroll
-            for (int u = 0; u < 4; ++u) lv[u] = ldg[int64_t(step_h(0)) * rows_pad + step_x0(0) + lane + 32 * u];
-            if (lane == 0)
+            if (lane == 0) {
+                const int nxt = item + int(gridDim.x);
+                if (nxt < n_items) {                                   // the next item's K/V into L2
+                    const BwdItem wn = bwd_decode(meta, hd, nxt, hkv);
+                    for (int c = 0; c < BWD_D / 64; ++c) {
+                        tma_prefetch_3d(&tmK, c * 64, wn.kh, wn.t.row0);
+                        tma_prefetch_3d(&tmV, c * 64, wn.kh, wn.t.row0);
+                    }
+                }
+                if (!bwait(&sm.k_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
+                mbar_arrive_expect_tx(&sm.k_full, BwdSmem::TILE);
+                for (int c = 0; c < BWD_D / 64; ++c)
+                    tma_load_3d(sm.k + c * BwdSmem::CHUNK, &tmK, c * 64, w.kh, w.t.row0, &sm.k_full);
                 for (int t = 0; t < 2 && t < n; ++t)
                     for (int c = 0; c < BWD_D / 64; ++c) {
                         tma_prefetch_3d(&tmQ, c * 64, step_h(t), step_x0(t));
                         tma_prefetch_3d(&tmdO, c * 64, step_h(t), step_x0(t));
                     }
+            }
+            float2 lv[4];                                              // rows lane + 32u of the current step
+#pragma unroll
+            for (int u = 0; u < 4; ++u) lv[u] = ldg[int64_t(step_h(0)) * rows_pad + step_x0(0) + lane + 32 * u];
             for (int t = 0; t < n; ++t, ++g) {
                 const int st = g % BwdSmem::QSTAGES;
+                const uint32_t ph = ((g / BwdSmem::QSTAGES) & 1) ^ 1;
                 const int h = step_h(t);
                 const int x0 = step_x0(t);
                 // next step's values and (two steps ahead) its tiles: their latency hides behind this step
@@ -341,22 +352,37 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         tma_prefetch_3d(&tmQ, c * 64, step_h(t + 2), step_x0(t + 2));
                         tma_prefetch_3d(&tmdO, c * 64, step_h(t + 2), step_x0(t + 2));
                     }
-                if (!bwait(&sm.q_empty[st], ((g / BwdSmem::QSTAGES) & 1) ^ 1, abort_flag)) goto done;
+                // Q(t) and its slice split(-lse / scale)
+                if (!bwait(&sm.q_empty[st], ph, abort_flag)) goto done;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const uint32_t off = aug_row_off(lane + 32 * u);
-                    *reinterpret_cast<uint2 *>(sm.aug_q[st] + off) = split3_bf16(lv[u].x);
-                    *reinterpret_cast<uint2 *>(sm.aug_do[st] + off) = split3_bf16(lv[u].y);
-                }
+                for (int u = 0; u < 4; ++u)
+                    *reinterpret_cast<uint2 *>(sm.aug_q[st] + aug_row_off(lane + 32 * u)) = split3_bf16(lv[u].x);
                 fence_proxy_async_smem();
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&sm.q_full[st], 2 * BwdSmem::TILE);
-                    for (int c = 0; c < BWD_D / 64; ++c) {
+                    mbar_arrive_expect_tx(&sm.q_full[st], BwdSmem::TILE);
+                    for (int c = 0; c < BWD_D / 64; ++c)
                         tma_load_3d(sm.q[st] + c * BwdSmem::CHUNK, &tmQ, c * 64, h, x0, &sm.q_full[st]);
-                        tma_load_3d(sm.dout[st] + c * BwdSmem::CHUNK, &tmdO, c * 64, h, x0, &sm.q_full[st]);
-                    }
                 } else {
                     mbar_arrive(&sm.q_full[st]);
+                }
+                if (t == 0 && lane == 0) {                             // V of the item (feeds dP^T only)
+                    if (!bwait(&sm.v_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
+                    mbar_arrive_expect_tx(&sm.v_full, BwdSmem::TILE);
+                    for (int c = 0; c < BWD_D / 64; ++c)
+                        tma_load_3d(sm.v + c * BwdSmem::CHUNK, &tmV, c * 64, w.kh, w.t.row0, &sm.v_full);
+                }
+                // dO(t) and its slice split(-D)
+                if (!bwait(&sm.do_empty[st], ph, abort_flag)) goto done;
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    *reinterpret_cast<uint2 *>(sm.aug_do[st] + aug_row_off(lane + 32 * u)) = split3_bf16(lv[u].y);
+                fence_proxy_async_smem();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sm.do_full[st], BwdSmem::TILE);
+                    for (int c = 0; c < BWD_D / 64; ++c)
+                        tma_load_3d(sm.dout[st] + c * BwdSmem::CHUNK, &tmdO, c * 64, h, x0, &sm.do_full[st]);
+                } else {
+                    mbar_arrive(&sm.do_full[st]);
                 }
                 if (t + 1 < n) {
 #pragma unroll
@@ -366,96 +392,123 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------------ MMA issuer (one thread)
-        if (lane == 0) {
+        // One flat walk over the CTA's steps g (across items). Per step: (a) S^T(g+1) as soon as the gradient warps
+        // have read S^T(g) into registers; (b) dK(g) and dV(g) once P^T(g) and dS^T(g) are in TMEM; (c) dP^T(g+1).
+        // MMAs from one thread execute in issue order, so dP^T(g+1) may overwrite the columns that dK(g)/dV(g)
+        // read, and the gradient warps' P(g+1) overlaps dK(g), dV(g) and dP^T(g+1).
+        if (lane == 0 && int(blockIdx.x) < n_items) {
             constexpr uint32_t ID_SDP = idesc_bf16(128, BWD_BM, 0, 0);     // S^T, dP^T (both K-major)
-            constexpr uint32_t ID_DV = idesc_bf16(128, BWD_D, 0, 1);       // dV (A TMEM, B MN-major)
-            constexpr uint32_t ID_DK = idesc_bf16(128, BWD_D, 0, 1);       // dK (A TMEM, B MN-major)
-            const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
-            uint32_t g = 0, it_n = 0;
-            // K-major x K-major product over d (S^T = K Q^T or dP^T = V dO^T)
+            constexpr uint32_t ID_KV = idesc_bf16(128, BWD_D, 0, 1);       // dK, dV (A TMEM, B MN-major)
+            // descriptors built once; a stage is a constant stride away (desc_adv)
+            constexpr uint32_t TB = BwdSmem::TILE, AB = BwdSmem::AUG;
+            const uint64_t k_desc = smem_desc(smem_u32(sm.k), 16, 1024);
+            const uint64_t v_desc = smem_desc(smem_u32(sm.v), 16, 1024);
+            const uint64_t q_desc = smem_desc(smem_u32(sm.q[0]), 16, 1024);          // K-major (S^T)
+            const uint64_t do_desc = smem_desc(smem_u32(sm.dout[0]), 16, 1024);
+            const uint64_t qn_desc = smem_desc(smem_u32(sm.q[0]), BwdSmem::CHUNK, 1024);      // N-major (dK)
+            const uint64_t don_desc = smem_desc(smem_u32(sm.dout[0]), BwdSmem::CHUNK, 1024);  // N-major (dV)
             const uint64_t ones_desc = smem_desc(smem_u32(sm.aug_ones), BwdSmem::AUG_LBO, BwdSmem::AUG_SBO, 0);
-            auto issue_kk = [&](uint32_t col, uint32_t a, uint32_t b, const uint8_t *aug) {
+            const uint64_t augq_desc = smem_desc(smem_u32(sm.aug_q[0]), BwdSmem::AUG_LBO, BwdSmem::AUG_SBO, 0);
+            const uint64_t augdo_desc = smem_desc(smem_u32(sm.aug_do[0]), BwdSmem::AUG_LBO, BwdSmem::AUG_SBO, 0);
+            auto issue_kk = [&](uint32_t col, uint64_t a, uint64_t b, uint64_t aug) {
+                const uint32_t d = tmem + col;
 #pragma unroll
                 for (int kk = 0; kk < BWD_D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * BwdSmem::CHUNK + (kk & 3) * 32;
-                    umma_ss(tmem + col, smem_desc(a + off, 16, 1024), smem_desc(b + off, 16, 1024), ID_SDP, kk > 0);
+                    umma_ss(d, desc_adv(a, off), desc_adv(b, off), ID_SDP, kk > 0);
                 }
                 // the extra slice: + (1,1,1) . split(value of the query row)
-                umma_ss(tmem + col, ones_desc, smem_desc(smem_u32(aug), BwdSmem::AUG_LBO, BwdSmem::AUG_SBO, 0),
-                        ID_SDP, 1u);
-            };
-            auto issue_dp = [&](uint32_t gg) -> bool {      // dP^T(gg): dK(gg - 1) has read dS^T (issue order)
-                tc_fence_after();
-                issue_kk(COL_DP, sv, smem_u32(sm.dout[gg % BwdSmem::QSTAGES]), sm.aug_do[gg % BwdSmem::QSTAGES]);
-                umma_commit(&sm.dp_full);
-                return true;
-            };
-            auto issue_s = [&](uint32_t gg) -> bool {       // S^T(gg), once its Q tile has landed
-                const int st = gg % BwdSmem::QSTAGES;
-                if (!bwait(&sm.q_full[st], (gg / BwdSmem::QSTAGES) & 1, abort_flag)) return false;
-                tc_fence_after();
-                issue_kk(COL_S, sk, smem_u32(sm.q[st]), sm.aug_q[st]);
-                umma_commit(&sm.s_full);
-                return true;
+                umma_ss(d, ones_desc, aug, ID_SDP, 1u);
             };
             const BWork *bws = meta_ptr<BWork>(meta, hd.off_bw);
             auto item_steps = [&](int it) { const BWork b = bws[bwd_item_split(it, hd.n_bw, hkv).x]; return (b.qb - b.qa) * r; };
-            int n_next = blockIdx.x < n_items ? item_steps(blockIdx.x) : 0;
-            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
-                const int n = n_next;                                  // loaded one item ahead
-                if (item + int(gridDim.x) < n_items) n_next = item_steps(item + gridDim.x);
-                if (!bwait(&sm.kv_full, it_n & 1, abort_flag)) goto done;
-                if (!issue_s(g)) goto done;
-                if (!issue_dp(g)) goto done;
-                if (n == 1) umma_commit(&sm.kv_empty);           // K and V feed S^T and dP^T only
-                if (!bwait(&sm.dkv_free, (it_n & 1) ^ 1, abort_flag)) goto done;
-                for (int t = 0; t < n; ++t, ++g) {
-                    const int st = g % BwdSmem::QSTAGES;
-                    const uint32_t sq = smem_u32(sm.q[st]), sdo = smem_u32(sm.dout[st]);
-                    // dV += P^T dO, as soon as the softmax warps have written P^T
-                    if (!bwait(&sm.p_ready, g & 1, abort_flag)) goto done;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < BWD_BM / 16; ++kk)
-                        umma_ts(tmem + COL_DV, tmem + COL_S + 64 * (kk >> 2) + 8 * (kk & 3),
-                                smem_desc(sdo + kk * 2048, BwdSmem::CHUNK, 1024), ID_DV, (t > 0 || kk > 0));
-                    // S^T of the next step may overwrite P^T now (MMAs run in issue order); issue it first only if
-                    // its tile has landed, so a late load never holds up dK of this step
-                    bool s_next = false;
-                    if (t + 1 < n && mbar_try_wait(&sm.q_full[(g + 1) % BwdSmem::QSTAGES], ((g + 1) / BwdSmem::QSTAGES) & 1)) {
-                        if (!issue_s(g + 1)) goto done;
-                        s_next = true;
-                    }
-                    // dK += dS^T Q once dS^T is in TMEM
-                    if (!bwait(&sm.ds_ready, g & 1, abort_flag)) goto done;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < BWD_BM / 16; ++kk)
-                        umma_ts(tmem + COL_DK, tmem + COL_DP + 64 * (kk >> 2) + 8 * (kk & 3),
-                                smem_desc(sq + kk * 2048, BwdSmem::CHUNK, 1024), ID_DK, (t > 0 || kk > 0));
-                    umma_commit(&sm.q_empty[st]);
-                    if (t + 1 < n && !s_next && !issue_s(g + 1)) goto done;
-                    if (t + 1 < n && !issue_dp(g + 1)) goto done;
-                    if (t + 2 == n) umma_commit(&sm.kv_empty);
+            // S^T(gg) (first of its item: after K lands) and dP^T(gg)
+            auto issue_s = [&](uint32_t gg, bool first, uint32_t item_par, bool last) -> bool {
+                const int st = gg % BwdSmem::QSTAGES;
+                if (first && !bwait(&sm.k_full, item_par, abort_flag)) return false;
+                if (!bwait(&sm.q_full[st], (gg / BwdSmem::QSTAGES) & 1, abort_flag)) return false;
+                tc_fence_after();
+                issue_kk(COL_S, k_desc, q_desc + uint64_t(st) * (TB >> 4), augq_desc + uint64_t(st) * (AB >> 4));
+                umma_commit(&sm.s_full);
+                if (last) umma_commit(&sm.k_empty);                  // K feeds S^T only
+                return true;
+            };
+            auto issue_dp = [&](uint32_t gg, bool first, uint32_t item_par, bool last) -> bool {
+                const int st = gg % BwdSmem::QSTAGES;
+                if (first && !bwait(&sm.v_full, item_par, abort_flag)) return false;
+                if (!bwait(&sm.do_full[st], (gg / BwdSmem::QSTAGES) & 1, abort_flag)) return false;
+                tc_fence_after();
+                issue_kk(COL_DP, v_desc, do_desc + uint64_t(st) * (TB >> 4), augdo_desc + uint64_t(st) * (AB >> 4));
+                umma_commit(&sm.dp_full);
+                if (last) umma_commit(&sm.v_empty);                  // V feeds dP^T only
+                return true;
+            };
+            int item = blockIdx.x, n = item_steps(item), t = 0;
+            uint32_t g = 0, it_n = 0;
+            if (!issue_s(0, true, 0, n == 1)) goto done;
+            if (!issue_dp(0, true, 0, n == 1)) goto done;
+            for (;;) {
+                // the step after g: (item2, t2) with n2 steps
+                int item2 = item, t2 = t + 1, n2 = n;
+                if (t2 == n) {
+                    item2 = item + int(gridDim.x);
+                    t2 = 0;
+                    n2 = item2 < n_items ? item_steps(item2) : 0;
                 }
-                umma_commit(&sm.dkv_full);
+                const bool have_next = item2 < n_items;
+                const bool next_first = have_next && t2 == 0;
+                const uint32_t par2 = (it_n + (next_first ? 1u : 0u)) & 1;
+                // (a) S^T(g+1) once the gradient warps hold S^T(g) in registers
+                if (have_next) {
+                    if (!bwait(&sm.s_free, g & 1, abort_flag)) goto done;
+                    if (!issue_s(g + 1, next_first, par2, t2 + 1 == n2)) goto done;
+                }
+                // (b) dK(g) += dS^T Q, dV(g) += P^T dO (A from TMEM: P^T and dS^T in the dP columns)
+                if (!bwait(&sm.pds_ready, g & 1, abort_flag)) goto done;
+                if (t == 0 && !bwait(&sm.dkv_free, (it_n & 1) ^ 1, abort_flag)) goto done;   // last item's epilogue read
+                tc_fence_after();
+                {
+                    const int st = g % BwdSmem::QSTAGES;
+                    const uint64_t bq = qn_desc + uint64_t(st) * (TB >> 4), bdo = don_desc + uint64_t(st) * (TB >> 4);
+                    const uint32_t acc0 = t > 0 ? 1u : 0u;
+#pragma unroll
+                    for (int kk = 0; kk < BWD_BM / 16; ++kk)
+                        umma_ts(tmem + COL_DK, tmem + COL_DP + 64 * (kk >> 2) + 32 + 8 * (kk & 3),
+                                desc_adv(bq, kk * 2048), ID_KV, kk > 0 ? 1u : acc0);
+                    umma_commit(&sm.q_empty[st]);
+#pragma unroll
+                    for (int kk = 0; kk < BWD_BM / 16; ++kk)
+                        umma_ts(tmem + COL_DV, tmem + COL_DP + 64 * (kk >> 2) + 8 * (kk & 3),
+                                desc_adv(bdo, kk * 2048), ID_KV, kk > 0 ? 1u : acc0);
+                    umma_commit(&sm.do_empty[st]);
+                    if (t + 1 == n) umma_commit(&sm.dkv_full);
+                }
+                if (!have_next) break;
+                // (c) dP^T(g+1): in issue order after dK(g), dV(g), which read these columns
+                if (!issue_dp(g + 1, next_first, par2, t2 + 1 == n2)) goto done;
+                ++g;
+                if (next_first) ++it_n;
+                item = item2;
+                t = t2;
+                n = n2;
             }
         }
     } else {
         // ------------------------------------------------------------------ gradient warpgroups (warps 0-7)
-        // Warpgroup x handles query columns [64x, 64x+64) of every step: P (phase 1) and dS (phase 2). Its P^T and
-        // dS^T (bf16) go into TMEM columns it has itself already read: S cols [64x, 64x+32) and dP cols
-        // [64x, 64x+32) of their regions. Per step the order is dS(t), P(t+1), so the next step's P overlaps this
-        // step's dK/dQ^T MMAs.
+        // Warpgroup x handles query columns [64x, 64x+64) of every step (TMEM lane = key row). Per step: read S^T
+        // (and free it for the next step's MMA), P^T = exp2(S'^T scale log2 e); read dP^T; dS^T = scale P^T dP'^T;
+        // then P^T and dS^T (bf16) go into the 64 dP columns this warpgroup has itself read: P^T in the first 32,
+        // dS^T in the last 32.
         const int wx = warp >> 2;                                      // column half
         const int wl = warp & 3;
-        const int jr = wl * 32 + lane;                                 // TMEM lane: key row (P, dS) or d (dQ^T)
+        const int jr = wl * 32 + lane;                                 // TMEM lane: key row
         const uint32_t lane_off = uint32_t(wl * 32) << 16;
         const int cb = 64 * wx;                                        // first query column of this half
         uint32_t g = 0, it_n = 0;
         const int32_t *key_end = meta_ptr<int32_t>(meta, hd.off_key_end);
-        // Item epilogue, run after the next item's first P so the MMA warp has S^T/dP^T work meanwhile:
-        // warpgroup 0 takes dK, warpgroup 1 dV; the accumulator is released as soon as it is in registers.
+        // Item epilogue, run inside the next item's first step (after its P, before its dS), when dK/dV of the
+        // item have long been complete: warpgroup 0 takes dK, warpgroup 1 dV, 64 columns at a time; the
+        // accumulator is released as soon as the last columns are in registers.
         bool ep_yin = false, ep_split = false;
         int64_t ep_row = 0;
         auto epilogue = [&](uint32_t en) -> bool {
@@ -465,7 +518,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             float *acc = (wx == 0 ? dk_acc : dv_acc) + ep_row;
             __nv_bfloat16 *dst = (wx == 0 ? dK : dV) + ep_row;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {                     // 64 columns at a time
+            for (int half = 0; half < 2; ++half) {
                 uint32_t a[32], b[32];
                 tmem_ld32(src + 64 * half, a);
                 tmem_ld32(src + 64 * half + 32, b);
@@ -478,8 +531,6 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             }
             return true;
         };
-        // The next item's work chunk is loaded at the start of this one and its key_end after this item's first P,
-        // so no global load latency sits on the first step of an item.
         auto key_end_of = [&](const BwdItem &b) {
             const int yy = b.t.row0 + jr;
             return yy < b.t.gstart + b.t.glen ? key_end[yy] : yy;
@@ -499,88 +550,75 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             const int y = w.t.row0 + jr;
             const int gend = w.t.gstart + w.t.glen;
             const bool yin = y < gend;
-            uint32_t pk[32];                                           // P^T of the current step, packed bf16
-            // phase 1 of step gg: P^T = exp2(S'^T * scale * log2 e) (S' already holds s - lse / scale)
-            auto phase_p = [&](uint32_t gg, int t) -> bool {
+            for (int t = 0; t < n; ++t, ++g) {
                 const int x0 = w.t.gstart + (w.qa + t / r) * BWD_BM;
                 const int lo = y - x0 - cb, hi = ke - x0 - cb;         // allowed columns [lo, hi) of this half
                 const bool all_in = __all_sync(0xffffffffu, lo <= 0 && hi >= 64);
-                if (!bwait(&sm.s_full, gg & 1, abort_flag)) return false;
+                // P^T = exp2(S'^T * scale * log2 e) (S' already holds s - lse / scale), packed bf16
+                uint32_t pk[32];
+                if (!bwait(&sm.s_full, g & 1, abort_flag)) goto done;
                 tc_fence_after();
-                uint32_t sr[64];
                 {
                     uint32_t a0[32], a1[32];
                     tmem_ld32(tmem + lane_off + COL_S + cb, a0);
                     tmem_ld32(tmem + lane_off + COL_S + cb + 32, a1);
                     tmem_wait_ld(a0, a1);
+                    tc_fence_before();
+                    mbar_arrive(&sm.s_free);                           // the next step's S^T may overwrite it
+                    if (all_in) {
+                        const float2 sl2v = make_float2(sl2, sl2);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) { sr[e] = a0[e]; sr[32 + e] = a1[e]; }
-                }
-                if (all_in) {
-                    const float2 sl2v = make_float2(sl2, sl2);
+                        for (int e = 0; e < 32; ++e) {
+                            const uint32_t u0 = e < 16 ? a0[2 * e] : a1[2 * e - 32];
+                            const uint32_t u1 = e < 16 ? a0[2 * e + 1] : a1[2 * e - 31];
+                            const float2 x = fmul2(make_float2(__uint_as_float(u0), __uint_as_float(u1)), sl2v);
+                            pk[e] = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
+                        }
+                    } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float2 x = fmul2(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
-                                               sl2v);
-                        pk[e] = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
+                        for (int e = 0; e < 32; ++e) {
+                            const int c = 2 * e;
+                            const uint32_t u0 = e < 16 ? a0[2 * e] : a1[2 * e - 32];
+                            const uint32_t u1 = e < 16 ? a0[2 * e + 1] : a1[2 * e - 31];
+                            const float p0 = (c >= lo && c < hi) ? ex2_approx(__uint_as_float(u0) * sl2) : 0.f;
+                            const float p1 = (c + 1 >= lo && c + 1 < hi) ? ex2_approx(__uint_as_float(u1) * sl2) : 0.f;
+                            pk[e] = pack_bf16x2(p0, p1);
+                        }
                     }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int c = 2 * e;
-                        const float p0 = (c >= lo && c < hi) ? ex2_approx(__uint_as_float(sr[c]) * sl2) : 0.f;
-                        const float p1 = (c + 1 >= lo && c + 1 < hi) ? ex2_approx(__uint_as_float(sr[c + 1]) * sl2) : 0.f;
-                        pk[e] = pack_bf16x2(p0, p1);
-                    }
                 }
-                uint32_t t0[16], t1[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) { t0[e] = pk[e]; t1[e] = pk[16 + e]; }
-                tmem_st16(tmem + lane_off + COL_S + cb, t0);
-                tmem_st16(tmem + lane_off + COL_S + cb + 16, t1);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&sm.p_ready);
-                return true;
-            };
-            if (n > 0 && !phase_p(g, 0)) goto done;
-            if (it_n > 0 && !epilogue(it_n - 1)) goto done;
-            if (nxt < n_items) ken = key_end_of(wn);
-            ep_yin = yin;
-            ep_split = w.split;
-            ep_row = (int64_t(y) * hkv + w.kh) * BWD_D;
-            for (int t = 0; t < n; ++t, ++g) {
-                // phase 2: dS^T = scale P^T dP'^T (dP' = dP - D already) -> TMEM dP columns this warpgroup has read
+                if (t == 0) {
+                    if (it_n > 0 && !epilogue(it_n - 1)) goto done;
+                    ep_yin = yin;
+                    ep_split = w.split;
+                    ep_row = (int64_t(y) * hkv + w.kh) * BWD_D;
+                    if (nxt < n_items) ken = key_end_of(wn);
+                }
+                // dS^T = scale P^T dP'^T (dP' = dP - D already)
                 if (!bwait(&sm.dp_full, g & 1, abort_flag)) goto done;
                 tc_fence_after();
                 {
-                    uint32_t pr[64];
-                    {
-                        uint32_t a0[32], a1[32];
-                        tmem_ld32(tmem + lane_off + COL_DP + cb, a0);
-                        tmem_ld32(tmem + lane_off + COL_DP + cb + 32, a1);
-                        tmem_wait_ld(a0, a1);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) { pr[e] = a0[e]; pr[32 + e] = a1[e]; }
-                    }
-                    uint32_t t0[16], t1[16];
+                    // two halves of 32 columns, so fewer registers are live at once
+                    uint32_t ds[32];
                     const float2 sc = make_float2(scale, scale);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const uint32_t p = pk[e];
-                        const float2 ds = fmul2(fmul2(make_float2(bf16lo(p), bf16hi(p)), sc),
-                                                make_float2(__uint_as_float(pr[2 * e]), __uint_as_float(pr[2 * e + 1])));
-                        const uint32_t dd = pack_bf16x2(ds.x, ds.y);
-                        if (e < 16) t0[e] = dd; else t1[e - 16] = dd;
+                    for (int hf = 0; hf < 2; ++hf) {
+                        uint32_t a0[32];
+                        tmem_ld32(tmem + lane_off + COL_DP + cb + 32 * hf, a0);
+                        tmem_wait_ld(a0);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const uint32_t p = pk[16 * hf + e];
+                            const float2 d2 = fmul2(fmul2(make_float2(bf16lo(p), bf16hi(p)), sc),
+                                                    make_float2(__uint_as_float(a0[2 * e]), __uint_as_float(a0[2 * e + 1])));
+                            ds[16 * hf + e] = pack_bf16x2(d2.x, d2.y);
+                        }
                     }
-                    tmem_st16(tmem + lane_off + COL_DP + cb, t0);
-                    tmem_st16(tmem + lane_off + COL_DP + cb + 16, t1);
+                    tmem_st32(tmem + lane_off + COL_DP + cb, pk);
+                    tmem_st32(tmem + lane_off + COL_DP + cb + 32, ds);
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&sm.ds_ready);
-                // next step's phase 1 while this step's dK runs
-                if (t + 1 < n && !phase_p(g + 1, t + 1)) goto done;
+                mbar_arrive(&sm.pds_ready);
             }
         }
         if (it_n > 0 && !epilogue(it_n - 1)) goto done;

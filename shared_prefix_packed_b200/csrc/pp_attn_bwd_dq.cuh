@@ -151,13 +151,20 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         if (lane == 0) {
             constexpr uint32_t ID_SP = idesc_bf16(128, 128, 0, 0);         // S, dP: K-major x K-major over d
             constexpr uint32_t ID_DQ = idesc_bf16(128, 128, 0, 1);         // dQ: A = dS (TMEM), B = K N-major
-            const uint32_t sq = smem_u32(sm.q), sdo = smem_u32(sm.dout);
             uint32_t kv_it = 0, it_n = 0, g = 0;                           // g: global key-tile step counter
-            auto issue_kk = [&](uint32_t col, uint32_t a, uint32_t b) {
+            // descriptors built once; a stage is a constant stride away (desc_adv)
+            constexpr uint32_t TB = DqSmem::TILE;
+            const uint64_t q_desc = smem_desc(smem_u32(sm.q), 16, 1024);
+            const uint64_t do_desc = smem_desc(smem_u32(sm.dout), 16, 1024);
+            const uint64_t k_desc = smem_desc(smem_u32(sm.k[0]), 16, 1024);
+            const uint64_t v_desc = smem_desc(smem_u32(sm.v[0]), 16, 1024);
+            const uint64_t kn_desc = smem_desc(smem_u32(sm.k[0]), DqSmem::CHUNK, 1024);   // N-major (dQ)
+            auto issue_kk = [&](uint32_t col, uint64_t a, uint64_t b) {
+                const uint32_t d = tmem + col;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * DqSmem::CHUNK + (kk & 3) * 32;
-                    umma_ss(tmem + col, smem_desc(a + off, 16, 1024), smem_desc(b + off, 16, 1024), ID_SP, kk > 0);
+                    umma_ss(d, desc_adv(a, off), desc_adv(b, off), ID_SP, kk > 0);
                 }
             };
             // S of key tile `it` (ring position) into the S region; releases Q after the item's last tile
@@ -165,7 +172,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 const int sk = it % DQ_KSTAGES;
                 if (!bwait(&sm.k_full[sk], (it / DQ_KSTAGES) & 1, abort_flag)) return false;
                 tc_fence_after();
-                issue_kk(COL_S, sq, smem_u32(sm.k[sk]));
+                issue_kk(COL_S, q_desc, k_desc + uint64_t(sk) * (TB >> 4));
                 umma_commit(&sm.s_full);
                 if (last) umma_commit(&sm.q_empty);
                 return true;
@@ -175,7 +182,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 const int sv = it % DQ_VSTAGES;
                 if (!bwait(&sm.v_full[sv], (it / DQ_VSTAGES) & 1, abort_flag)) return false;
                 tc_fence_after();
-                issue_kk(COL_DP + 128 * b, sdo, smem_u32(sm.v[sv]));
+                issue_kk(COL_DP + 128 * b, do_desc, v_desc + uint64_t(sv) * (TB >> 4));
                 umma_commit(&sm.dp_full[b]);
                 umma_commit(&sm.v_empty[sv]);
                 if (last) umma_commit(&sm.do_empty);
@@ -206,12 +213,13 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     if (j == 0 && !bwait(&sm.dq_free, (it_n & 1) ^ 1, abort_flag)) goto done;
                     tc_fence_after();
                     const int sk = kv_it % DQ_KSTAGES;
-                    const uint32_t skd = smem_u32(sm.k[sk]);
-                    const uint32_t cds = COL_DP + 128 * (g & 1);
+                    const uint64_t bk = kn_desc + uint64_t(sk) * (TB >> 4);
+                    const uint32_t ads = tmem + COL_DP + 128 * (g & 1);
+                    const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_ts(tmem + COL_DQ, tmem + cds + 32 * (kk >> 1) + 8 * (kk & 1),
-                                smem_desc(skd + kk * 2048, DqSmem::CHUNK, 1024), ID_DQ, (j > 0 || kk > 0));
+                        umma_ts(tmem + COL_DQ, ads + 32 * (kk >> 1) + 8 * (kk & 1), desc_adv(bk, kk * 2048), ID_DQ,
+                                kk > 0 ? 1u : acc0);
                     umma_commit(&sm.k_empty[sk]);
                 }
                 umma_commit(&sm.dq_full);

@@ -189,22 +189,26 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         constexpr uint32_t IDESC_S = idesc_bf16(128, FWD_BN, 0, 0);
         constexpr uint32_t IDESC_O = idesc_bf16(128, D, 0, 1);
         uint32_t kv_it = 0, n_it = 0, p_cnt[2] = {0, 0}, item_cnt[2] = {0, 0};
-        const uint32_t q_addr[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
+        // descriptors built once; a head slot or stage is a constant stride away (desc_adv)
+        constexpr uint32_t TB = FwdSmem<D>::TILE_BYTES;
+        const uint64_t q_desc = smem_desc(smem_u32(sm.q[0]), 16, 1024);
+        const uint64_t k_desc = smem_desc(smem_u32(sm.k[0]), 16, 1024);
+        const uint64_t v_desc = smem_desc(smem_u32(sm.v[0]), FwdSmem<D>::CHUNK_BYTES, 1024);
         auto issue_s = [&](int hs, int st) {
-            const uint32_t kb = smem_u32(sm.k[st]);
+            const uint64_t a = q_desc + uint64_t(hs) * (TB >> 4), b = k_desc + uint64_t(st) * (TB >> 4);
+            const uint32_t d = tmem + hs * 128;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * FwdSmem<D>::CHUNK_BYTES + (kk & 3) * 32;
-                umma_ss(tmem + hs * 128, smem_desc(q_addr[hs] + off, 16, 1024), smem_desc(kb + off, 16, 1024),
-                        IDESC_S, kk > 0);
+                umma_ss(d, desc_adv(a, off), desc_adv(b, off), IDESC_S, kk > 0);
             }
         };
         auto issue_pv = [&](int hs, int st, uint32_t acc) {
-            const uint32_t vb = smem_u32(sm.v[st]);
+            const uint64_t b = v_desc + uint64_t(st) * (TB >> 4);
+            const uint32_t d = tmem + 256 + hs * 128, a = tmem + hs * 128;
 #pragma unroll
             for (int kk = 0; kk < FWD_BN / 16; ++kk)
-                umma_ts(tmem + 256 + hs * 128, tmem + hs * 128 + kk * 8,
-                        smem_desc(vb + kk * 2048, FwdSmem<D>::CHUNK_BYTES, 1024), IDESC_O, (acc | kk) ? 1u : 0u);
+                umma_ts(d, a + kk * 8, desc_adv(b, kk * 2048), IDESC_O, (acc | kk) ? 1u : 0u);
         };
         for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
             const FwdItem w = fwd_decode(meta, hd, item, hq, hkv);
