@@ -662,7 +662,7 @@ def run_decode(args):
                    "cache_bytes_read_once": 2 * T * hkv * d * 2,
                    "cache_bytes_if_unpacked": unpacked,
                    "l2": f"K/V cache {2 * T * hkv * d * 2 / 2**20:.0f} MiB, larger than L2, no flush"},
-        "roofline": {"bound": "hbm", "kernel": "k_dec_plan + k_dec_partial + k_dec_combine", "achieved": round(gbs, 1),
+        "roofline": {"bound": "hbm", "kernel": "k_dec_plan + k_dec_chunk + k_dec_combine", "achieved": round(gbs, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
                      "traffic": None, "peak_source": peaks["source"] + " hbm_gbs", "bytes_per_launch": nbytes},
         "gpu_launches": 3 * args.steps}))

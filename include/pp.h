@@ -196,7 +196,8 @@ PP_API pp_status pp_attn_bwd_noalloc(const void *q, const void *k, const void *v
  * prefix and its own rows, the packed mask at the response's last row ("PackInfer" abstract: group-contiguous KV
  * and attention over packed query-key regions; "Preference Packing": the prompt is shared by its responses).
  * A prefix chunk is read from HBM once per group and serves all of the group's responses (flash-decoding in
- * 64-key chunks, fp32 partials combined per query).
+ * 128-key chunks on the tensor cores: the chunk's queries, every response that sees it times the r q heads of a kv
+ * head, form the rows of S = Q K^T and O = P V; fp32 partials are combined per query). hq / hkv <= 128.
  *   q: [n_resp, hq, d] bf16, n_resp = num_segments - num_groups (responses in packed order). k_cache, v_cache:
  *   [T, hkv, d] bf16. groups_d, cu_d: the device descriptors and segment bounds of the cache (as for
  *   pp_build_meta; every response of nonzero length has its query's K/V as its last row). d = 128.

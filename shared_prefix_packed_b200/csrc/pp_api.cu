@@ -96,15 +96,23 @@ pp_status get_encoder(EncodeTiledFn *fn) {
     return PP_OK;
 }
 
-// 3-D map over a [rows, heads, d] bf16 tensor: box = 64 elements x 1 head x box_rows rows, 128-byte swizzle.
+// 3-D map over a [rows, heads, d] bf16 tensor: box = 64 elements x box_heads heads x box_rows rows, 128-byte swizzle.
+pp_status make_map_3d_box(CUtensorMap *m, const void *base, int64_t rows, int heads, int d, int box_heads,
+                          int box_rows);
+
 pp_status make_map_3d(CUtensorMap *m, const void *base, int64_t rows, int heads, int d, int box_rows) {
+    return make_map_3d_box(m, base, rows, heads, d, 1, box_rows);
+}
+
+pp_status make_map_3d_box(CUtensorMap *m, const void *base, int64_t rows, int heads, int d, int box_heads,
+                          int box_rows) {
     EncodeTiledFn enc;
     pp_status st = get_encoder(&enc);
     if (st != PP_OK) return st;
     if (reinterpret_cast<uintptr_t>(base) % 16) return fail(PP_ERR_INVALID_ARG, "tensor base not 16-byte aligned");
     cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(heads), cuuint64_t(rows)};
     cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(heads) * d * 2};
-    cuuint32_t box[3] = {64, 1, cuuint32_t(box_rows)};
+    cuuint32_t box[3] = {64, cuuint32_t(box_heads), cuuint32_t(box_rows)};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -321,22 +329,28 @@ pp_status pp_decode_attn(const void *q, const void *k_cache, const void *v_cache
         if (reinterpret_cast<uintptr_t>(ptr) % 16) return fail(PP_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
     if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(PP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     if (!(softmax_scale >= 0.f) || std::isinf(softmax_scale)) return fail(PP_ERR_INVALID_ARG, "bad softmax_scale");
+    const int r = hq / hkv;
+    if (r > 128) return fail(PP_ERR_UNSUPPORTED, "decode supports at most 128 q heads per kv head (got %d)", r);
+    const int rb = 128 / r;                                  // responses per query block (r * rb <= 128 rows)
     const pp::DecPlan base = pp::dec_plan_layout(T, G, nseg, hq, 0);
-    const int64_t rec = 4 * int64_t(hq) * (pp::DEC_D + 2);
+    const int64_t rec = 4 * int64_t(hq) * pp::DEC_REC;
     if (ws_bytes < base.off_part + rec) return fail(PP_ERR_WORKSPACE, "workspace too small for the decode plan");
     const pp::DecPlan p = pp::dec_plan_layout(T, G, nseg, hq, (ws_bytes - base.off_part) / rec);
     DeviceInfo *di;
     if ((st = device_info(&di)) != PP_OK) return st;
+    CUtensorMap mq, mk, mv;
+    if ((st = make_map_3d_box(&mq, q, n_resp, hq, d, r, rb)) != PP_OK) return st;
+    if ((st = make_map_3d(&mk, k_cache, T, hkv, d, pp::DEC_CH)) != PP_OK) return st;
+    if ((st = make_map_3d(&mv, v_cache, T, hkv, d, pp::DEC_CH)) != PP_OK) return st;
     const float scale = softmax_scale == 0.f ? 1.f / std::sqrt(float(d)) : softmax_scale;
     cudaStream_t s = as_stream(stream);
     const int32_t *gd = reinterpret_cast<const int32_t *>(groups_d);
-    pp::k_dec_plan<<<1, 1024, 0, s>>>(gd, G, cu_d, nseg, T, workspace, p);
+    pp::k_dec_plan<<<1, 1024, 0, s>>>(gd, G, cu_d, nseg, T, rb, workspace, p);
     PP_CUDA(cudaGetLastError());
-    PP_CUDA(cudaFuncSetAttribute(pp::k_dec_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, pp::DEC_SMEM));
-    pp::k_dec_partial<<<di->sm_count, pp::DEC_THREADS, pp::DEC_SMEM, s>>>(
-        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k_cache),
-        static_cast<const __nv_bfloat16 *>(v_cache), gd, G, cu_d, nseg, hq, hkv, scale * 1.4426950408889634f,
-        workspace, p);
+    const int smem = int(sizeof(pp::DecSmem)) + 1024;
+    PP_CUDA(cudaFuncSetAttribute(pp::k_dec_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    pp::k_dec_chunk<<<di->sm_count, pp::DEC_THREADS, smem, s>>>(mq, mk, mv, gd, cu_d, nseg, hq, hkv, rb, n_resp,
+                                                                  scale * 1.4426950408889634f, workspace, p);
     PP_CUDA(cudaGetLastError());
     pp::k_dec_combine<<<grid_for(di->sm_count, 16, int64_t(n_resp) * hq), pp::DEC_D, 0, s>>>(
         gd, G, cu_d, nseg, hq, n_resp, workspace, p, static_cast<__nv_bfloat16 *>(o), lse);

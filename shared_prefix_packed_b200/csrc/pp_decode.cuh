@@ -4,43 +4,48 @@
 // response last ("PackInfer" abstract: group-contiguous KV, so a shared prefix is read once; "Preference Packing":
 // responses share the prompt's attention). Each response has one query, its newest token, which attends to the
 // group's prefix and to its own rows, under the same mask as the packed prefill.
-// Flash-decoding over 64-key chunks of every cache segment:
-//   k_dec_plan     one block: segment -> group, chunk counts and (chunk, query) pair offsets (scans).
-//   k_dec_partial  persistent grid over (chunk, kv head): loads the chunk's K/V once into shared memory and
-//                  computes, for every query that sees the chunk (all responses of the group for a prefix chunk,
-//                  one response for a response chunk) and each of the r q heads, the chunk's max, sum and
-//                  un-normalised output. A prefix chunk is therefore read from HBM once per group, not per response.
-//   k_dec_combine  per (response, q head): merges its partials (the group's prefix chunks, its own chunks).
+// Flash-decoding over 128-key chunks of every cache segment:
+//   k_dec_plan   one block: segment -> group, chunk counts, (chunk, query) record offsets and job offsets (scans).
+//   k_dec_chunk  persistent tcgen05 kernel over jobs (chunk, kv head, query block). A job's query block is every
+//                query that sees the chunk (all responses of the group for a prefix chunk, one response for a
+//                response chunk) times the r q heads of the kv head, up to 128 rows, gathered by one 3-D TMA box
+//                from q [n_resp, hq, d]. S = Q K^T and O = P V run on the tensor cores (M = 128 query rows, N = 128
+//                keys, then N = d); the softmax warps own one query row each. A prefix chunk is therefore read from
+//                HBM once per group (per query block), not once per response. Each job writes an fp32 record
+//                (max, sum, un-normalised O) per valid query row.
+//   k_dec_combine per (response, q head): merges its records (the group's prefix chunks, its own chunks).
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
-#include "pp_build.cuh"   // block_exclusive_scan, upper_bound_i32
+#include "pp_build.cuh"     // block_exclusive_scan, upper_bound_i32, g_dev_err
+#include "pp_ptx.cuh"
+#include "pp_attn_fwd.cuh"  // bwait
 
 namespace pp {
 
-constexpr int DEC_CH = 64;            // keys per chunk
-constexpr int DEC_THREADS = 256;
+constexpr int DEC_CH = 128;           // keys per chunk (the MMA N of S, the K of P V)
 constexpr int DEC_D = 128;            // head dim
-constexpr int DEC_MAXQ = 64;          // query vectors (responses x q heads of one kv head) per pass over a chunk
-constexpr int DEC_LD = DEC_D + 4;     // padded fp32 row of K and Q in shared memory: 8 lanes of 16 B hit 32 banks
-constexpr int DEC_SMEM = (2 * DEC_CH * DEC_LD + DEC_MAXQ * DEC_LD + DEC_MAXQ * DEC_CH) * 4;  // bytes; sV unpadded
+constexpr int DEC_REC = 132;          // floats per record: max (base 2), sum, two pad, O[128] (16-byte aligned)
+constexpr int DEC_STAGES = 3;         // K and V chunk rings
+constexpr int DEC_THREADS = 192;      // warps 0-3 softmax / records, warp 4 TMA, warp 5 TMEM + MMA
 
 // Plan layout in the workspace (int32 sections, sizes from G and nseg).
 struct DecPlan {
     int64_t off_first_seg;   // [G + 1] first segment of each group (exclusive scan of 1 + k_g)
     int64_t off_seg_group;   // [nseg]
     int64_t off_unit_off;    // [nseg + 1] chunks before each segment
-    int64_t off_pair_off;    // [nseg + 1] (chunk, query) pairs before each segment
-    int64_t off_counts;      // [4]: units, pairs, ok (1 if the plan fits), unused
-    int64_t off_part;        // fp32 partials: [pairs][hq][DEC_D + 2]
+    int64_t off_pair_off;    // [nseg + 1] (chunk, query) records before each segment
+    int64_t off_job_off;     // [nseg + 1] jobs (chunk, query block) before each segment
+    int64_t off_counts;      // [4]: units, records, ok (1 if the plan fits), jobs
+    int64_t off_part;        // fp32 records: [pairs][hq][DEC_REC]
     int64_t total;
-    int64_t max_pairs;       // partial records the workspace holds
+    int64_t max_pairs;       // records the workspace holds
 };
 
 __host__ __device__ inline int64_t dec_a256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
-// Section offsets for a workspace that holds max_pairs (chunk, query) partial records. The exact number of pairs
-// is sum over prefixes of nch * k_g plus sum over responses of nch, nch = ceil(len / DEC_CH); the host sizing call
+// Section offsets for a workspace that holds max_pairs (chunk, query) records. The exact number of records is the
+// sum over prefixes of nch * k_g plus the sum over responses of nch, nch = ceil(len / DEC_CH); the host sizing call
 // computes it from host copies of the descriptors.
 __host__ inline DecPlan dec_plan_layout(int64_t T, int32_t G, int32_t nseg, int32_t hq, int64_t max_pairs) {
     DecPlan p{};
@@ -49,8 +54,9 @@ __host__ inline DecPlan dec_plan_layout(int64_t T, int32_t G, int32_t nseg, int3
     p.off_seg_group = o; o = dec_a256(o + 4 * int64_t(nseg));
     p.off_unit_off = o;  o = dec_a256(o + 4 * int64_t(nseg + 1));
     p.off_pair_off = o;  o = dec_a256(o + 4 * int64_t(nseg + 1));
+    p.off_job_off = o;   o = dec_a256(o + 4 * int64_t(nseg + 1));
     p.off_counts = o;    o = dec_a256(o + 16);
-    p.off_part = o;      o = dec_a256(o + 4 * max_pairs * hq * (DEC_D + 2));
+    p.off_part = o;      o = dec_a256(o + 4 * max_pairs * hq * DEC_REC);
     p.total = o;
     p.max_pairs = max_pairs;
     (void)T;
@@ -60,17 +66,21 @@ __host__ inline DecPlan dec_plan_layout(int64_t T, int32_t G, int32_t nseg, int3
 template <typename T> __device__ __forceinline__ T *dec_ptr(void *ws, int64_t off) {
     return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
 }
+template <typename T> __device__ __forceinline__ const T *dec_ptr(const void *ws, int64_t off) {
+    return reinterpret_cast<const T *>(static_cast<const char *>(ws) + off);
+}
 
-// groups: pp_group_desc pairs {prefix_len, num_suffixes}; cu: int32[nseg + 1].
+// groups: pp_group_desc pairs {prefix_len, num_suffixes}; cu: int32[nseg + 1]. rb = responses per query block.
 __global__ void __launch_bounds__(1024) k_dec_plan(const int32_t *__restrict__ groups, int32_t G,
-                                                   const int32_t *__restrict__ cu, int32_t nseg, int64_t T, void *ws,
-                                                   DecPlan p) {
+                                                   const int32_t *__restrict__ cu, int32_t nseg, int64_t T, int rb,
+                                                   void *ws, DecPlan p) {
     __shared__ int32_t s_tmp[1024];
     __shared__ int32_t s_bad;
     int32_t *first_seg = dec_ptr<int32_t>(ws, p.off_first_seg);
     int32_t *seg_group = dec_ptr<int32_t>(ws, p.off_seg_group);
     int32_t *unit_off = dec_ptr<int32_t>(ws, p.off_unit_off);
     int32_t *pair_off = dec_ptr<int32_t>(ws, p.off_pair_off);
+    int32_t *job_off = dec_ptr<int32_t>(ws, p.off_job_off);
     int32_t *counts = dec_ptr<int32_t>(ws, p.off_counts);
     if (threadIdx.x == 0) s_bad = (cu[0] != 0 || int64_t(cu[nseg]) != T) ? 1 : 0;
     __syncthreads();
@@ -91,6 +101,7 @@ __global__ void __launch_bounds__(1024) k_dec_plan(const int32_t *__restrict__ g
             counts[0] = 0;
             counts[1] = 0;
             counts[2] = 0;
+            counts[3] = 0;
         }
         return;
     }
@@ -102,150 +113,308 @@ __global__ void __launch_bounds__(1024) k_dec_plan(const int32_t *__restrict__ g
         const int32_t q_per = (s == first_seg[g]) ? groups[2 * g + 1] : 1;
         unit_off[s] = nch;
         pair_off[s] = nch * q_per;
+        job_off[s] = nch * ((q_per + rb - 1) / rb);
     }
     if (threadIdx.x == 0) {
         unit_off[nseg] = 0;
         pair_off[nseg] = 0;
+        job_off[nseg] = 0;
     }
     __syncthreads();
     const int32_t U = block_exclusive_scan<1024>(unit_off, nseg + 1, s_tmp);
     __syncthreads();
     const int32_t NP = block_exclusive_scan<1024>(pair_off, nseg + 1, s_tmp);
+    __syncthreads();
+    const int32_t NJ = block_exclusive_scan<1024>(job_off, nseg + 1, s_tmp);
     if (threadIdx.x == 0) {
         const bool fits = int64_t(NP) <= p.max_pairs;
         if (!fits) atomicOr(&g_dev_err, DEVERR_BAD_GROUPS);   // descriptors differ from the sized ones
         counts[0] = fits ? U : 0;
         counts[1] = NP;
         counts[2] = fits ? 1 : 0;
+        counts[3] = fits ? NJ : 0;
     }
 }
 
-// q: [n_resp, hq, D] (one query per response, responses in packed order); k, v: [T, hkv, D] cache.
-__global__ void __launch_bounds__(DEC_THREADS) k_dec_partial(const __nv_bfloat16 *__restrict__ q,
-                                                             const __nv_bfloat16 *__restrict__ k,
-                                                             const __nv_bfloat16 *__restrict__ v,
-                                                             const int32_t *__restrict__ groups, int32_t G,
-                                                             const int32_t *__restrict__ cu, int32_t nseg, int hq,
-                                                             int hkv, float sl2, void *ws, DecPlan p) {
-    extern __shared__ float dsm[];
-    float *sK = dsm;                                           // [DEC_CH][DEC_LD]
-    float *sV = sK + DEC_CH * DEC_LD;                          // [DEC_CH][DEC_D]
-    float *sQ = sV + DEC_CH * DEC_LD;                          // [DEC_MAXQ][DEC_LD]
-    float *sS = sQ + DEC_MAXQ * DEC_LD;                        // [DEC_MAXQ][DEC_CH]
-    __shared__ float s_m[DEC_MAXQ], s_l[DEC_MAXQ];
+struct DecSmem {
+    static constexpr int TILE = 128 * DEC_D * 2;        // 128 rows x d bf16 (two 64-column 128-byte-swizzled chunks)
+    static constexpr int CHUNK = 128 * 64 * 2;
+    alignas(1024) uint8_t q[TILE];
+    alignas(1024) uint8_t k[DEC_STAGES][TILE];
+    alignas(1024) uint8_t v[DEC_STAGES][TILE];
+    uint64_t q_full, q_empty;
+    uint64_t k_full[DEC_STAGES], k_empty[DEC_STAGES], v_full[DEC_STAGES], v_empty[DEC_STAGES];
+    uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+    uint32_t tmem_base;
+    int abort_flag;
+};
+static_assert(sizeof(DecSmem) + 1024 <= 232448, "decode kernel shared memory exceeds 227 KB");
+
+// One job: chunk j of segment s for kv head kh and query block qb.
+struct DecJob {
+    int s, j, qb, kh;
+    int y0, yend;         // packed keys [y0, min(y0 + DEC_CH, yend)) of the chunk
+    int r0;               // response ordinal of the block's first query row
+    int nq;               // responses of this block that see the chunk (<= rb)
+    int64_t pbase;        // record of (this chunk, the block's first response)
+};
+
+__device__ __forceinline__ DecJob dec_job(const void *ws, const DecPlan &p, const int32_t *__restrict__ groups,
+                                          const int32_t *__restrict__ cu, int nseg, int J, int rb, int64_t jj) {
     const int32_t *first_seg = dec_ptr<int32_t>(ws, p.off_first_seg);
     const int32_t *seg_group = dec_ptr<int32_t>(ws, p.off_seg_group);
-    const int32_t *unit_off = dec_ptr<int32_t>(ws, p.off_unit_off);
     const int32_t *pair_off = dec_ptr<int32_t>(ws, p.off_pair_off);
-    const int32_t U = dec_ptr<int32_t>(ws, p.off_counts)[0];
-    float *part = dec_ptr<float>(ws, p.off_part);
+    const int32_t *job_off = dec_ptr<int32_t>(ws, p.off_job_off);
+    DecJob d;
+    d.kh = int(jj / J);
+    const int jl = int(jj % J);
+    d.s = upper_bound_i32(job_off, nseg + 1, jl) - 1;         // job_off[s] <= jl < job_off[s + 1]
+    const int g = seg_group[d.s];
+    const bool prefix = d.s == first_seg[g];
+    const int cnt = prefix ? groups[2 * g + 1] : 1;             // queries that see the segment
+    const int len = cu[d.s + 1] - cu[d.s];
+    const int nch = (len + DEC_CH - 1) / DEC_CH;
+    const int w = jl - job_off[d.s];                            // (query block, chunk), chunks fastest: one Q load
+    d.qb = w / nch;                                             // serves all chunks of the segment
+    d.j = w % nch;
+    d.y0 = cu[d.s] + d.j * DEC_CH;
+    d.yend = cu[d.s + 1];
+    const int resp0 = prefix ? first_seg[g] - g : d.s - g - 1;  // response ordinal = segment - group - 1
+    d.r0 = resp0 + d.qb * rb;
+    d.nq = min(rb, cnt - d.qb * rb);
+    d.pbase = int64_t(pair_off[d.s]) + int64_t(d.j) * cnt + int64_t(d.qb) * rb;
+    return d;
+}
+
+// q: [n_resp, hq, D] (one query per response, responses in packed order); k, v: [T, hkv, D] cache.
+// tmQ: 3-D map over q (d, hq, n_resp) with box (64, r, rb); tmK/tmV: 3-D maps over the cache, box (64, 1, 128).
+__global__ void __launch_bounds__(DEC_THREADS, 1)
+k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+            const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ groups, const int32_t *__restrict__ cu,
+            int32_t nseg, int hq, int hkv, int rb, int32_t n_resp, float sl2, void *ws, DecPlan p) {
+    extern __shared__ uint8_t smem_raw[];
+    DecSmem &sm = *reinterpret_cast<DecSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = hq / hkv;
-    for (int64_t w = blockIdx.x; w < int64_t(U) * hkv; w += gridDim.x) {
-        const int u = int(w / hkv), kh = int(w % hkv);
-        const int s = upper_bound_i32(unit_off, nseg + 1, u) - 1;   // unit_off[s] <= u < unit_off[s + 1]
-        const int j = u - unit_off[s];
-        const int g = seg_group[s];
-        const bool prefix = s == first_seg[g];
-        const int k_g = groups[2 * g + 1];
-        const int y0 = cu[s] + j * DEC_CH;
-        const int n = min(DEC_CH, cu[s + 1] - y0);
-        // queries that see this chunk: responses [r0, r0 + cnt) (response ordinal = segment - group - 1)
-        const int r0 = prefix ? first_seg[g] - g : s - g - 1;
-        const int cnt = prefix ? k_g : 1;
-        const int64_t pbase = int64_t(pair_off[s]) + int64_t(j) * cnt;   // pair of (this chunk, query r0)
-        // chunk K/V (kv head kh) into shared memory as fp32
-        for (int e = threadIdx.x; e < DEC_CH * (DEC_D / 8); e += DEC_THREADS) {
-            const int row = e / (DEC_D / 8), c8 = (e % (DEC_D / 8)) * 8;
-            float kv[2][8];
-            if (row < n) {
-                const int64_t off = (int64_t(y0 + row) * hkv + kh) * DEC_D + c8;
-                const uint4 uk = *reinterpret_cast<const uint4 *>(k + off);
-                const uint4 uv = *reinterpret_cast<const uint4 *>(v + off);
-                const uint32_t wk[4] = {uk.x, uk.y, uk.z, uk.w}, wv[4] = {uv.x, uv.y, uv.z, uv.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    kv[0][2 * i] = __uint_as_float(wk[i] << 16);
-                    kv[0][2 * i + 1] = __uint_as_float(wk[i] & 0xffff0000u);
-                    kv[1][2 * i] = __uint_as_float(wv[i] << 16);
-                    kv[1][2 * i + 1] = __uint_as_float(wv[i] & 0xffff0000u);
+    const int32_t J = dec_ptr<int32_t>(ws, p.off_counts)[3];
+    const int64_t n_jobs = int64_t(J) * hkv;
+    // contiguous job range per CTA: consecutive jobs share a query block (one Q load per segment and kv head)
+    const int64_t j_begin = n_jobs * blockIdx.x / gridDim.x, j_end = n_jobs * (blockIdx.x + 1) / gridDim.x;
+    volatile int *abort_flag = &sm.abort_flag;
+    float *part = dec_ptr<float>(ws, p.off_part);
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.q_full, 1);
+        mbar_init(&sm.q_empty, 1);
+        for (int s = 0; s < DEC_STAGES; ++s) {
+            mbar_init(&sm.k_full[s], 1);
+            mbar_init(&sm.k_empty[s], 1);
+            mbar_init(&sm.v_full[s], 1);
+            mbar_init(&sm.v_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.s_full[b], 1);
+            mbar_init(&sm.p_full[b], 128);
+            mbar_init(&sm.o_full[b], 1);
+            mbar_init(&sm.o_free[b], 128);
+        }
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    if (warp == 4 && lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    // TMEM: S_b [128 b, 128 b + 128), O_b [256 + 128 b, ...); P_b (bf16) over the first 64 columns of S_b
+    auto same_q = [&](const DecJob &a, const DecJob &b) { return a.kh == b.kh && a.r0 == b.r0; };
+
+    if (J == 0) {
+        // nothing planned (or the plan did not fit: the combine kernel reports it)
+    } else if (warp == 4) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t nq_loads = 0;
+            DecJob prev{};
+            for (int64_t jj = j_begin; jj < j_end; ++jj) {
+                const DecJob d = dec_job(ws, p, groups, cu, nseg, J, rb, jj);
+                const uint32_t u = uint32_t(jj - j_begin);
+                if (u == 0 || !same_q(d, prev)) {
+                    if (!bwait(&sm.q_empty, (nq_loads & 1) ^ 1, abort_flag)) break;
+                    ++nq_loads;
+                    mbar_arrive_expect_tx(&sm.q_full, uint32_t(r * rb) * DEC_D * 2);
+                    for (int c = 0; c < DEC_D / 64; ++c)
+                        tma_load_3d(sm.q + c * DecSmem::CHUNK, &tmQ, c * 64, d.kh * r, d.r0, &sm.q_full);
                 }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) kv[0][i] = kv[1][i] = 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                sK[row * DEC_LD + c8 + i] = kv[0][i];
-                sV[row * DEC_D + c8 + i] = kv[1][i];
+                prev = d;
+                const int st = u % DEC_STAGES;
+                const uint32_t ph = ((u / DEC_STAGES) & 1) ^ 1;
+                if (!bwait(&sm.k_empty[st], ph, abort_flag)) break;
+                mbar_arrive_expect_tx(&sm.k_full[st], DecSmem::TILE);
+                for (int c = 0; c < DEC_D / 64; ++c)
+                    tma_load_3d(sm.k[st] + c * DecSmem::CHUNK, &tmK, c * 64, d.kh, d.y0, &sm.k_full[st]);
+                if (!bwait(&sm.v_empty[st], ph, abort_flag)) break;
+                mbar_arrive_expect_tx(&sm.v_full[st], DecSmem::TILE);
+                for (int c = 0; c < DEC_D / 64; ++c)
+                    tma_load_3d(sm.v[st] + c * DecSmem::CHUNK, &tmV, c * 64, d.kh, d.y0, &sm.v_full[st]);
             }
         }
-        // query vectors in passes of DEC_MAXQ: index t = response (t / r) and q head (kh * r + t % r)
-        const int m_all = cnt * r;
-        for (int t0 = 0; t0 < m_all; t0 += DEC_MAXQ) {
-            const int m = min(DEC_MAXQ, m_all - t0);
-            __syncthreads();                                   // sK/sV written; previous pass done with sQ/sS
-            for (int e = threadIdx.x; e < m * (DEC_D / 8); e += DEC_THREADS) {
-                const int t = e / (DEC_D / 8), c8 = (e % (DEC_D / 8)) * 8;
-                const int resp = r0 + (t0 + t) / r, hh = kh * r + (t0 + t) % r;
-                const uint4 uq = *reinterpret_cast<const uint4 *>(q + (int64_t(resp) * hq + hh) * DEC_D + c8);
-                const uint32_t wq[4] = {uq.x, uq.y, uq.z, uq.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    sQ[t * DEC_LD + c8 + 2 * i] = __uint_as_float(wq[i] << 16);
-                    sQ[t * DEC_LD + c8 + 2 * i + 1] = __uint_as_float(wq[i] & 0xffff0000u);
+    } else if (warp == 5) {
+        // ------------------------------------------------------------------ MMA issuer (one thread)
+        // Order: S(0), S(1), PV(0), S(2), PV(1), ... S(u + 2) overwrites the columns PV(u) reads, after it in issue
+        // order; PV(u) also waits until the record warps have read O of job u - 2 (same buffer).
+        if (lane == 0 && j_begin < j_end) {
+            constexpr uint32_t ID_S = idesc_bf16(128, DEC_CH, 0, 0);
+            constexpr uint32_t ID_O = idesc_bf16(128, DEC_D, 0, 1);
+            constexpr uint32_t TB = DecSmem::TILE;
+            const uint64_t q_desc = smem_desc(smem_u32(sm.q), 16, 1024);
+            const uint64_t k_desc = smem_desc(smem_u32(sm.k[0]), 16, 1024);
+            const uint64_t v_desc = smem_desc(smem_u32(sm.v[0]), DecSmem::CHUNK, 1024);
+            const uint32_t nu = uint32_t(j_end - j_begin);
+            uint32_t nq_used = 0;
+            DecJob prev{};
+            auto issue_s = [&](uint32_t u) -> bool {
+                const DecJob d = dec_job(ws, p, groups, cu, nseg, J, rb, j_begin + u);
+                if (u == 0 || !same_q(d, prev)) {
+                    if (u > 0) umma_commit(&sm.q_empty);                 // the previous block's last S is issued
+                    if (!bwait(&sm.q_full, nq_used & 1, abort_flag)) return false;
+                    ++nq_used;
                 }
+                prev = d;
+                const int st = u % DEC_STAGES;
+                if (!bwait(&sm.k_full[st], (u / DEC_STAGES) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint64_t b = k_desc + uint64_t(st) * (TB >> 4);
+                const uint32_t dst = tmem + 128 * (u & 1);
+#pragma unroll
+                for (int kk = 0; kk < DEC_D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * DecSmem::CHUNK + (kk & 3) * 32;
+                    umma_ss(dst, desc_adv(q_desc, off), desc_adv(b, off), ID_S, kk > 0);
+                }
+                umma_commit(&sm.s_full[u & 1]);
+                umma_commit(&sm.k_empty[st]);
+                return true;
+            };
+            bool ok = issue_s(0) && (nu < 2 || issue_s(1));
+            for (uint32_t u = 0; ok && u < nu; ++u) {
+                const int b = u & 1, st = u % DEC_STAGES;
+                if (!bwait(&sm.p_full[b], (u >> 1) & 1, abort_flag)) break;
+                if (!bwait(&sm.o_free[b], ((u >> 1) & 1) ^ 1, abort_flag)) break;
+                if (!bwait(&sm.v_full[st], (u / DEC_STAGES) & 1, abort_flag)) break;
+                tc_fence_after();
+                const uint64_t bv = v_desc + uint64_t(st) * (TB >> 4);
+#pragma unroll
+                for (int kk = 0; kk < DEC_CH / 16; ++kk)
+                    umma_ts(tmem + 256 + 128 * b, tmem + 128 * b + kk * 8, desc_adv(bv, kk * 2048), ID_O, kk > 0);
+                umma_commit(&sm.o_full[b]);
+                umma_commit(&sm.v_empty[st]);
+                if (u + 2 < nu) ok = issue_s(u + 2);
             }
-            __syncthreads();
-            // scores in base-2 units: S[t][c] = q_t . k_c * scale * log2(e)
-            for (int e = threadIdx.x; e < m * DEC_CH; e += DEC_THREADS) {
-                const int t = e / DEC_CH, c = e % DEC_CH;
-                float acc = -INFINITY;
-                if (c < n) {
-                    const float4 *qa = reinterpret_cast<const float4 *>(sQ + t * DEC_LD);
-                    const float4 *ka = reinterpret_cast<const float4 *>(sK + c * DEC_LD);
-                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-                    for (int i = 0; i < DEC_D / 4; ++i) {
-                        const float4 x = qa[i], y = ka[i];
-                        a0 = fmaf(x.x, y.x, a0);
-                        a1 = fmaf(x.y, y.y, a1);
-                        a2 = fmaf(x.z, y.z, a2);
-                        a3 = fmaf(x.w, y.w, a3);
+            if (ok) umma_commit(&sm.q_empty);
+        }
+    } else {
+        // ------------------------------------------------------------------ softmax and record warps (0-3)
+        // Thread = query row t of the block (TMEM lane): response r0 + t / r, q head kh * r + t % r. Per job: P(u)
+        // into S_b, then the record of job u - 1 from O_{b'}; warps whose rows are all idle skip the TMEM traffic.
+        const int t = threadIdx.x;
+        const uint32_t lane_off = uint32_t(warp * 32) << 16;
+        const int tr = t / r, th = t % r;
+        const uint32_t nu = uint32_t(j_end - j_begin);
+        float m_prev = 0.f, l_prev = 0.f;
+        bool v_prev = false;
+        int64_t rec_prev = 0;
+        auto record = [&](uint32_t u) -> bool {                 // O of job u -> its record
+            const int b = u & 1;
+            if (!bwait(&sm.o_full[b], (u >> 1) & 1, abort_flag)) return false;
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, v_prev)) {
+#pragma unroll
+                for (int c = 0; c < DEC_D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_off + 256 + 128 * b + 32 * c, o);
+                    tmem_wait_ld(o);
+                    if (v_prev) {
+                        float4 *dst = reinterpret_cast<float4 *>(part + rec_prev + 4 + 32 * c);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                                 __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
                     }
-                    acc = ((a0 + a1) + (a2 + a3)) * sl2;
                 }
-                sS[t * DEC_CH + c] = acc;
+                if (v_prev) *reinterpret_cast<float4 *>(part + rec_prev) = make_float4(m_prev, l_prev, 0.f, 0.f);
             }
-            __syncthreads();
-            // per query: max and sum of 2^(S - max); S becomes the probabilities
-            for (int t = threadIdx.x; t < m; t += DEC_THREADS) {
-                float mx = -INFINITY;
-                for (int c = 0; c < n; ++c) mx = fmaxf(mx, sS[t * DEC_CH + c]);
-                float l = 0.f;
+            tc_fence_before();
+            mbar_arrive(&sm.o_free[b]);
+            return true;
+        };
+        for (uint32_t u = 0; u < nu; ++u) {
+            const DecJob d = dec_job(ws, p, groups, cu, nseg, J, rb, j_begin + u);
+            const int b = u & 1;
+            const bool valid = t < r * rb && tr < d.nq && d.r0 + tr < n_resp;
+            const int nk = min(DEC_CH, d.yend - d.y0);             // keys of the chunk inside the segment
+            if (!bwait(&sm.s_full[b], (u >> 1) & 1, abort_flag)) goto done;
+            tc_fence_after();
+            float m = -INFINITY, l = 0.f;
+            if (__any_sync(0xffffffffu, valid)) {
+                float s[DEC_CH];
+                {
+                    uint32_t r0[32], r1[32], r2[32], r3[32];
+                    tmem_ld32(tmem + lane_off + 128 * b, r0);
+                    tmem_ld32(tmem + lane_off + 128 * b + 32, r1);
+                    tmem_ld32(tmem + lane_off + 128 * b + 64, r2);
+                    tmem_ld32(tmem + lane_off + 128 * b + 96, r3);
+                    tmem_wait_ld(r0, r1, r2, r3);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        s[e] = __uint_as_float(r0[e]);
+                        s[32 + e] = __uint_as_float(r1[e]);
+                        s[64 + e] = __uint_as_float(r2[e]);
+                        s[96 + e] = __uint_as_float(r3[e]);
+                    }
+                }
+#pragma unroll
                 for (int c = 0; c < DEC_CH; ++c) {
-                    const float pv = c < n ? exp2f(sS[t * DEC_CH + c] - mx) : 0.f;
-                    sS[t * DEC_CH + c] = pv;
-                    l += pv;
+                    s[c] = (valid && c < nk) ? s[c] * sl2 : -INFINITY;
+                    m = fmaxf(m, s[c]);
                 }
-                s_m[t] = mx;
-                s_l[t] = l;
-            }
-            __syncthreads();
-            // un-normalised output and the partial record (max in base-2 units, sum, O[D])
-            for (int e = threadIdx.x; e < m * DEC_D; e += DEC_THREADS) {
-                const int t = e / DEC_D, dd = e % DEC_D;
-                float acc = 0.f;
-                for (int c = 0; c < n; ++c) acc = fmaf(sS[t * DEC_CH + c], sV[c * DEC_D + dd], acc);
-                const int resp_i = (t0 + t) / r, hh = kh * r + (t0 + t) % r;
-                float *rec = part + ((pbase + resp_i) * hq + hh) * (DEC_D + 2);
-                rec[2 + dd] = acc;
-                if (dd == 0) {
-                    rec[0] = s_m[t];
-                    rec[1] = s_l[t];
+                const float mu = m == -INFINITY ? 0.f : m;
+#pragma unroll
+                for (int c = 0; c < DEC_CH / 32; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ex2_approx(s[32 * c + 2 * e] - mu), p1 = ex2_approx(s[32 * c + 2 * e + 1] - mu);
+                        l += p0 + p1;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tmem + lane_off + 128 * b + 16 * c, pk);
                 }
+                tmem_wait_st();
             }
+            tc_fence_before();
+            mbar_arrive(&sm.p_full[b]);
+            if (u > 0 && !record(u - 1)) goto done;
+            v_prev = valid;
+            m_prev = m;
+            l_prev = l;
+            rec_prev = ((d.pbase + tr) * hq + d.kh * r + th) * int64_t(DEC_REC);
         }
-        __syncthreads();                                       // before the next chunk overwrites sK/sV
+        if (nu > 0 && !record(nu - 1)) goto done;
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -254,15 +423,15 @@ __global__ void __launch_bounds__(DEC_D) k_dec_combine(const int32_t *__restrict
                                                        const int32_t *__restrict__ cu, int32_t nseg, int hq,
                                                        int32_t n_resp, const void *ws, DecPlan p,
                                                        __nv_bfloat16 *__restrict__ o, float *__restrict__ lse) {
-    const int32_t *first_seg = reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + p.off_first_seg);
-    const int32_t *unit_off = reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + p.off_unit_off);
-    const int32_t *pair_off = reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + p.off_pair_off);
-    const float *part = reinterpret_cast<const float *>(static_cast<const char *>(ws) + p.off_part);
-    const int32_t ok = reinterpret_cast<const int32_t *>(static_cast<const char *>(ws) + p.off_counts)[2];
+    const int32_t *first_seg = dec_ptr<int32_t>(ws, p.off_first_seg);
+    const int32_t *unit_off = dec_ptr<int32_t>(ws, p.off_unit_off);
+    const int32_t *pair_off = dec_ptr<int32_t>(ws, p.off_pair_off);
+    const float *part = dec_ptr<float>(ws, p.off_part);
+    const int32_t ok = dec_ptr<int32_t>(ws, p.off_counts)[2];
     const int dd = threadIdx.x;
     for (int64_t w = blockIdx.x; w < int64_t(n_resp) * hq; w += gridDim.x) {
         const int resp = int(w / hq), hh = int(w % hq);
-        if (!ok) {                                             // the plan did not fit: no partials were written
+        if (!ok) {                                             // the plan did not fit: no records were written
             o[(int64_t(resp) * hq + hh) * DEC_D + dd] = __float2bfloat16_rn(__int_as_float(0x7fc00000));
             if (dd == 0) lse[int64_t(hh) * n_resp + resp] = __int_as_float(0x7fc00000);
             continue;
@@ -279,13 +448,13 @@ __global__ void __launch_bounds__(DEC_D) k_dec_combine(const int32_t *__restrict
         const int so = sp + 1 + i;                              // its own segment
         float M = -INFINITY, L = 0.f, acc = 0.f;
         auto merge = [&](int64_t pair) {
-            const float *rec = part + (pair * hq + hh) * (DEC_D + 2);
+            const float *rec = part + (pair * hq + hh) * DEC_REC;
             const float m = rec[0];
             if (m == -INFINITY) return;
             const float Mn = fmaxf(M, m);
             const float a = exp2f(M - Mn), b = exp2f(m - Mn);
             L = L * a + rec[1] * b;
-            acc = acc * a + rec[2 + dd] * b;
+            acc = acc * a + rec[4 + dd] * b;
             M = Mn;
         };
         const int nch_p = unit_off[sp + 1] - unit_off[sp];

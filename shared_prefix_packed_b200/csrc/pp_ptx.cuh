@@ -248,6 +248,26 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
     return r;
 }
 
+// 2^x for a pair on the FMA pipe, so a softmax can move part of its exponentials off the MUFU unit (16 per clock
+// per SM, as many cycles as the tensor core needs for the matching MMAs). Cody-Waite style: x = n + r with
+// n = rint(x) (adding and removing 1.5 * 2^23), r in [-0.5, 0.5]; 2^r by a cubic whose coefficients were fitted for
+// this library to the relative error of 2^r on that interval (maximum 7.5e-5, below the 2^-9 of the bf16 P it
+// feeds); 2^n enters through the exponent bits. x is clamped to >= -125, so a masked -inf gives about 2^-125.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+    constexpr float M = 12582912.f;                          // 1.5 * 2^23
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = fadd2(x, make_float2(M, M));             // rint(x) in the low mantissa bits
+    const float2 n = fadd2(t, make_float2(-M, -M));
+    const float2 r = ffma2(n, make_float2(-1.f, -1.f), x);    // x - n, exact
+    float2 p = ffma2(make_float2(0.055171649903059006f, 0.055171649903059006f), r,
+                     make_float2(0.2426111251115799f, 0.2426111251115799f));
+    p = ffma2(p, r, make_float2(0.6932609677314758f, 0.6932609677314758f));
+    p = ffma2(p, r, make_float2(0.9999280571937561f, 0.9999280571937561f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
