@@ -8,7 +8,7 @@
 // of q heads sharing one kv head) in cost order. Warp roles:
 //   warps 0-3  softmax for head slot 0 (TMEM lanes 0-127 = the tile's rows)
 //   warps 4-7  softmax for head slot 1
-//   warp 8     TMA producer: Q of both heads once per item, then K and V tiles through a 2-stage ring
+//   warp 8     TMA producer: Q of both heads once per item, then K (3-stage ring, one tile ahead) and V (2 stages)
 //   warp 9     TMEM allocator and the single MMA-issuing thread
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 [384,384+d); P_h (bf16) overwrites the first
 // 64 columns of S_h once the softmax has read S_h. Per key tile the MMA thread issues, ping-ponging the heads,
@@ -18,7 +18,9 @@
 // Only the key tiles the schedule lists are visited ("PackInfer" abstract: attention directly over the packed
 // query-key regions); sibling-response tiles are never loaded. FULL tiles skip the element mask.
 // Softmax: exp2 with the scale folded in; the running max is only raised when a tile's max exceeds it by more than
-// 8 (log2 units), so the O rescale (a TMEM round trip) is rare; the result is exact up to rounding either way.
+// 8 (log2 units), so the O rescale (a TMEM round trip) is rare; the result is exact up to rounding either way. One
+// pair of exponentials in FWD_POLY_EVERY is computed on the FMA pipe (ex2_poly2) instead of the MUFU unit, whose 16
+// results per clock per SM would otherwise take as long as the tile's MMAs.
 #pragma once
 #include <cuda_bf16.h>
 #include "pp_meta.cuh"
@@ -28,7 +30,9 @@
 namespace pp {
 
 constexpr int FWD_THREADS = 320;
-constexpr int FWD_STAGES = 2;
+constexpr int FWD_KSTAGES = 3;   // K is needed one step earlier than V (S(j+1) is issued right after PV(j))
+constexpr int FWD_VSTAGES = 2;
+constexpr int FWD_POLY_EVERY = 4; // one pair in four exponentials goes to the FMA pipe (ex2_poly2)
 constexpr float FWD_RESCALE_THRESHOLD = 8.0f;
 constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;   // bounded waits: 2 s, then the kernel reports and leaves
 
@@ -81,14 +85,16 @@ struct FwdSmem {
     static constexpr int TILE_BYTES = 128 * D * 2;      // one 128-row tile of bf16 [rows][D]
     static constexpr int CHUNK_BYTES = 128 * 64 * 2;    // one 64-column swizzled chunk of such a tile
     alignas(1024) uint8_t q[2][TILE_BYTES];
-    alignas(1024) uint8_t k[FWD_STAGES][TILE_BYTES];
-    alignas(1024) uint8_t v[FWD_STAGES][TILE_BYTES];
+    alignas(1024) uint8_t k[FWD_KSTAGES][TILE_BYTES];
+    alignas(1024) uint8_t v[FWD_VSTAGES][TILE_BYTES];
     uint64_t q_full, q_empty;
-    uint64_t k_full[FWD_STAGES], k_empty[FWD_STAGES], v_full[FWD_STAGES], v_empty[FWD_STAGES];
+    uint64_t k_full[FWD_KSTAGES], k_empty[FWD_KSTAGES], v_full[FWD_VSTAGES], v_empty[FWD_VSTAGES];
     uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
     uint32_t tmem_base;
     int abort_flag;
 };
+
+static_assert(sizeof(FwdSmem<128>) + 1024 <= 232448, "forward shared memory exceeds 227 KB");
 
 struct FwdItem {
     QTile t;
@@ -128,9 +134,11 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (threadIdx.x == 0) {
         mbar_init(&sm.q_full, 1);
         mbar_init(&sm.q_empty, 1);
-        for (int s = 0; s < FWD_STAGES; ++s) {
+        for (int s = 0; s < FWD_KSTAGES; ++s) {
             mbar_init(&sm.k_full[s], 1);
             mbar_init(&sm.k_empty[s], 1);
+        }
+        for (int s = 0; s < FWD_VSTAGES; ++s) {
             mbar_init(&sm.v_full[s], 1);
             mbar_init(&sm.v_empty[s], 1);
         }
@@ -170,15 +178,22 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 for (int c = 0; c < D / 64; ++c)
                     tma_load_3d(sm.q[hs] + c * FwdSmem<D>::CHUNK_BYTES, &tmQ, c * 64, w.h0 + hs, w.t.row0,
                                 &sm.q_full);
-            for (int j = 0; j < n; ++j, ++kv_it) {
-                const int y0 = w.t.gstart + qtile_kv(w.t, j) * FWD_BN;
-                const int s = kv_it % FWD_STAGES;
-                const uint32_t ph = (kv_it / FWD_STAGES) & 1;
-                if (!bwait(&sm.k_empty[s], ph ^ 1, abort_flag)) goto done;
+            // K runs one tile ahead of V: K(j + 1) is issued before V(j), since S(j + 1) follows PV(j) directly
+            auto load_k = [&](uint32_t it, int jj) -> bool {
+                const int s = it % FWD_KSTAGES;
+                if (!bwait(&sm.k_empty[s], ((it / FWD_KSTAGES) & 1) ^ 1, abort_flag)) return false;
                 mbar_arrive_expect_tx(&sm.k_full[s], FwdSmem<D>::TILE_BYTES);
+                const int y0 = w.t.gstart + qtile_kv(w.t, jj) * FWD_BN;
                 for (int c = 0; c < D / 64; ++c)
                     tma_load_3d(sm.k[s] + c * FwdSmem<D>::CHUNK_BYTES, &tmK, c * 64, w.kh, y0, &sm.k_full[s]);
-                if (!bwait(&sm.v_empty[s], ph ^ 1, abort_flag)) goto done;
+                return true;
+            };
+            if (n > 0 && !load_k(kv_it, 0)) goto done;
+            for (int j = 0; j < n; ++j, ++kv_it) {
+                if (j + 1 < n && !load_k(kv_it + 1, j + 1)) goto done;
+                const int y0 = w.t.gstart + qtile_kv(w.t, j) * FWD_BN;
+                const int s = kv_it % FWD_VSTAGES;
+                if (!bwait(&sm.v_empty[s], ((kv_it / FWD_VSTAGES) & 1) ^ 1, abort_flag)) goto done;
                 mbar_arrive_expect_tx(&sm.v_full[s], FwdSmem<D>::TILE_BYTES);
                 for (int c = 0; c < D / 64; ++c)
                     tma_load_3d(sm.v[s] + c * FwdSmem<D>::CHUNK_BYTES, &tmV, c * 64, w.kh, y0, &sm.v_full[s]);
@@ -215,8 +230,8 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const int n = qtile_nkv(w.t);
             if (!bwait(&sm.q_full, n_it & 1, abort_flag)) goto done;
             ++n_it;
-            int st = kv_it % FWD_STAGES;
-            if (!bwait(&sm.k_full[st], (kv_it / FWD_STAGES) & 1, abort_flag)) goto done;
+            int st = kv_it % FWD_KSTAGES;
+            if (!bwait(&sm.k_full[st], (kv_it / FWD_KSTAGES) & 1, abort_flag)) goto done;
             tc_fence_after();
             for (int hs = 0; hs < w.nh; ++hs) {
                 issue_s(hs, st);
@@ -224,11 +239,11 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             umma_commit(&sm.k_empty[st]);
             for (int j = 0; j < n; ++j) {
-                st = (kv_it + j) % FWD_STAGES;
-                const int st2 = (kv_it + j + 1) % FWD_STAGES;
-                if (!bwait(&sm.v_full[st], ((kv_it + j) / FWD_STAGES) & 1, abort_flag)) goto done;
+                st = (kv_it + j) % FWD_VSTAGES;
+                const int st2 = (kv_it + j + 1) % FWD_KSTAGES;
+                if (!bwait(&sm.v_full[st], ((kv_it + j) / FWD_VSTAGES) & 1, abort_flag)) goto done;
                 bool have_next = j + 1 < n;
-                if (have_next && !bwait(&sm.k_full[st2], ((kv_it + j + 1) / FWD_STAGES) & 1, abort_flag)) goto done;
+                if (have_next && !bwait(&sm.k_full[st2], ((kv_it + j + 1) / FWD_KSTAGES) & 1, abort_flag)) goto done;
                 for (int hs = 0; hs < w.nh; ++hs) {
                     if (j == 0 && !bwait(&sm.o_free[hs], (item_cnt[hs] & 1) ^ 1, abort_flag)) goto done;
                     if (!bwait(&sm.p_full[hs], p_cnt[hs] & 1, abort_flag)) goto done;
@@ -325,8 +340,15 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const float2 x = ffma2(make_float2(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]), sl2v, nmu);
-                        const float p0 = ex2_approx(x.x);
-                        const float p1 = ex2_approx(x.y);
+                        float p0, p1;
+                        if (e % FWD_POLY_EVERY == FWD_POLY_EVERY - 1) {     // this pair on the FMA pipe
+                            const float2 pp = ex2_poly2(x);
+                            p0 = pp.x;
+                            p1 = pp.y;
+                        } else {
+                            p0 = ex2_approx(x.x);
+                            p1 = ex2_approx(x.y);
+                        }
                         ls[e & 1] = fadd2(ls[e & 1], make_float2(p0, p1));
                         pk[e] = pack_bf16x2(p0, p1);
                     }
