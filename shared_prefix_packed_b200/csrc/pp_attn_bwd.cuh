@@ -13,18 +13,19 @@
 // k_bwd_tc: a work item is (key tile of 128 rows, kv head, chunk of the query tiles that attend it). Seen from key
 // y the attending queries are one interval [y, e(y)) (pp_meta.cuh), so a key tile's query tiles are one contiguous
 // range; prefix key tiles (attended by every response of the group) get long ranges and are split into chunks so
-// the persistent grid stays balanced. Per step (query tile of 128 rows, one q head of the kv head), four MMAs, all
-// with N = 128 (an N = 64 MMA costs as long as an N = 128 one on this part):
+// the persistent grid stays balanced. Per step (query tile of 128 rows, one q head of the kv head), four products,
+// all with N = 128:
 //   S^T  = K Q^T                          TMEM S
 //   dP^T = V dO^T                         TMEM dP
-//   gradient warps, phase 1: P^T = exp(S^T - lse) -> TMEM S (bf16)          -> dV may start
-//   dV  += P^T dO        (A from TMEM)    TMEM dV
-//   gradient warps, phase 2: dS^T = scale P^T (dP^T - D) -> TMEM dP (bf16)
+//   gradient warps: read S^T (the S columns are then free for the next step), P^T = exp(S^T - lse); read dP^T,
+//                   dS^T = scale P^T (dP^T - D); P^T and dS^T (bf16) go into the dP columns they have read
 //   dK  += dS^T Q        (A from TMEM)    TMEM dK
-// Two gradient warpgroups each own half of the query columns of a step, and run dS(t) before P(t+1) so the next
-// step's P overlaps this step's dK. dK/dV stay in TMEM for the whole item; an unsplit key tile writes them as bf16,
-// a split one adds its fp32 partial into the workspace (one add per element and chunk).
-// TMEM (512 columns): S/P [0,128), dP/dS [128,256), dV [256,384), dK [384,512).
+//   dV  += P^T dO        (A from TMEM)    TMEM dV
+// Two threads issue the MMAs: one S^T and dP^T, the other dK and dV (a thread needs about 50 cycles to issue an
+// MMA, so one issuer that also polls barriers would starve the tensor pipe). dK/dV stay in TMEM for the whole item;
+// an unsplit key tile writes them as bf16, a split one adds its fp32 partial into the workspace (one add per element
+// and chunk).
+// TMEM (512 columns): S [0,128), dP / (P^T, dS^T) [128,256), dV [256,384), dK [384,512).
 // Per-query values folded into the MMAs: the gradient warps own a key row each and would otherwise need the lse
 // and D of all 128 query columns per step (a shared-memory or shuffle broadcast per element, which measured
 // several times slower than the exp itself). Instead one extra K = 16 slice is appended to the S^T and dP^T
@@ -33,11 +34,12 @@
 // P^T = exp2(S'^T * scale * log2 e) and dS^T = P^T * dP'^T * scale need nothing but the TMEM values. The extra
 // slices cost 2 of 34 MMAs per step. They live in shared memory as 128 x 16 bf16 tiles in the no-swizzle
 // core-matrix layout; the producer warp writes the query side for each step.
-// Q/dO tiles come through a 2-stage ring, prefetched into L2 two steps ahead.
+// Q/dO tiles come through 2-stage rings with separate barriers (Q is freed by dK, dO by dV), prefetched into L2 two
+// steps ahead.
 // Work items run in cost order within groups of four kv heads (bwd_item_split): cost order balances the static
 // round-robin, and the head groups bound the Q/dO rows that concurrently running items read, so they are reused
-// from L2 across key tiles. Each item's metadata is loaded one item ahead, and an item's epilogue (dK/dV out of
-// TMEM) runs after the next item's first P, so the next item's S^T/dP^T keep the tensor pipe busy meanwhile.
+// from L2 across key tiles. An item's epilogue (dK/dV out of TMEM) runs inside the next item's first step, between
+// its P and its dS, when dK/dV of the item have long been complete.
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -48,7 +50,7 @@
 
 namespace pp {
 
-constexpr int BWD_THREADS = 320;   // 8 gradient warps, producer, MMA
+constexpr int BWD_THREADS = 352;   // 8 gradient warps, producer, two MMA issuers
 constexpr int BWD_D = 128;
 
 struct BwdWorkspace {
@@ -164,7 +166,7 @@ struct BwdSmem {
     alignas(1024) uint8_t aug_do[QSTAGES][AUG];          // query side for dP^T: split(-D)
     uint64_t k_full, k_empty, v_full, v_empty, dkv_full, dkv_free;
     uint64_t q_full[QSTAGES], q_empty[QSTAGES], do_full[QSTAGES], do_empty[QSTAGES];
-    uint64_t s_full, s_free, dp_full, pds_ready;
+    uint64_t s_full, s_free, dp_full, pds_ready, dkdv_done;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -270,6 +272,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         mbar_init(&sm.s_free, 256);
         mbar_init(&sm.dp_full, 1);
         mbar_init(&sm.pds_ready, 256);
+        mbar_init(&sm.dkdv_done, 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -390,23 +393,25 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 }
             }
         }
-    } else if (warp == 9) {
-        // ------------------------------------------------------------------ MMA issuer (one thread)
-        // One flat walk over the CTA's steps g (across items). Per step: (a) S^T(g+1) as soon as the gradient warps
-        // have read S^T(g) into registers; (b) dK(g) and dV(g) once P^T(g) and dS^T(g) are in TMEM; (c) dP^T(g+1).
-        // MMAs from one thread execute in issue order, so dP^T(g+1) may overwrite the columns that dK(g)/dV(g)
-        // read, and the gradient warps' P(g+1) overlaps dK(g), dV(g) and dP^T(g+1).
-        if (lane == 0 && int(blockIdx.x) < n_items) {
-            constexpr uint32_t ID_SDP = idesc_bf16(128, BWD_BM, 0, 0);     // S^T, dP^T (both K-major)
-            constexpr uint32_t ID_KV = idesc_bf16(128, BWD_D, 0, 1);       // dK, dV (A TMEM, B MN-major)
+    } else if (warp == 9 || warp == 10) {
+        // ------------------------------------------------------------------ MMA issuers (one thread each)
+        // Issuing one MMA takes a thread about 50 cycles, close to the 64 an N = 128 MMA runs, so a single issuer
+        // that also polls barriers leaves the tensor pipe idle; two issuers overlap one's polls with the other's
+        // MMAs. Warp 9 issues the score products, warp 10 the gradient products:
+        //   warp 9:  S^T(g+1) once the gradient warps hold S^T(g) in registers, then dP^T(g+1) once dK(g) and
+        //            dV(g) have read P^T(g) and dS^T(g) from the dP columns (dkdv_done);
+        //   warp 10: dK(g) and dV(g) once P^T(g) and dS^T(g) are in TMEM (pds_ready).
+        constexpr uint32_t ID_SDP = idesc_bf16(128, BWD_BM, 0, 0);     // S^T, dP^T (both K-major)
+        constexpr uint32_t ID_KV = idesc_bf16(128, BWD_D, 0, 1);       // dK, dV (A TMEM, B MN-major)
+        constexpr uint32_t TB = BwdSmem::TILE, AB = BwdSmem::AUG;
+        const BWork *bws = meta_ptr<BWork>(meta, hd.off_bw);
+        auto item_steps = [&](int it) { const BWork b = bws[bwd_item_split(it, hd.n_bw, hkv).x]; return (b.qb - b.qa) * r; };
+        if (warp == 9 && lane == 0 && int(blockIdx.x) < n_items) {
             // descriptors built once; a stage is a constant stride away (desc_adv)
-            constexpr uint32_t TB = BwdSmem::TILE, AB = BwdSmem::AUG;
             const uint64_t k_desc = smem_desc(smem_u32(sm.k), 16, 1024);
             const uint64_t v_desc = smem_desc(smem_u32(sm.v), 16, 1024);
-            const uint64_t q_desc = smem_desc(smem_u32(sm.q[0]), 16, 1024);          // K-major (S^T)
+            const uint64_t q_desc = smem_desc(smem_u32(sm.q[0]), 16, 1024);
             const uint64_t do_desc = smem_desc(smem_u32(sm.dout[0]), 16, 1024);
-            const uint64_t qn_desc = smem_desc(smem_u32(sm.q[0]), BwdSmem::CHUNK, 1024);      // N-major (dK)
-            const uint64_t don_desc = smem_desc(smem_u32(sm.dout[0]), BwdSmem::CHUNK, 1024);  // N-major (dV)
             const uint64_t ones_desc = smem_desc(smem_u32(sm.aug_ones), BwdSmem::AUG_LBO, BwdSmem::AUG_SBO, 0);
             const uint64_t augq_desc = smem_desc(smem_u32(sm.aug_q[0]), BwdSmem::AUG_LBO, BwdSmem::AUG_SBO, 0);
             const uint64_t augdo_desc = smem_desc(smem_u32(sm.aug_do[0]), BwdSmem::AUG_LBO, BwdSmem::AUG_SBO, 0);
@@ -420,8 +425,6 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 // the extra slice: + (1,1,1) . split(value of the query row)
                 umma_ss(d, ones_desc, aug, ID_SDP, 1u);
             };
-            const BWork *bws = meta_ptr<BWork>(meta, hd.off_bw);
-            auto item_steps = [&](int it) { const BWork b = bws[bwd_item_split(it, hd.n_bw, hkv).x]; return (b.qb - b.qa) * r; };
             // S^T(gg) (first of its item: after K lands) and dP^T(gg)
             auto issue_s = [&](uint32_t gg, bool first, uint32_t item_par, bool last) -> bool {
                 const int st = gg % BwdSmem::QSTAGES;
@@ -448,27 +451,36 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             if (!issue_s(0, true, 0, n == 1)) goto done;
             if (!issue_dp(0, true, 0, n == 1)) goto done;
             for (;;) {
-                // the step after g: (item2, t2) with n2 steps
                 int item2 = item, t2 = t + 1, n2 = n;
                 if (t2 == n) {
                     item2 = item + int(gridDim.x);
                     t2 = 0;
                     n2 = item2 < n_items ? item_steps(item2) : 0;
                 }
-                const bool have_next = item2 < n_items;
-                const bool next_first = have_next && t2 == 0;
+                if (item2 >= n_items) break;
+                const bool next_first = t2 == 0;
                 const uint32_t par2 = (it_n + (next_first ? 1u : 0u)) & 1;
-                // (a) S^T(g+1) once the gradient warps hold S^T(g) in registers
-                if (have_next) {
-                    if (!bwait(&sm.s_free, g & 1, abort_flag)) goto done;
-                    if (!issue_s(g + 1, next_first, par2, t2 + 1 == n2)) goto done;
-                }
-                // (b) dK(g) += dS^T Q, dV(g) += P^T dO (A from TMEM: P^T and dS^T in the dP columns)
-                if (!bwait(&sm.pds_ready, g & 1, abort_flag)) goto done;
-                if (t == 0 && !bwait(&sm.dkv_free, (it_n & 1) ^ 1, abort_flag)) goto done;   // last item's epilogue read
-                tc_fence_after();
-                {
+                if (!bwait(&sm.s_free, g & 1, abort_flag)) goto done;
+                if (!issue_s(g + 1, next_first, par2, t2 + 1 == n2)) goto done;
+                if (!bwait(&sm.dkdv_done, g & 1, abort_flag)) goto done;   // dK(g), dV(g) read the dP columns
+                if (!issue_dp(g + 1, next_first, par2, t2 + 1 == n2)) goto done;
+                ++g;
+                if (next_first) ++it_n;
+                item = item2;
+                t = t2;
+                n = n2;
+            }
+        } else if (warp == 10 && lane == 0) {
+            const uint64_t qn_desc = smem_desc(smem_u32(sm.q[0]), BwdSmem::CHUNK, 1024);      // N-major (dK)
+            const uint64_t don_desc = smem_desc(smem_u32(sm.dout[0]), BwdSmem::CHUNK, 1024);  // N-major (dV)
+            uint32_t g = 0, it_n = 0;
+            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+                const int n = item_steps(item);
+                for (int t = 0; t < n; ++t, ++g) {
                     const int st = g % BwdSmem::QSTAGES;
+                    if (!bwait(&sm.pds_ready, g & 1, abort_flag)) goto done;
+                    if (t == 0 && !bwait(&sm.dkv_free, (it_n & 1) ^ 1, abort_flag)) goto done;   // epilogue read
+                    tc_fence_after();
                     const uint64_t bq = qn_desc + uint64_t(st) * (TB >> 4), bdo = don_desc + uint64_t(st) * (TB >> 4);
                     const uint32_t acc0 = t > 0 ? 1u : 0u;
 #pragma unroll
@@ -481,16 +493,9 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         umma_ts(tmem + COL_DV, tmem + COL_DP + 64 * (kk >> 2) + 8 * (kk & 3),
                                 desc_adv(bdo, kk * 2048), ID_KV, kk > 0 ? 1u : acc0);
                     umma_commit(&sm.do_empty[st]);
+                    umma_commit(&sm.dkdv_done);
                     if (t + 1 == n) umma_commit(&sm.dkv_full);
                 }
-                if (!have_next) break;
-                // (c) dP^T(g+1): in issue order after dK(g), dV(g), which read these columns
-                if (!issue_dp(g + 1, next_first, par2, t2 + 1 == n2)) goto done;
-                ++g;
-                if (next_first) ++it_n;
-                item = item2;
-                t = t2;
-                n = n2;
             }
         }
     } else {

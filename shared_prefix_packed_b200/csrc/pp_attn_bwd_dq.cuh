@@ -12,10 +12,10 @@
 // Recomputing S and dP costs 16 of the 24 MMAs per tile; in exchange dQ needs no fp32 accumulator and no
 // reduction traffic (which measured about 6 TB/s at best on L2-resident data, below what the key-side kernel
 // would otherwise need).
-// Warp roles (576 threads): warps 0-15 form four gradient warpgroups, each taking 32 key columns of every tile
+// Warp roles (608 threads): warps 0-15 form four gradient warpgroups, each taking 32 key columns of every tile
 // (its own slice of S and dP, P kept packed in registers, its dS written into dP columns it has itself read);
 // warp 16 is the TMA producer (Q and dO once per item, K through a 3-stage ring, V through a 2-stage ring); warp 17
-// allocates TMEM and issues MMAs.
+// allocates TMEM and issues S and dP; warp 18 issues dQ.
 // TMEM: S [0,128), dP/dS double-buffered [128,256) and [256,384), dQ [384,512). The second dP buffer lets dP of
 // the next key tile run while dS of this one is still being formed, so the gradient warps go from P(j+1) straight
 // to dS(j+1) without waiting on dQ(j).
@@ -28,7 +28,7 @@
 
 namespace pp {
 
-constexpr int DQ_THREADS = 576;      // 16 gradient warps, producer, MMA
+constexpr int DQ_THREADS = 608;      // 16 gradient warps, producer, two MMA issuers
 constexpr int DQ_KSTAGES = 3;         // K is held from S(j) (issued one tile early) to dQ(j)
 constexpr int DQ_VSTAGES = 2;         // V only feeds dP(j)
 constexpr int DQ_GRAD = 512;          // gradient threads (4 warpgroups x 32 key columns)
@@ -42,7 +42,7 @@ struct DqSmem {
     alignas(1024) uint8_t v[DQ_VSTAGES][TILE];
     uint64_t q_full, q_empty, do_full, do_empty, dq_full, dq_free;
     uint64_t k_full[DQ_KSTAGES], k_empty[DQ_KSTAGES], v_full[DQ_VSTAGES], v_empty[DQ_VSTAGES];
-    uint64_t s_full, s_free, dp_full[2], ds_ready[2];   // ds_ready by step parity (see the gradient warps)
+    uint64_t s_full, s_free, dp_full[2], ds_ready[2], dq_done[2];   // ds_ready by step parity (see the gradient warps)
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -94,6 +94,8 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         mbar_init(&sm.dp_full[1], 1);
         mbar_init(&sm.ds_ready[0], DQ_GRAD);
         mbar_init(&sm.ds_ready[1], DQ_GRAD);
+        mbar_init(&sm.dq_done[0], 1);
+        mbar_init(&sm.dq_done[1], 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -146,19 +148,24 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 }
             }
         }
-    } else if (warp == 17) {
-        // ------------------------------------------------------------------ MMA issuer (one thread)
-        if (lane == 0) {
-            constexpr uint32_t ID_SP = idesc_bf16(128, 128, 0, 0);         // S, dP: K-major x K-major over d
-            constexpr uint32_t ID_DQ = idesc_bf16(128, 128, 0, 1);         // dQ: A = dS (TMEM), B = K N-major
+    } else if (warp == 17 || warp == 18) {
+        // ------------------------------------------------------------------ MMA issuers (one thread each)
+        // Issuing one MMA takes a thread about 50 cycles, close to the 64 an N = 128 MMA runs, so a single issuer
+        // that also polls barriers leaves the tensor pipe idle. Warp 17 issues S and dP, warp 18 issues dQ:
+        //   warp 17: S(j+1) once the gradient warps hold S(j) in registers; dP(j+1) into buffer (j+1) % 2 once dQ(j-1)
+        //            has read dS(j-1) from that buffer (dq_done);
+        //   warp 18: dQ(j) += dS(j) K(j) once dS(j) is in TMEM (ds_ready), then frees K(j).
+        constexpr uint32_t ID_SP = idesc_bf16(128, 128, 0, 0);         // S, dP: K-major x K-major over d
+        constexpr uint32_t ID_DQ = idesc_bf16(128, 128, 0, 1);         // dQ: A = dS (TMEM), B = K N-major
+        constexpr uint32_t TB = DqSmem::TILE;
+        const QTile *qts = meta_ptr<QTile>(meta, hd.off_qts);
+        if (warp == 17 && lane == 0) {
             uint32_t kv_it = 0, it_n = 0, g = 0;                           // g: global key-tile step counter
             // descriptors built once; a stage is a constant stride away (desc_adv)
-            constexpr uint32_t TB = DqSmem::TILE;
             const uint64_t q_desc = smem_desc(smem_u32(sm.q), 16, 1024);
             const uint64_t do_desc = smem_desc(smem_u32(sm.dout), 16, 1024);
             const uint64_t k_desc = smem_desc(smem_u32(sm.k[0]), 16, 1024);
             const uint64_t v_desc = smem_desc(smem_u32(sm.v[0]), 16, 1024);
-            const uint64_t kn_desc = smem_desc(smem_u32(sm.k[0]), DqSmem::CHUNK, 1024);   // N-major (dQ)
             auto issue_kk = [&](uint32_t col, uint64_t a, uint64_t b) {
                 const uint32_t d = tmem + col;
 #pragma unroll
@@ -177,37 +184,44 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 if (last) umma_commit(&sm.q_empty);
                 return true;
             };
-            // dP of key tile `it` into dP buffer `b`; frees its V stage, and dO after the item's last tile
-            auto issue_dp = [&](uint32_t it, uint32_t b, bool last) -> bool {
+            // dP of key tile `it` into dP buffer `b`; frees its V stage, and dO after the item's last tile. Buffer b
+            // last held dS(gg - 2), read by dQ(gg - 2) on the other issuer.
+            auto issue_dp = [&](uint32_t it, uint32_t gg, bool last) -> bool {
                 const int sv = it % DQ_VSTAGES;
+                if (gg >= 2 && !bwait(&sm.dq_done[gg & 1], ((gg - 2) >> 1) & 1, abort_flag)) return false;
                 if (!bwait(&sm.v_full[sv], (it / DQ_VSTAGES) & 1, abort_flag)) return false;
                 tc_fence_after();
-                issue_kk(COL_DP + 128 * b, do_desc, v_desc + uint64_t(sv) * (TB >> 4));
-                umma_commit(&sm.dp_full[b]);
+                issue_kk(COL_DP + 128 * (gg & 1), do_desc, v_desc + uint64_t(sv) * (TB >> 4));
+                umma_commit(&sm.dp_full[gg & 1]);
                 umma_commit(&sm.v_empty[sv]);
                 if (last) umma_commit(&sm.do_empty);
                 return true;
             };
-            const QTile *qts = meta_ptr<QTile>(meta, hd.off_qts);
             int n_next = blockIdx.x < n_items ? qtile_nkv(qts[blockIdx.x / hq]) : 0;
             for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
                 const int n = n_next;                                  // loaded one item ahead
                 if (item + int(gridDim.x) < n_items) n_next = qtile_nkv(qts[(item + gridDim.x) / hq]);
-                // S and dP of the first key tile. Buffer reuse is safe by issue order: dP buffer g%2 last held
-                // dS(g-2), read by dQ(g-2); the S region was released by s_free(g-1).
+                // S and dP of the first key tile; the S region was released by s_free(g - 1)
                 if (!bwait(&sm.q_full, it_n & 1, abort_flag)) goto done;
                 if (g > 0 && !bwait(&sm.s_free, (g - 1) & 1, abort_flag)) goto done;
                 if (!issue_s(kv_it, n == 1)) goto done;
                 if (!bwait(&sm.do_full, it_n & 1, abort_flag)) goto done;
-                if (!issue_dp(kv_it, g & 1, n == 1)) goto done;
+                if (!issue_dp(kv_it, g, n == 1)) goto done;
                 for (int j = 0; j < n; ++j, ++kv_it, ++g) {
                     if (j + 1 < n) {
-                        // next tile's dP into the other buffer (its dS(g-1) was read by dQ(g-1), issued earlier),
-                        // then its S once the gradient warps have read this tile's S
-                        if (!issue_dp(kv_it + 1, (g + 1) & 1, j + 2 == n)) goto done;
+                        // the next tile's dP into the other buffer, then its S once this tile's S has been read
+                        if (!issue_dp(kv_it + 1, g + 1, j + 2 == n)) goto done;
                         if (!bwait(&sm.s_free, g & 1, abort_flag)) goto done;
                         if (!issue_s(kv_it + 1, j + 2 == n)) goto done;
                     }
+                }
+            }
+        } else if (warp == 18 && lane == 0) {
+            const uint64_t kn_desc = smem_desc(smem_u32(sm.k[0]), DqSmem::CHUNK, 1024);   // N-major (dQ)
+            uint32_t kv_it = 0, it_n = 0, g = 0;
+            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+                const int n = qtile_nkv(qts[item / hq]);
+                for (int j = 0; j < n; ++j, ++kv_it, ++g) {
                     // dQ += dS K once dS is in TMEM (and, for the first tile, the last item's dQ has been read)
                     if (!bwait(&sm.ds_ready[g & 1], (g >> 1) & 1, abort_flag)) goto done;
                     if (j == 0 && !bwait(&sm.dq_free, (it_n & 1) ^ 1, abort_flag)) goto done;
@@ -221,6 +235,7 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         umma_ts(tmem + COL_DQ, ads + 32 * (kk >> 1) + 8 * (kk & 1), desc_adv(bk, kk * 2048), ID_DQ,
                                 kk > 0 ? 1u : acc0);
                     umma_commit(&sm.k_empty[sk]);
+                    umma_commit(&sm.dq_done[g & 1]);
                 }
                 umma_commit(&sm.dq_full);
             }
