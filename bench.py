@@ -67,6 +67,21 @@ def unpacked_layout(P, S):
     return Pu, Su
 
 
+def shard_groups(P, S, world):
+    """Split one batch's groups across `world` ranks, longest processing time first: groups in decreasing order of
+    their allowed pairs (their attention cost), each to the rank with the least cost so far (ties: lowest rank).
+    Groups are independent (no attention crosses them), so each rank runs its share with no data-path collective.
+    Returns one sorted list of group indices per rank."""
+    cost = [pair_count([p], [ss]) for p, ss in zip(P, S)]
+    load = [0] * world
+    parts = [[] for _ in range(world)]
+    for g in sorted(range(len(P)), key=lambda g: (-cost[g], g)):
+        r = min(range(world), key=lambda r: (load[r], r))
+        parts[r].append(g)
+        load[r] += cost[g]
+    return [sorted(x) for x in parts]
+
+
 def flops_of(name, P, S):
     w = W.WORKLOADS[name]
     pairs = pair_count(P, S)
@@ -206,6 +221,13 @@ def run_gpu(args):
     name = args.workload
     w = W.WORKLOADS[name]
     P, S = W.group_lengths(name)
+    P_all, S_all = P, S
+    if args.shard == "groups":
+        # strong scaling: one batch, its groups split across the ranks (LPT on pair cost), no data-path collective
+        mine = shard_groups(P, S, world)[rank]
+        P, S = [P[g] for g in mine], [S[g] for g in mine]
+        if not P:
+            raise SystemExit(f"rank {rank}: no group to run ({len(P_all)} groups for {world} ranks)")
     inp = W.make_inputs(name, P, S, seed=rank_tensor_seed(name, rank))
     hq, hkv, d = w.num_heads_q, w.num_heads_kv, w.head_dim
     T = W.packed_total(P, S)
@@ -272,12 +294,16 @@ def run_gpu(args):
     step_ms = [m[0].elapsed_time(m[4]) for m in marks]
     median_ms = max_over_ranks(statistics.median(step_ms), dev, dist)
     ms_per_step = max_over_ranks(ms, dev, dist) / args.steps
+    if args.shard == "groups":                     # the whole batch's useful work, once, over the slowest rank
+        _, fa, fb = flops_of(name, P_all, S_all)
+        job_flops = fa + fb
+    else:
+        job_flops = (f_fwd + f_bwd) * world
 
     extras = {}
     if not args.no_extras:
         extras = measure_extras(args, name, P, S, batch, q, k, v, dout, stream, dev)
-    total_flops = (f_fwd + f_bwd) * world
-    value = aggregate_tflops(f_fwd + f_bwd, world, ms_per_step)
+    value = job_flops / (ms_per_step * 1e-3) / 1e12
 
     # ---- end to end through the public API with pinned host buffers
     e2e = None
@@ -351,7 +377,7 @@ def run_gpu(args):
         b.record(stream)
         torch.cuda.synchronize(dev)
         te = max_over_ranks(a.elapsed_time(b) / e_steps, dev, dist)
-        e2e = {"value": round(aggregate_tflops(f_fwd + f_bwd, world, te), 2), "unit": "TFLOP/s",
+        e2e = {"value": round(job_flops / (te * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                "ms_per_step": round(te, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if world > 1:
@@ -378,12 +404,15 @@ def run_gpu(args):
     line = {
         "metric": "packed-prefix attn fwd+bwd useful TFLOP/s", "value": round(value, 2), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16"
+        "higher_is_better": True, "scaling": "strong" if args.shard == "groups" else "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16"
         else "fp32", "data": "synthetic",
         "config": {"workload": f"{name}: {w.description}", "T": T, "groups": len(P), "allowed_pairs_per_head": pairs,
                    "unpacked_pairs_per_head": unpacked_pairs(P, S), "useful_gflop_per_rank": (f_fwd + f_bwd) / 1e9,
                    "l2": f"inputs larger than L2 ({(q.numel() + k.numel() + v.numel()) * 2 / 2**20:.0f} MiB of Q/K/V "
-                         f"per rank vs 126 MiB), no flush", "parallelism": f"weak-scaled replicas x{world}"},
+                         f"per rank vs 126 MiB), no flush",
+                   "parallelism": (f"one batch's groups split across {world} ranks (LPT on pair cost)"
+                                   if args.shard == "groups" else f"weak-scaled replicas x{world}")},
         "frac_of_peak": round(value / world / peaks["bf16_tflops"], 4),
         "frac_of_peak_sustained": round(value / world / peaks["bf16_tflops_sustained"], 4)
         if peaks.get("bf16_tflops_sustained") else None,
@@ -799,6 +828,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "groups"],
+                    help="N>1: every rank its own batch (weak scaling, default) or one batch's groups split across the "
+                         "ranks by LPT on pair cost (strong scaling)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the rope/meta GB/s and the unpacked comparison measured after the timed region")
     ap.add_argument("--vocab", type=int, default=W.LOGPROB_VOCAB, help="vocabulary of the --logprobs read-out")

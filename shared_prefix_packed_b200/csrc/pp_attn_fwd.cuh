@@ -32,7 +32,7 @@ namespace pp {
 constexpr int FWD_THREADS = 320;
 constexpr int FWD_KSTAGES = 3;   // K is needed one step earlier than V (S(j+1) is issued right after PV(j))
 constexpr int FWD_VSTAGES = 2;
-constexpr int FWD_POLY_EVERY = 2; // one pair in two exponentials goes to the FMA pipe (ex2_poly2)
+constexpr int FWD_POLY_EVERY = 4; // one pair in four exponentials goes to the FMA pipe (ex2_poly2)
 constexpr float FWD_RESCALE_THRESHOLD = 8.0f;
 constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;   // bounded waits: 2 s, then the kernel reports and leaves
 

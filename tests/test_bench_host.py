@@ -23,3 +23,20 @@ def test_pair_count_matches_oracle():
     for name in ("tiny", "dpo"):
         P, S = W.group_lengths(name)
         assert bench.pair_count(P, S) == oracle.allowed_pair_count(P, S)
+
+
+def test_shard_groups_lpt_partition():
+    """Every group lands on exactly one rank, the split is deterministic, and LPT keeps the heaviest and lightest
+    rank within one group's cost of each other."""
+    for name in ("dpo", "grpo", "hetero"):
+        P, S = W.group_lengths(name)
+        costs = [bench.pair_count([p], [ss]) for p, ss in zip(P, S)]
+        for world in (1, 2, 3, 4, 8):
+            parts = bench.shard_groups(P, S, world)
+            assert len(parts) == world
+            flat = sorted(g for part in parts for g in part)
+            assert flat == list(range(len(P)))
+            loads = [sum(costs[g] for g in part) for part in parts]
+            if len(P) >= world:
+                assert max(loads) - min(loads) <= max(costs)
+            assert parts == bench.shard_groups(P, S, world)
