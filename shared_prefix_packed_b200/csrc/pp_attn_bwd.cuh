@@ -17,10 +17,12 @@
 // all with N = 128:
 //   S^T  = K Q^T                          TMEM S
 //   dP^T = V dO^T                         TMEM dP
-//   gradient warps: read S^T (the S columns are then free for the next step), P^T = exp(S^T - lse); read dP^T,
-//                   dS^T = scale P^T (dP^T - D); P^T and dS^T (bf16) go into the dP columns they have read
-//   dK  += dS^T Q        (A from TMEM)    TMEM dK
+//   gradient warps: read S^T (S^T(g+1) may then be issued), P^T = exp(S^T - lse); read dP^T; P^T (bf16) into
+//                   the dP columns they have read                                          -> dV may start
 //   dV  += P^T dO        (A from TMEM)    TMEM dV
+//   gradient warps: dS^T = scale P^T (dP^T - D) (bf16) into the other dP columns they read  -> dK may start
+//   dK  += dS^T Q        (A from TMEM)    TMEM dK
+// S^T(g+1) is issued as soon as S^T(g) is in registers, so P(g+1) overlaps dV(g), dK(g) and dP^T(g+1).
 // Two threads issue the MMAs: one S^T and dP^T, the other dK and dV (a thread needs about 50 cycles to issue an
 // MMA, so one issuer that also polls barriers would starve the tensor pipe). dK/dV stay in TMEM for the whole item;
 // an unsplit key tile writes them as bf16, a split one adds its fp32 partial into the workspace (one add per element
@@ -166,7 +168,7 @@ struct BwdSmem {
     alignas(1024) uint8_t aug_do[QSTAGES][AUG];          // query side for dP^T: split(-D)
     uint64_t k_full, k_empty, v_full, v_empty, dkv_full, dkv_free;
     uint64_t q_full[QSTAGES], q_empty[QSTAGES], do_full[QSTAGES], do_empty[QSTAGES];
-    uint64_t s_full, s_free, dp_full, pds_ready, dkdv_done;
+    uint64_t s_full, s_free, dp_full, dp_free, p_ready, ds_ready;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -269,10 +271,11 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             mbar_init(&sm.do_empty[b], 1);
         }
         mbar_init(&sm.s_full, 1);
-        mbar_init(&sm.s_free, 256);
+        mbar_init(&sm.s_free, 256);                      // the gradient warps have read S^T(g)
         mbar_init(&sm.dp_full, 1);
-        mbar_init(&sm.pds_ready, 256);
-        mbar_init(&sm.dkdv_done, 1);
+        mbar_init(&sm.dp_free, 1);                       // dV(g) and dK(g) have read P^T(g), dS^T(g) (dP columns)
+        mbar_init(&sm.p_ready, 256);
+        mbar_init(&sm.ds_ready, 256);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -398,9 +401,9 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         // Issuing one MMA takes a thread about 50 cycles, close to the 64 an N = 128 MMA runs, so a single issuer
         // that also polls barriers leaves the tensor pipe idle; two issuers overlap one's polls with the other's
         // MMAs. Warp 9 issues the score products, warp 10 the gradient products:
-        //   warp 9:  S^T(g+1) once the gradient warps hold S^T(g) in registers, then dP^T(g+1) once dK(g) and
-        //            dV(g) have read P^T(g) and dS^T(g) from the dP columns (dkdv_done);
-        //   warp 10: dK(g) and dV(g) once P^T(g) and dS^T(g) are in TMEM (pds_ready).
+        //   warp 9:  S^T(g+1) once the gradient warps hold S^T(g) in registers (s_free), then dP^T(g+1) once dV(g)
+        //            and dK(g) have read P^T(g) and dS^T(g) from the dP columns (dp_free);
+        //   warp 10: dV(g) once P^T(g) is in TMEM (p_ready), then dK(g) once dS^T(g) is (ds_ready).
         constexpr uint32_t ID_SDP = idesc_bf16(128, BWD_BM, 0, 0);     // S^T, dP^T (both K-major)
         constexpr uint32_t ID_KV = idesc_bf16(128, BWD_D, 0, 1);       // dK, dV (A TMEM, B MN-major)
         constexpr uint32_t TB = BwdSmem::TILE, AB = BwdSmem::AUG;
@@ -460,9 +463,9 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 if (item2 >= n_items) break;
                 const bool next_first = t2 == 0;
                 const uint32_t par2 = (it_n + (next_first ? 1u : 0u)) & 1;
-                if (!bwait(&sm.s_free, g & 1, abort_flag)) goto done;
+                if (!bwait(&sm.s_free, g & 1, abort_flag)) goto done;      // S^T(g) is in registers
                 if (!issue_s(g + 1, next_first, par2, t2 + 1 == n2)) goto done;
-                if (!bwait(&sm.dkdv_done, g & 1, abort_flag)) goto done;   // dK(g), dV(g) read the dP columns
+                if (!bwait(&sm.dp_free, g & 1, abort_flag)) goto done;     // dV(g), dK(g) read the dP columns
                 if (!issue_dp(g + 1, next_first, par2, t2 + 1 == n2)) goto done;
                 ++g;
                 if (next_first) ++it_n;
@@ -478,22 +481,26 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 const int n = item_steps(item);
                 for (int t = 0; t < n; ++t, ++g) {
                     const int st = g % BwdSmem::QSTAGES;
-                    if (!bwait(&sm.pds_ready, g & 1, abort_flag)) goto done;
-                    if (t == 0 && !bwait(&sm.dkv_free, (it_n & 1) ^ 1, abort_flag)) goto done;   // epilogue read
-                    tc_fence_after();
                     const uint64_t bq = qn_desc + uint64_t(st) * (TB >> 4), bdo = don_desc + uint64_t(st) * (TB >> 4);
                     const uint32_t acc0 = t > 0 ? 1u : 0u;
-#pragma unroll
-                    for (int kk = 0; kk < BWD_BM / 16; ++kk)
-                        umma_ts(tmem + COL_DK, tmem + COL_DP + 64 * (kk >> 2) + 32 + 8 * (kk & 3),
-                                desc_adv(bq, kk * 2048), ID_KV, kk > 0 ? 1u : acc0);
-                    umma_commit(&sm.q_empty[st]);
+                    // dV += P^T dO as soon as P^T is in the dP columns (the epilogue has read the last item's dV)
+                    if (!bwait(&sm.p_ready, g & 1, abort_flag)) goto done;
+                    if (t == 0 && !bwait(&sm.dkv_free, (it_n & 1) ^ 1, abort_flag)) goto done;
+                    tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < BWD_BM / 16; ++kk)
                         umma_ts(tmem + COL_DV, tmem + COL_DP + 64 * (kk >> 2) + 8 * (kk & 3),
                                 desc_adv(bdo, kk * 2048), ID_KV, kk > 0 ? 1u : acc0);
                     umma_commit(&sm.do_empty[st]);
-                    umma_commit(&sm.dkdv_done);
+                    // dK += dS^T Q once dS^T is in the dP columns
+                    if (!bwait(&sm.ds_ready, g & 1, abort_flag)) goto done;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < BWD_BM / 16; ++kk)
+                        umma_ts(tmem + COL_DK, tmem + COL_DP + 64 * (kk >> 2) + 32 + 8 * (kk & 3),
+                                desc_adv(bq, kk * 2048), ID_KV, kk > 0 ? 1u : acc0);
+                    umma_commit(&sm.q_empty[st]);
+                    umma_commit(&sm.dp_free);
                     if (t + 1 == n) umma_commit(&sm.dkv_full);
                 }
             }
@@ -501,9 +508,9 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     } else {
         // ------------------------------------------------------------------ gradient warpgroups (warps 0-7)
         // Warpgroup x handles query columns [64x, 64x+64) of every step (TMEM lane = key row). Per step: read S^T
-        // (and free it for the next step's MMA), P^T = exp2(S'^T scale log2 e); read dP^T; dS^T = scale P^T dP'^T;
-        // then P^T and dS^T (bf16) go into the 64 dP columns this warpgroup has itself read: P^T in the first 32,
-        // dS^T in the last 32.
+        // (the next step's S^T may then be issued), P^T = exp2(S'^T scale log2 e); read dP^T; P^T (bf16) into the
+        // first 32 of the 64 dP columns it reads -> p_ready (dV may start); dS^T = scale P^T dP'^T (bf16) into the
+        // last 32 -> ds_ready (dK may start). The next step's dP^T waits for both.
         const int wx = warp >> 2;                                      // column half
         const int wl = warp & 3;
         const int jr = wl * 32 + lane;                                 // TMEM lane: key row
@@ -598,11 +605,11 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     ep_row = (int64_t(y) * hkv + w.kh) * BWD_D;
                     if (nxt < n_items) ken = key_end_of(wn);
                 }
-                // dS^T = scale P^T dP'^T (dP' = dP - D already)
+                // dP^T, then P^T (bf16) into the first 32 of the 64 dP columns this warpgroup reads (dV may start),
+                // then dS^T = scale P^T dP'^T (dP' = dP - D already) into the last 32 (dK may start)
                 if (!bwait(&sm.dp_full, g & 1, abort_flag)) goto done;
                 tc_fence_after();
                 {
-                    // two halves of 32 columns, so fewer registers are live at once
                     uint32_t ds[32];
                     const float2 sc = make_float2(scale, scale);
 #pragma unroll
@@ -610,6 +617,12 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         uint32_t a0[32];
                         tmem_ld32(tmem + lane_off + COL_DP + cb + 32 * hf, a0);
                         tmem_wait_ld(a0);
+                        if (hf == 0) {                                 // these columns are read: P^T goes there
+                            tmem_st32(tmem + lane_off + COL_DP + cb, pk);
+                            tmem_wait_st();
+                            tc_fence_before();
+                            mbar_arrive(&sm.p_ready);
+                        }
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             const uint32_t p = pk[16 * hf + e];
@@ -618,12 +631,11 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                             ds[16 * hf + e] = pack_bf16x2(d2.x, d2.y);
                         }
                     }
-                    tmem_st32(tmem + lane_off + COL_DP + cb, pk);
                     tmem_st32(tmem + lane_off + COL_DP + cb + 32, ds);
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&sm.pds_ready);
+                mbar_arrive(&sm.ds_ready);
             }
         }
         if (it_n > 0 && !epilogue(it_n - 1)) goto done;

@@ -10,7 +10,8 @@
 //                query that sees the chunk (all responses of the group for a prefix chunk, one response for a
 //                response chunk) times the r q heads of the kv head, up to 128 rows, gathered by one 3-D TMA box
 //                from q [n_resp, hq, d]. S = Q K^T and O = P V run on the tensor cores (M = 128 query rows, N = 128
-//                keys, then N = d); the softmax warps own one query row each. A prefix chunk is therefore read from
+//                keys, then N = d); two softmax warpgroups take alternate jobs, each thread one query row. A prefix
+//                chunk is therefore read from
 //                HBM once per group (per query block), not once per response. Each job writes an fp32 record
 //                (max, sum, un-normalised O) per valid query row.
 //   k_dec_combine per (response, q head): merges its records (the group's prefix chunks, its own chunks).
@@ -27,7 +28,7 @@ constexpr int DEC_CH = 128;           // keys per chunk (the MMA N of S, the K o
 constexpr int DEC_D = 128;            // head dim
 constexpr int DEC_REC = 132;          // floats per record: max (base 2), sum, two pad, O[128] (16-byte aligned)
 constexpr int DEC_STAGES = 3;         // K and V chunk rings
-constexpr int DEC_THREADS = 192;      // warps 0-3 softmax / records, warp 4 TMA, warp 5 TMEM + MMA
+constexpr int DEC_THREADS = 320;      // warps 0-7 softmax / records (two warpgroups), warp 8 TMA, warp 9 MMA
 
 // Plan layout in the workspace (int32 sections, sizes from G and nseg).
 struct DecPlan {
@@ -221,11 +222,11 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == 8 && lane == 0) {
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
@@ -239,7 +240,7 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 
     if (J == 0) {
         // nothing planned (or the plan did not fit: the combine kernel reports it)
-    } else if (warp == 4) {
+    } else if (warp == 8) {
         // ------------------------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t nq_loads = 0;
@@ -267,7 +268,7 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     tma_load_3d(sm.v[st] + c * DecSmem::CHUNK, &tmV, c * 64, d.kh, d.y0, &sm.v_full[st]);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------------ MMA issuer (one thread)
         // Order: S(0), S(1), PV(0), S(2), PV(1), ... S(u + 2) overwrites the columns PV(u) reads, after it in issue
         // order; PV(u) also waits until the record warps have read O of job u - 2 (same buffer).
@@ -321,49 +322,24 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             if (ok) umma_commit(&sm.q_empty);
         }
     } else {
-        // ------------------------------------------------------------------ softmax and record warps (0-3)
-        // Thread = query row t of the block (TMEM lane): response r0 + t / r, q head kh * r + t % r. Per job: P(u)
-        // into S_b, then the record of job u - 1 from O_{b'}; warps whose rows are all idle skip the TMEM traffic.
-        const int t = threadIdx.x;
-        const uint32_t lane_off = uint32_t(warp * 32) << 16;
+        // ------------------------------------------------------------------ softmax and record warpgroups (0-7)
+        // Warpgroup b (warps 4b..4b+3) takes the jobs u with u % 2 == b, so it always uses TMEM buffer b, and the
+        // two warpgroups' chains (S -> P -> PV -> record) overlap. Thread = query row t of the block (TMEM lane):
+        // response r0 + t / r, q head kh * r + t % r. Warps whose rows are all idle skip the TMEM traffic.
+        const int b = warp >> 2;
+        const int t = threadIdx.x & 127;
+        const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
         const int tr = t / r, th = t % r;
         const uint32_t nu = uint32_t(j_end - j_begin);
-        float m_prev = 0.f, l_prev = 0.f;
-        bool v_prev = false;
-        int64_t rec_prev = 0;
-        auto record = [&](uint32_t u) -> bool {                 // O of job u -> its record
-            const int b = u & 1;
-            if (!bwait(&sm.o_full[b], (u >> 1) & 1, abort_flag)) return false;
-            tc_fence_after();
-            if (__any_sync(0xffffffffu, v_prev)) {
-#pragma unroll
-                for (int c = 0; c < DEC_D / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(tmem + lane_off + 256 + 128 * b + 32 * c, o);
-                    tmem_wait_ld(o);
-                    if (v_prev) {
-                        float4 *dst = reinterpret_cast<float4 *>(part + rec_prev + 4 + 32 * c);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            dst[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
-                                                 __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
-                    }
-                }
-                if (v_prev) *reinterpret_cast<float4 *>(part + rec_prev) = make_float4(m_prev, l_prev, 0.f, 0.f);
-            }
-            tc_fence_before();
-            mbar_arrive(&sm.o_free[b]);
-            return true;
-        };
-        for (uint32_t u = 0; u < nu; ++u) {
+        for (uint32_t u = b; u < nu; u += 2) {
             const DecJob d = dec_job(ws, p, groups, cu, nseg, J, rb, j_begin + u);
-            const int b = u & 1;
             const bool valid = t < r * rb && tr < d.nq && d.r0 + tr < n_resp;
             const int nk = min(DEC_CH, d.yend - d.y0);             // keys of the chunk inside the segment
             if (!bwait(&sm.s_full[b], (u >> 1) & 1, abort_flag)) goto done;
             tc_fence_after();
             float m = -INFINITY, l = 0.f;
-            if (__any_sync(0xffffffffu, valid)) {
+            const bool any = __any_sync(0xffffffffu, valid);
+            if (any) {
                 float s[DEC_CH];
                 {
                     uint32_t r0[32], r1[32], r2[32], r3[32];
@@ -401,18 +377,34 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             }
             tc_fence_before();
             mbar_arrive(&sm.p_full[b]);
-            if (u > 0 && !record(u - 1)) goto done;
-            v_prev = valid;
-            m_prev = m;
-            l_prev = l;
-            rec_prev = ((d.pbase + tr) * hq + d.kh * r + th) * int64_t(DEC_REC);
+            // the job's O (PV(u)) -> its record (max in base-2 units, sum, two pad, O[128])
+            if (!bwait(&sm.o_full[b], (u >> 1) & 1, abort_flag)) goto done;
+            tc_fence_after();
+            if (any) {
+                const int64_t rec = ((d.pbase + tr) * hq + d.kh * r + th) * int64_t(DEC_REC);
+#pragma unroll
+                for (int c = 0; c < DEC_D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_off + 256 + 128 * b + 32 * c, o);
+                    tmem_wait_ld(o);
+                    if (valid) {
+                        float4 *dst = reinterpret_cast<float4 *>(part + rec + 4 + 32 * c);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                                 __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+                    }
+                }
+                if (valid) *reinterpret_cast<float4 *>(part + rec) = make_float4(m, l, 0.f, 0.f);
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.o_free[b]);
         }
-        if (nu > 0 && !record(nu - 1)) goto done;
     }
 done:
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

@@ -193,7 +193,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 // the address field holds address >> 4 in its low 14 bits, so the move is one add on the 64-bit value (no carry
 // leaves the field while addresses stay below 256 KB). The MMA issue loops build each tile's descriptor once and
 // step it with these adds, so the issuing thread spends almost nothing between two tcgen05.mma instructions.
-__device__ __forceinline__ uint64_t desc_adv(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+__device__ __forceinline__ uint64_t desc_adv(uint64_t d, uint32_t bytes) {
+    // only the low word changes: one 32-bit add, and the pair is re-formed without a carry chain
+    uint64_t r;
+    asm("{\n\t.reg .b32 lo, hi;\n\tmov.b64 {lo, hi}, %1;\n\tadd.u32 lo, lo, %2;\n\tmov.b64 %0, {lo, hi};\n\t}"
+        : "=l"(r) : "l"(d), "r"(bytes >> 4));
+    return r;
+}
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D. a_mn/b_mn: operand is MN-major (1) or K-major (0).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
     return (1u << 4)                                   // D format fp32
