@@ -333,9 +333,11 @@ pp_status pp_decode_attn(const void *q, const void *k_cache, const void *v_cache
     if (r > 128) return fail(PP_ERR_UNSUPPORTED, "decode supports at most 128 q heads per kv head (got %d)", r);
     const int rb = 128 / r;                                  // responses per query block (r * rb <= 128 rows)
     const pp::DecPlan base = pp::dec_plan_layout(T, G, nseg, hq, 0);
-    const int64_t rec = 4 * int64_t(hq) * pp::DEC_REC;
-    if (ws_bytes < base.off_part + rec) return fail(PP_ERR_WORKSPACE, "workspace too small for the decode plan");
-    const pp::DecPlan p = pp::dec_plan_layout(T, G, nseg, hq, (ws_bytes - base.off_part) / rec);
+    const int64_t rec = 4 * int64_t(hq) * pp::DEC_REC + 32;   // one record per q head, and one job entry
+    if (ws_bytes < base.off_jobs + rec) return fail(PP_ERR_WORKSPACE, "workspace too small for the decode plan");
+    int64_t mp = (ws_bytes - base.off_jobs) / rec;            // upper bound; trimmed for the sections' alignment
+    while (mp > 0 && pp::dec_plan_layout(T, G, nseg, hq, mp).total > ws_bytes) --mp;
+    const pp::DecPlan p = pp::dec_plan_layout(T, G, nseg, hq, mp);
     DeviceInfo *di;
     if ((st = device_info(&di)) != PP_OK) return st;
     CUtensorMap mq, mk, mv;

@@ -32,6 +32,7 @@ constexpr int DQ_THREADS = 608;      // 16 gradient warps, producer, two MMA iss
 constexpr int DQ_KSTAGES = 3;         // K is held from S(j) (issued one tile early) to dQ(j)
 constexpr int DQ_VSTAGES = 2;         // V only feeds dP(j)
 constexpr int DQ_GRAD = 512;          // gradient threads (4 warpgroups x 32 key columns)
+constexpr int DQ_POLY_EVERY = 4;      // one exponential pair in four on the FMA pipe (ex2_poly2), the rest on MUFU
 
 struct DqSmem {
     static constexpr int TILE = 128 * 128 * 2;
@@ -329,8 +330,15 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         const int c = 2 * e;
                         const float2 x = ffma2(make_float2(__uint_as_float(a0[c]), __uint_as_float(a0[c + 1])), sl2v,
                                                c0v);
-                        float p0 = ex2_approx(x.x);
-                        float p1 = ex2_approx(x.y);
+                        float p0, p1;
+                        if (e % DQ_POLY_EVERY == DQ_POLY_EVERY - 1) {       // this pair on the FMA pipe
+                            const float2 pp = ex2_poly2(x);
+                            p0 = pp.x;
+                            p1 = pp.y;
+                        } else {
+                            p0 = ex2_approx(x.x);
+                            p1 = ex2_approx(x.y);
+                        }
                         if (cls != TILE_FULL) {
                             if (!(c <= lim_diag && (c < lim_pfx || c >= lim_seg))) p0 = 0.f;
                             if (!(c + 1 <= lim_diag && (c + 1 < lim_pfx || c + 1 >= lim_seg))) p1 = 0.f;

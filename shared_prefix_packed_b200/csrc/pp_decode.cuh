@@ -38,6 +38,7 @@ struct DecPlan {
     int64_t off_pair_off;    // [nseg + 1] (chunk, query) records before each segment
     int64_t off_job_off;     // [nseg + 1] jobs (chunk, query block) before each segment
     int64_t off_counts;      // [4]: units, records, ok (1 if the plan fits), jobs
+    int64_t off_jobs;        // DecJobRec[max_pairs]: every job decoded once (jobs <= records)
     int64_t off_part;        // fp32 records: [pairs][hq][DEC_REC]
     int64_t total;
     int64_t max_pairs;       // records the workspace holds
@@ -57,6 +58,7 @@ __host__ inline DecPlan dec_plan_layout(int64_t T, int32_t G, int32_t nseg, int3
     p.off_pair_off = o;  o = dec_a256(o + 4 * int64_t(nseg + 1));
     p.off_job_off = o;   o = dec_a256(o + 4 * int64_t(nseg + 1));
     p.off_counts = o;    o = dec_a256(o + 16);
+    p.off_jobs = o;      o = dec_a256(o + 32 * max_pairs);
     p.off_part = o;      o = dec_a256(o + 4 * max_pairs * hq * DEC_REC);
     p.total = o;
     p.max_pairs = max_pairs;
@@ -70,6 +72,15 @@ template <typename T> __device__ __forceinline__ T *dec_ptr(void *ws, int64_t of
 template <typename T> __device__ __forceinline__ const T *dec_ptr(const void *ws, int64_t off) {
     return reinterpret_cast<const T *>(static_cast<const char *>(ws) + off);
 }
+
+// One job (a 128-key chunk of a segment x a query block), decoded once by the plan kernel so that the roles of the
+// chunk kernel read it with one load instead of searching the segment offsets.
+struct alignas(16) DecJobRec {
+    int32_t y0, yend;    // packed keys [y0, min(y0 + DEC_CH, yend)) of the chunk
+    int32_t r0, nq;      // first response of the query block and how many of its responses see the chunk
+    int32_t pbase;       // record of (this chunk, the block's first response)
+    int32_t pad[3];
+};
 
 // groups: pp_group_desc pairs {prefix_len, num_suffixes}; cu: int32[nseg + 1]. rb = responses per query block.
 __global__ void __launch_bounds__(1024) k_dec_plan(const int32_t *__restrict__ groups, int32_t G,
@@ -127,6 +138,28 @@ __global__ void __launch_bounds__(1024) k_dec_plan(const int32_t *__restrict__ g
     const int32_t NP = block_exclusive_scan<1024>(pair_off, nseg + 1, s_tmp);
     __syncthreads();
     const int32_t NJ = block_exclusive_scan<1024>(job_off, nseg + 1, s_tmp);
+    if (int64_t(NP) <= p.max_pairs) {                          // the job table (NJ <= NP entries) fits too
+        DecJobRec *jobs = dec_ptr<DecJobRec>(ws, p.off_jobs);
+        for (int s = threadIdx.x; s < nseg; s += blockDim.x) {
+            const int g = seg_group[s];
+            const bool prefix = s == first_seg[g];
+            const int cnt = prefix ? groups[2 * g + 1] : 1;    // queries that see the segment
+            const int nch = unit_off[s + 1] - unit_off[s];
+            const int resp0 = prefix ? first_seg[g] - g : s - g - 1;   // response ordinal = segment - group - 1
+            const int nw = job_off[s + 1] - job_off[s];
+            for (int w = 0; w < nw; ++w) {                     // (query block, chunk), chunks fastest: one Q load
+                const int qb = w / nch, j = w % nch;           // serves all chunks of the segment
+                DecJobRec r;
+                r.y0 = cu[s] + j * DEC_CH;
+                r.yend = cu[s + 1];
+                r.r0 = resp0 + qb * rb;
+                r.nq = min(rb, cnt - qb * rb);
+                r.pbase = pair_off[s] + j * cnt + qb * rb;
+                r.pad[0] = r.pad[1] = r.pad[2] = 0;
+                jobs[job_off[s] + w] = r;
+            }
+        }
+    }
     if (threadIdx.x == 0) {
         const bool fits = int64_t(NP) <= p.max_pairs;
         if (!fits) atomicOr(&g_dev_err, DEVERR_BAD_GROUPS);   // descriptors differ from the sized ones
@@ -151,39 +184,24 @@ struct DecSmem {
 };
 static_assert(sizeof(DecSmem) + 1024 <= 232448, "decode kernel shared memory exceeds 227 KB");
 
-// One job: chunk j of segment s for kv head kh and query block qb.
+// One job: chunk of one segment, kv head kh, one query block.
 struct DecJob {
-    int s, j, qb, kh;
+    int kh;
     int y0, yend;         // packed keys [y0, min(y0 + DEC_CH, yend)) of the chunk
     int r0;               // response ordinal of the block's first query row
     int nq;               // responses of this block that see the chunk (<= rb)
     int64_t pbase;        // record of (this chunk, the block's first response)
 };
 
-__device__ __forceinline__ DecJob dec_job(const void *ws, const DecPlan &p, const int32_t *__restrict__ groups,
-                                          const int32_t *__restrict__ cu, int nseg, int J, int rb, int64_t jj) {
-    const int32_t *first_seg = dec_ptr<int32_t>(ws, p.off_first_seg);
-    const int32_t *seg_group = dec_ptr<int32_t>(ws, p.off_seg_group);
-    const int32_t *pair_off = dec_ptr<int32_t>(ws, p.off_pair_off);
-    const int32_t *job_off = dec_ptr<int32_t>(ws, p.off_job_off);
+__device__ __forceinline__ DecJob dec_job(const void *ws, const DecPlan &p, int J, int64_t jj) {
+    const DecJobRec r = dec_ptr<DecJobRec>(ws, p.off_jobs)[jj % J];
     DecJob d;
     d.kh = int(jj / J);
-    const int jl = int(jj % J);
-    d.s = upper_bound_i32(job_off, nseg + 1, jl) - 1;         // job_off[s] <= jl < job_off[s + 1]
-    const int g = seg_group[d.s];
-    const bool prefix = d.s == first_seg[g];
-    const int cnt = prefix ? groups[2 * g + 1] : 1;             // queries that see the segment
-    const int len = cu[d.s + 1] - cu[d.s];
-    const int nch = (len + DEC_CH - 1) / DEC_CH;
-    const int w = jl - job_off[d.s];                            // (query block, chunk), chunks fastest: one Q load
-    d.qb = w / nch;                                             // serves all chunks of the segment
-    d.j = w % nch;
-    d.y0 = cu[d.s] + d.j * DEC_CH;
-    d.yend = cu[d.s + 1];
-    const int resp0 = prefix ? first_seg[g] - g : d.s - g - 1;  // response ordinal = segment - group - 1
-    d.r0 = resp0 + d.qb * rb;
-    d.nq = min(rb, cnt - d.qb * rb);
-    d.pbase = int64_t(pair_off[d.s]) + int64_t(d.j) * cnt + int64_t(d.qb) * rb;
+    d.y0 = r.y0;
+    d.yend = r.yend;
+    d.r0 = r.r0;
+    d.nq = r.nq;
+    d.pbase = r.pbase;
     return d;
 }
 
@@ -246,7 +264,7 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             uint32_t nq_loads = 0;
             DecJob prev{};
             for (int64_t jj = j_begin; jj < j_end; ++jj) {
-                const DecJob d = dec_job(ws, p, groups, cu, nseg, J, rb, jj);
+                const DecJob d = dec_job(ws, p, J, jj);
                 const uint32_t u = uint32_t(jj - j_begin);
                 if (u == 0 || !same_q(d, prev)) {
                     if (!bwait(&sm.q_empty, (nq_loads & 1) ^ 1, abort_flag)) break;
@@ -283,7 +301,7 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             uint32_t nq_used = 0;
             DecJob prev{};
             auto issue_s = [&](uint32_t u) -> bool {
-                const DecJob d = dec_job(ws, p, groups, cu, nseg, J, rb, j_begin + u);
+                const DecJob d = dec_job(ws, p, J, j_begin + u);
                 if (u == 0 || !same_q(d, prev)) {
                     if (u > 0) umma_commit(&sm.q_empty);                 // the previous block's last S is issued
                     if (!bwait(&sm.q_full, nq_used & 1, abort_flag)) return false;
@@ -332,7 +350,7 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int tr = t / r, th = t % r;
         const uint32_t nu = uint32_t(j_end - j_begin);
         for (uint32_t u = b; u < nu; u += 2) {
-            const DecJob d = dec_job(ws, p, groups, cu, nseg, J, rb, j_begin + u);
+            const DecJob d = dec_job(ws, p, J, j_begin + u);
             const bool valid = t < r * rb && tr < d.nq && d.r0 + tr < n_resp;
             const int nk = min(DEC_CH, d.yend - d.y0);             // keys of the chunk inside the segment
             if (!bwait(&sm.s_full[b], (u >> 1) & 1, abort_flag)) goto done;
