@@ -334,8 +334,8 @@ pp_status pp_decode_attn(const void *q, const void *k_cache, const void *v_cache
     const int rb = 128 / r;                                  // responses per query block (r * rb <= 128 rows)
     const pp::DecPlan base = pp::dec_plan_layout(T, G, nseg, hq, 0);
     const int64_t rec = 4 * int64_t(hq) * pp::DEC_REC + 32;   // one record per q head, and one job entry
-    if (ws_bytes < base.off_jobs + rec) return fail(PP_ERR_WORKSPACE, "workspace too small for the decode plan");
-    int64_t mp = (ws_bytes - base.off_jobs) / rec;            // upper bound; trimmed for the sections' alignment
+    if (ws_bytes < base.total + rec) return fail(PP_ERR_WORKSPACE, "workspace too small for the decode plan");
+    int64_t mp = (ws_bytes - base.total) / rec;               // upper bound; trimmed for the sections' alignment
     while (mp > 0 && pp::dec_plan_layout(T, G, nseg, hq, mp).total > ws_bytes) --mp;
     const pp::DecPlan p = pp::dec_plan_layout(T, G, nseg, hq, mp);
     DeviceInfo *di;
@@ -354,8 +354,8 @@ pp_status pp_decode_attn(const void *q, const void *k_cache, const void *v_cache
     pp::k_dec_chunk<<<di->sm_count, pp::DEC_THREADS, smem, s>>>(mq, mk, mv, gd, cu_d, nseg, hq, hkv, rb, n_resp,
                                                                   scale * 1.4426950408889634f, workspace, p);
     PP_CUDA(cudaGetLastError());
-    pp::k_dec_combine<<<grid_for(di->sm_count, 16, int64_t(n_resp) * hq), pp::DEC_D, 0, s>>>(
-        gd, G, cu_d, nseg, hq, n_resp, workspace, p, static_cast<__nv_bfloat16 *>(o), lse);
+    pp::k_dec_combine<<<grid_for(di->sm_count, 3, (int64_t(n_resp) * hq + pp::DEC_COMB_WARPS - 1) / pp::DEC_COMB_WARPS),
+                        pp::DEC_COMB_WARPS * 32, 0, s>>>(hq, n_resp, workspace, p, static_cast<__nv_bfloat16 *>(o), lse);
     PP_CUDA(cudaGetLastError());
     return PP_OK;
 }

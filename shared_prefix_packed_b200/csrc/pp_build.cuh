@@ -21,28 +21,68 @@ __device__ int32_t g_dev_err;  // this device's error word, read and cleared by 
 
 __device__ __forceinline__ void set_dev_err(int32_t bits) { atomicOr(&g_dev_err, bits); }
 
-// Block-wide exclusive scan of `n` int32 values in place (one block, any n), returns the total.
-template <int NT>
-__device__ int32_t block_exclusive_scan(int32_t *a, int n, int32_t *s_tmp) {
-    int32_t carry = 0;
+// Block-wide exclusive scans of K int32 arrays of length n, in place (one block of NT threads, NT a multiple of 32
+// and at most 1024, any n): warp-shuffle scans, then one scan of the warp totals, two block barriers per NT
+// elements. tot[k] receives array k's total. s_tmp holds at least 32 * K ints; every thread of the block calls it.
+template <int NT, int K>
+__device__ void block_exclusive_scan_multi(int32_t *const (&a)[K], int n, int32_t *s_tmp, int32_t (&tot)[K]) {
+    static_assert(NT % 32 == 0 && NT <= 1024, "block size");
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int32_t carry[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) carry[k] = 0;
     for (int base = 0; base < n; base += NT) {
         const int i = base + threadIdx.x;
-        const int32_t v = i < n ? a[i] : 0;
-        s_tmp[threadIdx.x] = v;
-        __syncthreads();
-        for (int off = 1; off < NT; off <<= 1) {
-            const int32_t t = threadIdx.x >= off ? s_tmp[threadIdx.x - off] : 0;
-            __syncthreads();
-            s_tmp[threadIdx.x] += t;
-            __syncthreads();
+        int32_t v[K], x[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            v[k] = i < n ? a[k][i] : 0;
+            x[k] = v[k];
         }
-        const int32_t incl = s_tmp[threadIdx.x];
-        if (i < n) a[i] = carry + incl - v;
-        const int32_t tot = s_tmp[NT - 1];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1)
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+                const int32_t t = __shfl_up_sync(0xffffffffu, x[k], off);
+                if (lane >= off) x[k] += t;
+            }
+        if (lane == 31)
+#pragma unroll
+            for (int k = 0; k < K; ++k) s_tmp[k * 32 + wid] = x[k];
         __syncthreads();
-        carry += tot;
+        if (wid == 0) {
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+                int32_t y = lane < NW ? s_tmp[k * 32 + lane] : 0;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int32_t t = __shfl_up_sync(0xffffffffu, y, off);
+                    if (lane >= off) y += t;
+                }
+                if (lane < NW) s_tmp[k * 32 + lane] = y;           // inclusive scan of the warp totals
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            const int32_t before = wid > 0 ? s_tmp[k * 32 + wid - 1] : 0;
+            if (i < n) a[k][i] = carry[k] + before + x[k] - v[k];
+            carry[k] += s_tmp[k * 32 + NW - 1];
+        }
+        __syncthreads();                                           // s_tmp is rewritten by the next round
     }
-    return carry;
+#pragma unroll
+    for (int k = 0; k < K; ++k) tot[k] = carry[k];
+}
+
+// One array: block_exclusive_scan_multi with K = 1; returns the total.
+template <int NT>
+__device__ int32_t block_exclusive_scan(int32_t *a, int n, int32_t *s_tmp) {
+    int32_t *const arr[1] = {a};
+    int32_t tot[1];
+    block_exclusive_scan_multi<NT, 1>(arr, n, s_tmp, tot);
+    return tot[0];
 }
 
 __device__ __forceinline__ int upper_bound_i32(const int32_t *a, int n, int32_t key) {
@@ -208,10 +248,12 @@ __global__ void k_meta_tiles(void *meta, const int32_t *__restrict__ qoff, const
 // Stage 4 (one block): cost-ordered forward tiles and backward work chunks (counting sort, longest first).
 template <int NT>
 __global__ void __launch_bounds__(NT) k_meta_sort(void *meta, int32_t *chunk_off, BWork *bw_tmp) {
-    __shared__ int32_t s_tmp[NT];
+    __shared__ int32_t s_tmp[32];
     __shared__ int32_t s_hist[SORT_BINS];
+    __shared__ int32_t s_nsplit;
     MetaHeader *h = meta_ptr<MetaHeader>(meta, 0);
     if (h->dev_err) return;
+    if (threadIdx.x == 0) s_nsplit = 0;
     const int nq = h->n_qt, nk = h->n_kt;
     const QTile *qt = meta_ptr<QTile>(meta, h->off_qt);
     const KTile *kt = meta_ptr<KTile>(meta, h->off_kt);
@@ -259,16 +301,13 @@ __global__ void __launch_bounds__(NT) k_meta_sort(void *meta, int32_t *chunk_off
             bw_tmp[chunk_off[i] + c] = w;
         }
     }
-    s_tmp[threadIdx.x] = nsplit_local;
-    __syncthreads();
+    if (nsplit_local) atomicAdd(&s_nsplit, nsplit_local);
     for (int b = threadIdx.x; b < SORT_BINS; b += NT) s_hist[b] = 0;
+    __syncthreads();
     if (threadIdx.x == 0) {
-        int ns = 0;
-        for (int i = 0; i < NT; ++i) ns += s_tmp[i];
-        h->n_split = ns;
+        h->n_split = s_nsplit;
         h->n_bw = nbw;
     }
-    __syncthreads();
     for (int i = threadIdx.x; i < nbw; i += NT) atomicAdd(&s_hist[min(bw_tmp[i].qb - bw_tmp[i].qa, SORT_BINS - 1)], 1);
     __syncthreads();
     for (int b = threadIdx.x; b < SORT_BINS; b += NT) chunk_off[SORT_BINS - 1 - b] = s_hist[b];

@@ -14,7 +14,7 @@
 //                chunk is therefore read from
 //                HBM once per group (per query block), not once per response. Each job writes an fp32 record
 //                (max, sum, un-normalised O) per valid query row.
-//   k_dec_combine per (response, q head): merges its records (the group's prefix chunks, its own chunks).
+//   k_dec_combine one warp per (response, q head): merges its records (the group's prefix chunks, its own chunks).
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -39,6 +39,7 @@ struct DecPlan {
     int64_t off_job_off;     // [nseg + 1] jobs (chunk, query block) before each segment
     int64_t off_counts;      // [4]: units, records, ok (1 if the plan fits), jobs
     int64_t off_jobs;        // DecJobRec[max_pairs]: every job decoded once (jobs <= records)
+    int64_t off_resp;        // DecRespRec[nseg - G]: where each response's records lie
     int64_t off_part;        // fp32 records: [pairs][hq][DEC_REC]
     int64_t total;
     int64_t max_pairs;       // records the workspace holds
@@ -59,6 +60,7 @@ __host__ inline DecPlan dec_plan_layout(int64_t T, int32_t G, int32_t nseg, int3
     p.off_job_off = o;   o = dec_a256(o + 4 * int64_t(nseg + 1));
     p.off_counts = o;    o = dec_a256(o + 16);
     p.off_jobs = o;      o = dec_a256(o + 32 * max_pairs);
+    p.off_resp = o;      o = dec_a256(o + 32 * int64_t(nseg - G));
     p.off_part = o;      o = dec_a256(o + 4 * max_pairs * hq * DEC_REC);
     p.total = o;
     p.max_pairs = max_pairs;
@@ -82,11 +84,19 @@ struct alignas(16) DecJobRec {
     int32_t pad[3];
 };
 
+// Where one response's records lie: its prefix chunks' records are pp0 + j * stride (j < nch_p), its own chunks'
+// records po + j (j < nch_o).
+struct alignas(16) DecRespRec {
+    int32_t pp0, stride, nch_p, po, nch_o;
+    int32_t pad[3];
+};
+
 // groups: pp_group_desc pairs {prefix_len, num_suffixes}; cu: int32[nseg + 1]. rb = responses per query block.
 __global__ void __launch_bounds__(1024) k_dec_plan(const int32_t *__restrict__ groups, int32_t G,
                                                    const int32_t *__restrict__ cu, int32_t nseg, int64_t T, int rb,
                                                    void *ws, DecPlan p) {
-    __shared__ int32_t s_tmp[1024];
+    constexpr int NT = 1024;
+    __shared__ int32_t s_tmp[3 * 32];
     __shared__ int32_t s_bad;
     int32_t *first_seg = dec_ptr<int32_t>(ws, p.off_first_seg);
     int32_t *seg_group = dec_ptr<int32_t>(ws, p.off_seg_group);
@@ -96,17 +106,16 @@ __global__ void __launch_bounds__(1024) k_dec_plan(const int32_t *__restrict__ g
     int32_t *counts = dec_ptr<int32_t>(ws, p.off_counts);
     if (threadIdx.x == 0) s_bad = (cu[0] != 0 || int64_t(cu[nseg]) != T) ? 1 : 0;
     __syncthreads();
-    for (int s = threadIdx.x; s < nseg; s += blockDim.x)
+    for (int s = threadIdx.x; s < nseg; s += NT)
         if (cu[s + 1] < cu[s]) s_bad = 1;                      // segment bounds must stay inside [0, T]
-    for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    for (int g = threadIdx.x; g < G; g += NT) {
         const int32_t kg = groups[2 * g + 1];
         if (kg < 0) s_bad = 1;
         first_seg[g] = 1 + (kg < 0 ? 0 : kg);
     }
     if (threadIdx.x == 0) first_seg[G] = 0;
     __syncthreads();
-    const int32_t tot_seg = block_exclusive_scan<1024>(first_seg, G + 1, s_tmp);
-    __syncthreads();
+    const int32_t tot_seg = block_exclusive_scan<NT>(first_seg, G + 1, s_tmp);
     if (tot_seg != nseg || s_bad) {                            // descriptors disagree with the segments
         if (threadIdx.x == 0) {
             atomicOr(&g_dev_err, DEVERR_BAD_GROUPS);
@@ -117,9 +126,11 @@ __global__ void __launch_bounds__(1024) k_dec_plan(const int32_t *__restrict__ g
         }
         return;
     }
-    for (int s = threadIdx.x; s < nseg; s += blockDim.x) {
-        const int g = upper_bound_i32(first_seg, G + 1, s) - 1;   // first_seg[g] <= s < first_seg[g + 1]
-        seg_group[s] = g;
+    for (int g = threadIdx.x; g < G; g += NT)                  // each group labels its own run of segments
+        for (int s = first_seg[g]; s < first_seg[g + 1]; ++s) seg_group[s] = g;
+    __syncthreads();
+    for (int s = threadIdx.x; s < nseg; s += NT) {
+        const int g = seg_group[s];
         const int32_t len = cu[s + 1] - cu[s];
         const int32_t nch = len > 0 ? (len + DEC_CH - 1) / DEC_CH : 0;
         const int32_t q_per = (s == first_seg[g]) ? groups[2 * g + 1] : 1;
@@ -133,35 +144,49 @@ __global__ void __launch_bounds__(1024) k_dec_plan(const int32_t *__restrict__ g
         job_off[nseg] = 0;
     }
     __syncthreads();
-    const int32_t U = block_exclusive_scan<1024>(unit_off, nseg + 1, s_tmp);
-    __syncthreads();
-    const int32_t NP = block_exclusive_scan<1024>(pair_off, nseg + 1, s_tmp);
-    __syncthreads();
-    const int32_t NJ = block_exclusive_scan<1024>(job_off, nseg + 1, s_tmp);
-    if (int64_t(NP) <= p.max_pairs) {                          // the job table (NJ <= NP entries) fits too
+    int32_t *const arrs[3] = {unit_off, pair_off, job_off};
+    int32_t tots[3];
+    block_exclusive_scan_multi<NT, 3>(arrs, nseg + 1, s_tmp, tots);
+    const int32_t U = tots[0], NP = tots[1], NJ = tots[2];
+    const bool fits = int64_t(NP) <= p.max_pairs;              // the job table (NJ <= NP entries) fits too
+    if (fits) {
         DecJobRec *jobs = dec_ptr<DecJobRec>(ws, p.off_jobs);
-        for (int s = threadIdx.x; s < nseg; s += blockDim.x) {
+        DecRespRec *resp_tab = dec_ptr<DecRespRec>(ws, p.off_resp);
+        for (int s = threadIdx.x; s < nseg; s += NT) {
             const int g = seg_group[s];
-            const bool prefix = s == first_seg[g];
-            const int cnt = prefix ? groups[2 * g + 1] : 1;    // queries that see the segment
+            const int sp = first_seg[g];
+            const bool prefix = s == sp;
+            const int kg = groups[2 * g + 1];
+            const int cnt = prefix ? kg : 1;                   // queries that see the segment
             const int nch = unit_off[s + 1] - unit_off[s];
-            const int resp0 = prefix ? first_seg[g] - g : s - g - 1;   // response ordinal = segment - group - 1
+            const int resp0 = prefix ? sp - g : s - g - 1;     // response ordinal = segment - group - 1
             const int nw = job_off[s + 1] - job_off[s];
+            const int y_s = cu[s], y_e = cu[s + 1], pb = pair_off[s], jb = job_off[s];
             for (int w = 0; w < nw; ++w) {                     // (query block, chunk), chunks fastest: one Q load
                 const int qb = w / nch, j = w % nch;           // serves all chunks of the segment
                 DecJobRec r;
-                r.y0 = cu[s] + j * DEC_CH;
-                r.yend = cu[s + 1];
+                r.y0 = y_s + j * DEC_CH;
+                r.yend = y_e;
                 r.r0 = resp0 + qb * rb;
                 r.nq = min(rb, cnt - qb * rb);
-                r.pbase = pair_off[s] + j * cnt + qb * rb;
+                r.pbase = pb + j * cnt + qb * rb;
                 r.pad[0] = r.pad[1] = r.pad[2] = 0;
-                jobs[job_off[s] + w] = r;
+                jobs[jb + w] = r;
+            }
+            if (!prefix) {
+                const int i = s - sp - 1;                      // response index within the group
+                DecRespRec rr;
+                rr.pp0 = pair_off[sp] + i;
+                rr.stride = kg;
+                rr.nch_p = unit_off[sp + 1] - unit_off[sp];
+                rr.po = pb;
+                rr.nch_o = nch;
+                rr.pad[0] = rr.pad[1] = rr.pad[2] = 0;
+                resp_tab[resp0] = rr;
             }
         }
     }
     if (threadIdx.x == 0) {
-        const bool fits = int64_t(NP) <= p.max_pairs;
         if (!fits) atomicOr(&g_dev_err, DEVERR_BAD_GROUPS);   // descriptors differ from the sized ones
         counts[0] = fits ? U : 0;
         counts[1] = NP;
@@ -429,53 +454,77 @@ done:
 }
 
 // o: [n_resp, hq, D] bf16; lse: [hq, n_resp] fp32 (natural log).
-__global__ void __launch_bounds__(DEC_D) k_dec_combine(const int32_t *__restrict__ groups, int32_t G,
-                                                       const int32_t *__restrict__ cu, int32_t nseg, int hq,
-                                                       int32_t n_resp, const void *ws, DecPlan p,
-                                                       __nv_bfloat16 *__restrict__ o, float *__restrict__ lse) {
-    const int32_t *first_seg = dec_ptr<int32_t>(ws, p.off_first_seg);
-    const int32_t *unit_off = dec_ptr<int32_t>(ws, p.off_unit_off);
-    const int32_t *pair_off = dec_ptr<int32_t>(ws, p.off_pair_off);
+constexpr int DEC_COMB_WARPS = 8;
+
+// One warp per (response, q head); a lane owns four of the d outputs. The records' maxima are read first (one lane
+// per record) to get the common max M; then the records are summed with weights 2^(m - M), eight records' loads in
+// flight per lane.
+__global__ void __launch_bounds__(DEC_COMB_WARPS * 32, 3) k_dec_combine(int hq, int32_t n_resp, const void *ws,
+                                                                     DecPlan p, __nv_bfloat16 *__restrict__ o,
+                                                                     float *__restrict__ lse) {
+    constexpr int UNROLL = 8;
+    const DecRespRec *resp_tab = dec_ptr<DecRespRec>(ws, p.off_resp);
     const float *part = dec_ptr<float>(ws, p.off_part);
     const int32_t ok = dec_ptr<int32_t>(ws, p.off_counts)[2];
-    const int dd = threadIdx.x;
-    for (int64_t w = blockIdx.x; w < int64_t(n_resp) * hq; w += gridDim.x) {
+    const int lane = threadIdx.x & 31;
+    const int64_t n_units = int64_t(n_resp) * hq, stride = int64_t(gridDim.x) * DEC_COMB_WARPS;
+    for (int64_t w = int64_t(blockIdx.x) * DEC_COMB_WARPS + (threadIdx.x >> 5); w < n_units; w += stride) {
         const int resp = int(w / hq), hh = int(w % hq);
+        __nv_bfloat162 *orow = reinterpret_cast<__nv_bfloat162 *>(o + (int64_t(resp) * hq + hh) * DEC_D + 4 * lane);
+        float *lrow = lse + int64_t(hh) * n_resp + resp;
         if (!ok) {                                             // the plan did not fit: no records were written
-            o[(int64_t(resp) * hq + hh) * DEC_D + dd] = __float2bfloat16_rn(__int_as_float(0x7fc00000));
-            if (dd == 0) lse[int64_t(hh) * n_resp + resp] = __int_as_float(0x7fc00000);
+            const float nan = __int_as_float(0x7fc00000);
+            orow[0] = __floats2bfloat162_rn(nan, nan);
+            orow[1] = __floats2bfloat162_rn(nan, nan);
+            if (lane == 0) *lrow = nan;
             continue;
         }
-        // group of the response: the last g with first_seg[g] - g <= resp (responses before group g)
-        int lo = 0, hi = G;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (first_seg[mid] - mid <= resp) lo = mid + 1; else hi = mid;
-        }
-        const int g = lo - 1;
-        const int sp = first_seg[g], k_g = groups[2 * g + 1];
-        const int i = resp - (first_seg[g] - g);               // response index within the group
-        const int so = sp + 1 + i;                              // its own segment
-        float M = -INFINITY, L = 0.f, acc = 0.f;
-        auto merge = [&](int64_t pair) {
-            const float *rec = part + (pair * hq + hh) * DEC_REC;
-            const float m = rec[0];
-            if (m == -INFINITY) return;
-            const float Mn = fmaxf(M, m);
-            const float a = exp2f(M - Mn), b = exp2f(m - Mn);
-            L = L * a + rec[1] * b;
-            acc = acc * a + rec[4 + dd] * b;
-            M = Mn;
+        const DecRespRec rr = resp_tab[resp];
+        const int n = rr.nch_p + rr.nch_o;
+        auto rec_of = [&](int j) -> const float * {
+            const int64_t pair = j < rr.nch_p ? int64_t(rr.pp0) + int64_t(j) * rr.stride : int64_t(rr.po) + (j - rr.nch_p);
+            return part + (pair * hq + hh) * DEC_REC;
         };
-        const int nch_p = unit_off[sp + 1] - unit_off[sp];
-        for (int j = 0; j < nch_p; ++j) merge(int64_t(pair_off[sp]) + int64_t(j) * k_g + i);
-        const int nch_o = unit_off[so + 1] - unit_off[so];
-        for (int j = 0; j < nch_o; ++j) merge(int64_t(pair_off[so]) + j);
+        float M = -INFINITY;
+        for (int j = lane; j < n; j += 32) M = fmaxf(M, rec_of(j)[0]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        float L = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        auto add = [&](float m, float l, float4 v) {
+            if (m == -INFINITY) return;                        // a chunk with no key visible to this row
+            const float wgt = exp2f(m - M);
+            L = fmaf(l, wgt, L);
+            acc.x = fmaf(v.x, wgt, acc.x);
+            acc.y = fmaf(v.y, wgt, acc.y);
+            acc.z = fmaf(v.z, wgt, acc.z);
+            acc.w = fmaf(v.w, wgt, acc.w);
+        };
+        if (M != -INFINITY) {
+            int j = 0;
+            for (; j + UNROLL <= n; j += UNROLL) {
+                float m[UNROLL], l[UNROLL];
+                float4 v[UNROLL];
+#pragma unroll
+                for (int u = 0; u < UNROLL; ++u) {
+                    const float *r = rec_of(j + u);
+                    m[u] = r[0];
+                    l[u] = r[1];
+                    v[u] = *reinterpret_cast<const float4 *>(r + 4 + 4 * lane);
+                }
+#pragma unroll
+                for (int u = 0; u < UNROLL; ++u) add(m[u], l[u], v[u]);
+            }
+            for (; j < n; ++j) {
+                const float *r = rec_of(j);
+                add(r[0], r[1], *reinterpret_cast<const float4 *>(r + 4 + 4 * lane));
+            }
+        }
         const bool any = L > 0.f;
-        o[(int64_t(resp) * hq + hh) * DEC_D + dd] = __float2bfloat16_rn(any ? acc / L : 0.f);
-        if (dd == 0) lse[int64_t(hh) * n_resp + resp] = any ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
-        (void)cu;
-        (void)nseg;
+        const float inv = any ? 1.f / L : 0.f;
+        orow[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        orow[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+        if (lane == 0) *lrow = any ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
     }
 }
 
