@@ -351,7 +351,7 @@ pp_status pp_decode_attn(const void *q, const void *k_cache, const void *v_cache
     PP_CUDA(cudaGetLastError());
     const int smem = int(sizeof(pp::DecSmem)) + 1024;
     PP_CUDA(cudaFuncSetAttribute(pp::k_dec_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    pp::k_dec_chunk<<<di->sm_count, pp::DEC_THREADS, smem, s>>>(mq, mk, mv, gd, cu_d, nseg, hq, hkv, rb, n_resp,
+    pp::k_dec_chunk<<<di->sm_count, pp::DEC_THREADS, smem, s>>>(mq, mk, mv, hq, hkv, rb, n_resp,
                                                                   scale * 1.4426950408889634f, workspace, p);
     PP_CUDA(cudaGetLastError());
     pp::k_dec_combine<<<grid_for(di->sm_count, 3, (int64_t(n_resp) * hq + pp::DEC_COMB_WARPS - 1) / pp::DEC_COMB_WARPS),

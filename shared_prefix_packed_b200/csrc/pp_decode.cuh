@@ -234,16 +234,12 @@ __device__ __forceinline__ DecJob dec_job(const void *ws, const DecPlan &p, int 
 // tmQ: 3-D map over q (d, hq, n_resp) with box (64, r, rb); tmK/tmV: 3-D maps over the cache, box (64, 1, 128).
 __global__ void __launch_bounds__(DEC_THREADS, 1)
 k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-            const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ groups, const int32_t *__restrict__ cu,
-            int32_t nseg, int hq, int hkv, int rb, int32_t n_resp, float sl2, void *ws, DecPlan p) {
+            const __grid_constant__ CUtensorMap tmV, int hq, int hkv, int rb, int32_t n_resp, float sl2, void *ws,
+            DecPlan p) {
     extern __shared__ uint8_t smem_raw[];
     DecSmem &sm = *reinterpret_cast<DecSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = hq / hkv;
-    const int32_t J = dec_ptr<int32_t>(ws, p.off_counts)[3];
-    const int64_t n_jobs = int64_t(J) * hkv;
-    // contiguous job range per CTA: consecutive jobs share a query block (one Q load per segment and kv head)
-    const int64_t j_begin = n_jobs * blockIdx.x / gridDim.x, j_end = n_jobs * (blockIdx.x + 1) / gridDim.x;
     volatile int *abort_flag = &sm.abort_flag;
     float *part = dec_ptr<float>(ws, p.off_part);
 
@@ -277,6 +273,10 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    const int32_t J = dec_ptr<int32_t>(ws, p.off_counts)[3];
+    const int64_t n_jobs = int64_t(J) * hkv;
+    // contiguous job range per CTA: consecutive jobs share a query block (one Q load per segment and kv head)
+    const int64_t j_begin = n_jobs * blockIdx.x / gridDim.x, j_end = n_jobs * (blockIdx.x + 1) / gridDim.x;
     const uint32_t tmem = sm.tmem_base;
     // TMEM: S_b [128 b, 128 b + 128), O_b [256 + 128 b, ...); P_b (bf16) over the first 64 columns of S_b
     auto same_q = [&](const DecJob &a, const DecJob &b) { return a.kh == b.kh && a.r0 == b.r0; };
@@ -380,9 +380,10 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             const int nk = min(DEC_CH, d.yend - d.y0);             // keys of the chunk inside the segment
             if (!bwait(&sm.s_full[b], (u >> 1) & 1, abort_flag)) goto done;
             tc_fence_after();
-            float m = -INFINITY, l = 0.f;
+            float m = -INFINITY, l = 0.f;                          // record: max of S * sl2 (base 2), sum of P
             const bool any = __any_sync(0xffffffffu, valid);
             if (any) {
+                // Rows that are not valid are not masked: their P and O are never read.
                 float s[DEC_CH];
                 {
                     uint32_t r0[32], r1[32], r2[32], r3[32];
@@ -399,20 +400,28 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                         s[96 + e] = __uint_as_float(r3[e]);
                     }
                 }
+                if (nk < DEC_CH) {                                 // the segment's last chunk: keys past its end
 #pragma unroll
-                for (int c = 0; c < DEC_CH; ++c) {
-                    s[c] = (valid && c < nk) ? s[c] * sl2 : -INFINITY;
-                    m = fmaxf(m, s[c]);
+                    for (int c = 0; c < DEC_CH; ++c)
+                        if (c >= nk) s[c] = -INFINITY;
                 }
-                const float mu = m == -INFINITY ? 0.f : m;
+                float mx = s[0];
+#pragma unroll
+                for (int c = 1; c + 1 < DEC_CH; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
+                mx = fmaxf(mx, s[DEC_CH - 1]);
+                // the scale is positive, so max(S) * sl2 is the max of the scaled row; P = 2^(S * sl2 - mu)
+                const float mu = mx == -INFINITY ? 0.f : mx * sl2;
+                m = mx == -INFINITY ? -INFINITY : mu;
 #pragma unroll
                 for (int c = 0; c < DEC_CH / 32; ++c) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2_approx(s[32 * c + 2 * e] - mu), p1 = ex2_approx(s[32 * c + 2 * e + 1] - mu);
-                        l += p0 + p1;
-                        pk[e] = pack_bf16x2(p0, p1);
+                        const float2 x = ffma2(make_float2(s[32 * c + 2 * e], s[32 * c + 2 * e + 1]),
+                                               make_float2(sl2, sl2), make_float2(-mu, -mu));
+                        const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                        l += pp.x + pp.y;
+                        pk[e] = pack_bf16x2(pp.x, pp.y);
                     }
                     tmem_st16(tmem + lane_off + 128 * b + 16 * c, pk);
                 }
