@@ -85,23 +85,26 @@ __global__ void k_bwd_pre(const __nv_bfloat16 *__restrict__ O, const __nv_bfloat
                           int hq, float inv_scale, const void *__restrict__ meta, float *__restrict__ dk_acc,
                           float *__restrict__ dv_acc, int hkv) {
     {
+        // zero the fp32 dK/dV rows of split key tiles (their chunks add into them). A unit is 16 rows of one key
+        // tile: the rows of a tile are contiguous ([rows][hkv][d]), so a unit is one contiguous run of float4.
         const MetaHeader hd = *meta_ptr<MetaHeader>(meta, 0);
         if (hd.dev_err == 0 && hd.n_split > 0) {
             const KTile *kts = meta_ptr<KTile>(meta, hd.off_kt);
-            const int64_t per_row = int64_t(hkv) * (BWD_D / 4);       // float4 per row
-            const int64_t per_tile = 128 * per_row;
-            const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+            const int per_row = hkv * (BWD_D / 4);                     // float4 per row
             const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < int64_t(hd.n_kt) * per_tile;
-                 e += stride) {
-                const KTile t = kts[e / per_tile];
+            for (int u = blockIdx.x; u < hd.n_kt * 8; u += gridDim.x) {
+                const KTile t = kts[u >> 3];
                 if (t.nch <= 1) continue;
-                const int64_t rem = e % per_tile;
-                const int64_t row = t.row0 + rem / per_row;
-                if (row >= t.gstart + t.glen) continue;
-                const int64_t off = row * hkv * BWD_D + (rem % per_row) * 4;
-                *reinterpret_cast<float4 *>(dk_acc + off) = z;
-                *reinterpret_cast<float4 *>(dv_acc + off) = z;
+                const int r0 = (u & 7) * 16;
+                const int rows = min(16, t.gstart + t.glen - t.row0 - r0);
+                if (rows <= 0) continue;
+                const int64_t base = (int64_t(t.row0) + r0) * per_row;
+                float4 *dk4 = reinterpret_cast<float4 *>(dk_acc) + base;
+                float4 *dv4 = reinterpret_cast<float4 *>(dv_acc) + base;
+                for (int e = threadIdx.x; e < rows * per_row; e += blockDim.x) {
+                    dk4[e] = z;
+                    dv4[e] = z;
+                }
             }
         }
     }
@@ -650,29 +653,32 @@ done:
 }
 
 // ------------------------------------------------------------------------------------------------- convert
-// dK/dV rows of split key tiles = bf16(fp32 accumulators).
+// dK/dV rows of split key tiles = bf16(fp32 accumulators). A unit is 16 rows of one key tile (contiguous rows).
 __global__ void k_bwd_convert(const void *__restrict__ meta, const float *__restrict__ dk_acc,
                               const float *__restrict__ dv_acc, __nv_bfloat16 *__restrict__ dK,
                               __nv_bfloat16 *__restrict__ dV, int hkv) {
     const MetaHeader hd = *meta_ptr<MetaHeader>(meta, 0);
     if (hd.dev_err || hd.n_split == 0) return;
-    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
     const KTile *kts = meta_ptr<KTile>(meta, hd.off_kt);
-    const int64_t per_tile = int64_t(128) * hkv * (BWD_D / 4);
-    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < int64_t(hd.n_kt) * per_tile; e += stride) {
-        const KTile t = kts[e / per_tile];
+    const int per_row = hkv * (BWD_D / 4);                             // float4 (four elements) per row
+    for (int u = blockIdx.x; u < hd.n_kt * 8; u += gridDim.x) {
+        const KTile t = kts[u >> 3];
         if (t.nch <= 1) continue;
-        const int64_t rem = e % per_tile;
-        const int64_t row = t.row0 + rem / (hkv * (BWD_D / 4));
-        if (row >= t.gstart + t.glen) continue;
-        const int64_t off = row * hkv * BWD_D + (rem % (hkv * (BWD_D / 4))) * 4;
+        const int r0 = (u & 7) * 16;
+        const int rows = min(16, t.gstart + t.glen - t.row0 - r0);
+        if (rows <= 0) continue;
+        const int64_t base = (int64_t(t.row0) + r0) * per_row;
         for (int which = 0; which < 2; ++which) {
-            const float4 a = *reinterpret_cast<const float4 *>((which ? dv_acc : dk_acc) + off);
-            __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
-            uint2 u;
-            u.x = *reinterpret_cast<uint32_t *>(&lo);
-            u.y = *reinterpret_cast<uint32_t *>(&hi);
-            *reinterpret_cast<uint2 *>((which ? dV : dK) + off) = u;
+            const float4 *src = reinterpret_cast<const float4 *>(which ? dv_acc : dk_acc) + base;
+            uint2 *dst = reinterpret_cast<uint2 *>(which ? dV : dK) + base;
+            for (int e = threadIdx.x; e < rows * per_row; e += blockDim.x) {
+                const float4 a = src[e];
+                __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+                uint2 v;
+                v.x = *reinterpret_cast<uint32_t *>(&lo);
+                v.y = *reinterpret_cast<uint32_t *>(&hi);
+                dst[e] = v;
+            }
         }
     }
 }
