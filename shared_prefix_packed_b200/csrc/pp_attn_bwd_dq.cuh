@@ -127,6 +127,13 @@ k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
                 const DqItem w = dq_decode(meta, hd, item, hq, hkv);
                 const int n = qtile_nkv(w.t);
+                if (item + int(gridDim.x) < n_items) {                 // the next item's Q and dO into L2
+                    const DqItem wn = dq_decode(meta, hd, item + gridDim.x, hq, hkv);
+                    for (int c = 0; c < 2; ++c) {
+                        tma_prefetch_3d(&tmQ, c * 64, wn.h, wn.t.row0);
+                        tma_prefetch_3d(&tmdO, c * 64, wn.h, wn.t.row0);
+                    }
+                }
                 if (!bwait(&sm.q_empty, (it_n & 1) ^ 1, abort_flag)) goto done;
                 mbar_arrive_expect_tx(&sm.q_full, DqSmem::TILE);
                 for (int c = 0; c < 2; ++c)

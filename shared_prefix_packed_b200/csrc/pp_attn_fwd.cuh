@@ -171,6 +171,11 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
             const FwdItem w = fwd_decode(meta, hd, item, hq, hkv);
             const int n = qtile_nkv(w.t);
+            if (item + int(gridDim.x) < n_items) {                     // the next item's Q into L2 (read once, so
+                const FwdItem wn = fwd_decode(meta, hd, item + gridDim.x, hq, hkv);   // a miss otherwise)
+                for (int hs = 0; hs < wn.nh; ++hs)
+                    for (int c = 0; c < D / 64; ++c) tma_prefetch_3d(&tmQ, c * 64, wn.h0 + hs, wn.t.row0);
+            }
             if (!bwait(&sm.q_empty, (n_it & 1) ^ 1, abort_flag)) goto done;
             ++n_it;
             mbar_arrive_expect_tx(&sm.q_full, w.nh * FwdSmem<D>::TILE_BYTES);
