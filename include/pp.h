@@ -136,6 +136,17 @@ PP_API pp_status pp_rope(void *q, void *k, const int32_t *pos_ids_d, int64_t T, 
 PP_API pp_status pp_workspace_bytes(int32_t which, int64_t T, int32_t hq, int32_t hkv, int32_t d, int64_t *bytes);
 
 /* ---------------------------------------------------------------------------------------------------------------
+ * pp_bwd_ds_bytes (host only): extra backward workspace, beyond pp_workspace_bytes(PP_PASS_BWD, ...), that lets
+ * pp_attn_bwd keep one dS tile (128 keys x 128 queries, bf16, 32 KiB) per backward step and form dq from them
+ * instead of recomputing the scores. A step is (key tile of 128 rows, query tile of 128 rows that attends it, q
+ * head), for every kv head; the count follows the mask (same descriptors as pp_build_meta). groups_host,
+ * cu_host: host copies of the descriptors and segment bounds; *bytes (host) receives 1024 + steps * 32768.
+ * Returns PP_ERR_INVALID_ARG for descriptors that disagree with the segments.
+ */
+PP_API pp_status pp_bwd_ds_bytes(const pp_group_desc *groups_host, int32_t G, const int32_t *cu_host,
+                                 int32_t nseg, int32_t hq, int32_t hkv, int64_t *bytes);
+
+/* ---------------------------------------------------------------------------------------------------------------
  * pp_attn_fwd: O and the per-row log-sum-exp of exact packed attention.
  *   s_ij = softmax_scale * q_i . k_j over the allowed keys j of row i (q head h reads kv head h / (hq/hkv));
  *   lse_i = ln sum_j exp(s_ij) (natural log of the scaled scores); o_i = sum_j exp(s_ij - lse_i) v_j.
@@ -158,9 +169,11 @@ PP_API pp_status pp_attn_fwd(const void *q, const void *k, const void *v, const 
  *   workspace: ws_bytes >= pp_workspace_bytes(PP_PASS_BWD, ...), 256-byte aligned, contents need not be
  *   initialised. It holds (-lse/scale, -D) per row and q head, and fp32 dK/dV for the prefix key tiles, which are
  *   attended by every response of their group and so are split into chunks whose partials are added there (fp32
- *   reduction adds, one per element and chunk) before conversion to bf16. dq needs no scratch: each row tile of
- *   dq is produced by exactly one CTA, which recomputes the tile's scores and dP instead of exchanging partials.
- *   The result is deterministic except for the order of those dK/dV adds.
+ *   reduction adds, one per element and chunk) before conversion to bf16. Each row tile of dq is produced by exactly
+ *   one CTA (no reduction). If ws_bytes also covers pp_bwd_ds_bytes(...) for the batch, the dK/dV kernel keeps
+ *   every step's dS tile after the base workspace and dq is formed from them (the fast path); otherwise the dq
+ *   kernel recomputes the tile's scores and dP. The choice is made on the device from the batch's step count, so
+ *   either size is valid. The result is deterministic except for the order of the dK/dV adds.
  */
 PP_API pp_status pp_attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
                       const void *dout, const void *meta_d, int64_t T, int32_t hq, int32_t hkv, int32_t d,

@@ -8,7 +8,7 @@ binding (``_lib``) plus :class:`PackedBatch`, which allocates the buffers with t
 """
 from ._lib import (  # noqa: F401
     PP_BF16, PP_FP32, PP_PASS_BWD, PP_PASS_FWD, PPError,
-    pp_attn_bwd, pp_attn_fwd, pp_build_meta, pp_decode_attn, pp_decode_workspace_bytes, pp_get_status,
+    pp_attn_bwd, pp_attn_fwd, pp_build_meta, pp_bwd_ds_bytes, pp_decode_attn, pp_decode_workspace_bytes, pp_get_status,
     pp_meta_bounds, pp_meta_schedule, pp_meta_tiles, pp_pack_batch, pp_plan_batches,
     pp_response_logprobs,
     pp_rope,

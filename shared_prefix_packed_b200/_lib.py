@@ -45,6 +45,7 @@ SIGNATURES = {
                                    _VP]),
     "pp_plan_batches": (_I32, [_VP, _I32, _I64, _I32, _VP, _VP, _VP]),
     "pp_decode_workspace_bytes": (_I32, [_VP, _I32, _VP, _I32, _I32, _I64P]),
+    "pp_bwd_ds_bytes": (_I32, [_VP, _I32, _VP, _I32, _I32, _I32, _I64P]),
     "pp_decode_attn": (_I32, [_VP, _VP, _VP, _VP, _I32, _VP, _I32, _I64, _I32, _I32, _I32, _F32, _VP, _VP, _VP, _I64,
                               _VP]),
     "pp_pack_batch": (_I32, [_VP, _VP, _I32, _VP, _VP, _I32, _VP, _I32, _VP, _I64, _VP, _VP, _VP, _VP, _VP]),
@@ -186,6 +187,17 @@ def pp_decode_workspace_bytes(groups_host, cu_host, hq: int) -> int:
     c = cu_host.contiguous()
     _call("pp_decode_workspace_bytes", ctypes.c_void_p(g.data_ptr()), g.shape[0], ctypes.c_void_p(c.data_ptr()),
           c.numel() - 1, hq, ctypes.byref(out))
+    return out.value
+
+
+def pp_bwd_ds_bytes(groups_host, cu_host, hq: int, hkv: int) -> int:
+    """Extra backward workspace for the kept-dS path. groups_host: int32 [G, 2] CPU tensor; cu_host: int32 [nseg + 1]
+    CPU tensor."""
+    out = ctypes.c_int64(0)
+    g = groups_host.contiguous()
+    c = cu_host.contiguous()
+    _call("pp_bwd_ds_bytes", ctypes.c_void_p(g.data_ptr()), g.shape[0], ctypes.c_void_p(c.data_ptr()), c.numel() - 1,
+          hq, hkv, ctypes.byref(out))
     return out.value
 
 

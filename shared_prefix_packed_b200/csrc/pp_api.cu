@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -282,6 +283,41 @@ pp_status pp_workspace_bytes(int32_t which, int64_t T, int32_t hq, int32_t hkv, 
     return PP_OK;
 }
 
+pp_status pp_bwd_ds_bytes(const pp_group_desc *groups_host, int32_t G, const int32_t *cu_host, int32_t nseg,
+                          int32_t hq, int32_t hkv, int64_t *bytes) {
+    if (!groups_host || !cu_host || !bytes) return fail(PP_ERR_INVALID_ARG, "NULL pointer argument");
+    if (G < 0 || nseg < 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0)
+        return fail(PP_ERR_INVALID_ARG, "need G, num_segments >= 0 and hq a multiple of hkv");
+    const int64_t r = hq / hkv;
+    // one step per (key tile, attending query tile, q head): key tile b of a group of length L, prefix P, covers
+    // keys [128 b, 128 b + 128); its queries run from its own first row to e = L for a prefix tile, else to the end
+    // of the segment of its last key (the same rule as the schedule builder's)
+    int64_t steps = 0;
+    int32_t s = 0;
+    for (int32_t g = 0; g < G; ++g) {
+        const int32_t P = groups_host[g].prefix_len, k = groups_host[g].num_suffixes;
+        if (k < 0 || P < 0 || s + 1 + int64_t(k) > nseg) return fail(PP_ERR_INVALID_ARG, "descriptors exceed num_segments");
+        const int32_t start = cu_host[s], end = cu_host[s + 1 + k];
+        const int32_t L = end - start;
+        if (cu_host[s + 1] - start != P || L < P) return fail(PP_ERR_INVALID_ARG, "prefix length disagrees with segments");
+        int32_t seg = s + 1;                                        // segment of the current key (responses)
+        for (int32_t y0 = 0; y0 < L; y0 += pp::BWD_BN) {
+            const int32_t ylast = std::min(y0 + pp::BWD_BN, L) - 1;
+            int32_t e = L;
+            if (y0 >= P) {
+                while (seg < s + 1 + k && cu_host[seg + 1] - start <= ylast) ++seg;
+                e = cu_host[seg + 1] - start;
+            }
+            const int64_t qa = y0 / pp::BWD_BM, qb = (e + pp::BWD_BM - 1) / pp::BWD_BM;
+            steps += (qb - qa) * r * hkv;                          // every q head of every kv head
+        }
+        s += 1 + k;
+    }
+    if (s != nseg) return fail(PP_ERR_INVALID_ARG, "num_segments must equal sum_g (1 + k_g)");
+    *bytes = pp::BWD_DS_ALIGN + steps * pp::BWD_DS_TILE_BYTES;
+    return PP_OK;
+}
+
 // Exact (chunk, query) pair count of the decode plan, from host copies of the descriptors and segment bounds.
 static pp_status decode_pairs(const pp_group_desc *groups, int32_t G, const int32_t *cu, int32_t nseg, int64_t *pairs) {
     int64_t np = 0;
@@ -502,8 +538,8 @@ pp_status pp_attn_bwd(const void *q, const void *k, const void *v, const void *o
     const float scale = softmax_scale == 0.f ? 1.f / std::sqrt(float(d)) : softmax_scale;
     DeviceInfo *di;
     if ((st = device_info(&di)) != PP_OK) return st;
-    return pp::launch_bwd(q, k, v, o, lse, dout, meta_d, T, hq, hkv, d, scale, dq, dk, dv, workspace, di->sm_count,
-                          as_stream(stream), make_map_3d, fail);
+    return pp::launch_bwd(q, k, v, o, lse, dout, meta_d, T, hq, hkv, d, scale, dq, dk, dv, workspace, ws_bytes,
+                          di->sm_count, as_stream(stream), make_map_3d, make_map_3d_box, fail);
 }
 
 pp_status pp_attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const float *lse,

@@ -180,6 +180,7 @@ static_assert(sizeof(BwdSmem) + 1024 <= 232448, "dK/dV kernel shared memory exce
 struct BwdItem {
     KTile t;
     int qa, qb, split, kh;
+    int slot0;        // dS slot of the chunk's first step
 };
 
 // Work item -> (work chunk, kv head). Items run in groups of up to four kv heads; within a group, chunks in cost
@@ -204,6 +205,7 @@ __device__ __forceinline__ BwdItem bwd_decode(const void *meta, const MetaHeader
     it.qa = w.qa;
     it.qb = w.qb;
     it.split = w.split;
+    it.slot0 = w.slot0;
     return it;
 }
 
@@ -228,20 +230,16 @@ __device__ __forceinline__ void bwd_store_kv64(const uint32_t (&a)[32], const ui
         for (int e = 0; e < 8; ++e)
             red_add_v4(acc + 32 + 4 * e, __uint_as_float(b[4 * e]), __uint_as_float(b[4 * e + 1]),
                        __uint_as_float(b[4 * e + 2]), __uint_as_float(b[4 * e + 3]));
-    } else {
-        uint4 *o = reinterpret_cast<uint4 *>(dst);
+    } else {                                                   // 128 bytes: four 32-byte stores
+        auto pk = [](const uint32_t *x, int i) { return pack_bf16x2(__uint_as_float(x[i]), __uint_as_float(x[i + 1])); };
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            o[e] = make_uint4(pack_bf16x2(__uint_as_float(a[8 * e]), __uint_as_float(a[8 * e + 1])),
-                              pack_bf16x2(__uint_as_float(a[8 * e + 2]), __uint_as_float(a[8 * e + 3])),
-                              pack_bf16x2(__uint_as_float(a[8 * e + 4]), __uint_as_float(a[8 * e + 5])),
-                              pack_bf16x2(__uint_as_float(a[8 * e + 6]), __uint_as_float(a[8 * e + 7])));
+        for (int e = 0; e < 2; ++e)
+            st_global_v8(dst + 16 * e, pk(a, 16 * e), pk(a, 16 * e + 2), pk(a, 16 * e + 4), pk(a, 16 * e + 6),
+                         pk(a, 16 * e + 8), pk(a, 16 * e + 10), pk(a, 16 * e + 12), pk(a, 16 * e + 14));
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            o[4 + e] = make_uint4(pack_bf16x2(__uint_as_float(b[8 * e]), __uint_as_float(b[8 * e + 1])),
-                                  pack_bf16x2(__uint_as_float(b[8 * e + 2]), __uint_as_float(b[8 * e + 3])),
-                                  pack_bf16x2(__uint_as_float(b[8 * e + 4]), __uint_as_float(b[8 * e + 5])),
-                                  pack_bf16x2(__uint_as_float(b[8 * e + 6]), __uint_as_float(b[8 * e + 7])));
+        for (int e = 0; e < 2; ++e)
+            st_global_v8(dst + 32 + 16 * e, pk(b, 16 * e), pk(b, 16 * e + 2), pk(b, 16 * e + 4), pk(b, 16 * e + 6),
+                         pk(b, 16 * e + 8), pk(b, 16 * e + 10), pk(b, 16 * e + 12), pk(b, 16 * e + 14));
     }
 }
 
@@ -251,7 +249,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
          const void *__restrict__ meta, const float2 *__restrict__ ldg,
          float *__restrict__ dk_acc, float *__restrict__ dv_acc,
          __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV, int hq, int hkv, int64_t rows_pad,
-         float scale, float sl2) {
+         float scale, float sl2, __nv_bfloat16 *__restrict__ ds_buf, int64_t ds_cap) {
     extern __shared__ uint8_t smem_raw[];
     BwdSmem &sm = *reinterpret_cast<BwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -519,6 +517,8 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         const int jr = wl * 32 + lane;                                 // TMEM lane: key row
         const uint32_t lane_off = uint32_t(wl * 32) << 16;
         const int cb = 64 * wx;                                        // first query column of this half
+        // dS kept for the dQ kernel: slot s holds the step's dS^T tile, [128 key rows][128 query columns] bf16
+        const bool keep_ds = ds_buf != nullptr && int64_t(hd.n_slots) * hkv <= ds_cap;
         uint32_t g = 0, it_n = 0;
         const int32_t *key_end = meta_ptr<int32_t>(meta, hd.off_key_end);
         // Item epilogue, run inside the next item's first step (after its P, before its dS), when dK/dV of the
@@ -635,10 +635,18 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         }
                     }
                     tmem_st32(tmem + lane_off + COL_DP + cb + 32, ds);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&sm.ds_ready);
+                    if (keep_ds) {   // this key row's 64 query columns of dS, after dK(g) has been released
+                        const int64_t slot = int64_t(w.kh) * hd.n_slots + w.slot0 + t;   // slots: kv head major
+                        __nv_bfloat16 *dst = ds_buf + (slot * BWD_BN + jr) * BWD_BM + cb;   // 32-byte aligned
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            st_global_v8(dst + 16 * e, ds[8 * e], ds[8 * e + 1], ds[8 * e + 2], ds[8 * e + 3],
+                                         ds[8 * e + 4], ds[8 * e + 5], ds[8 * e + 6], ds[8 * e + 7]);
+                    }
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&sm.ds_ready);
             }
         }
         if (it_n > 0 && !epilogue(it_n - 1)) goto done;
@@ -687,10 +695,19 @@ __global__ void k_bwd_convert(const void *__restrict__ meta, const float *__rest
 typedef pp_status (*MakeMapFn)(CUtensorMap *, const void *, int64_t, int, int, int);
 typedef pp_status (*FailFn)(pp_status, const char *, ...);
 
+// Bytes of one kept dS tile (one backward step) and the alignment of the dS region after the base workspace.
+constexpr int64_t BWD_DS_TILE_BYTES = int64_t(BWD_BN) * BWD_BM * 2;
+constexpr int64_t BWD_DS_ALIGN = 1024;
+
+typedef pp_status (*MakeMapBoxFn)(CUtensorMap *, const void *, int64_t, int, int, int, int);
+
+// ws_bytes beyond the base layout holds kept dS tiles: if all the batch's steps fit, the key-side kernel writes them
+// and k_bwd_dq_ds forms dQ from them; otherwise k_bwd_dq recomputes S and dP. Both dQ kernels are launched and the
+// one whose case does not hold returns at once (the slot count is only known on the device).
 inline pp_status launch_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
                             const void *dout, const void *meta, int64_t T, int hq, int hkv, int d, float scale,
-                            void *dq, void *dk, void *dv, void *workspace, int sm_count, cudaStream_t s,
-                            MakeMapFn make_map, FailFn fail) {
+                            void *dq, void *dk, void *dv, void *workspace, int64_t ws_bytes, int sm_count,
+                            cudaStream_t s, MakeMapFn make_map, MakeMapBoxFn make_map_box, FailFn fail) {
     if (d != BWD_D) return fail(PP_ERR_UNSUPPORTED, "backward supports head dim 128 only (got %d)", d);
     const BwdWorkspace L = bwd_workspace_layout(T, hq, hkv, d);
     char *ws = static_cast<char *>(workspace);
@@ -700,12 +717,18 @@ inline pp_status launch_bwd(const void *q, const void *k, const void *v, const v
     const void *ptrs[8] = {q, k, v, o, dout, dq, dk, dv};
     for (const void *p : ptrs)
         if (reinterpret_cast<uintptr_t>(p) % 16) return fail(PP_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
-    CUtensorMap mq, mk, mv, mdo;
+    CUtensorMap mq, mk, mv, mdo, mds;
     pp_status st;
     if ((st = make_map(&mq, q, T, hq, d, BWD_BM)) != PP_OK) return st;
     if ((st = make_map(&mk, k, T, hkv, d, BWD_BN)) != PP_OK) return st;
     if ((st = make_map(&mv, v, T, hkv, d, BWD_BN)) != PP_OK) return st;
     if ((st = make_map(&mdo, dout, T, hq, d, BWD_BM)) != PP_OK) return st;
+    // the dS region: what the workspace holds past the base layout, in whole tiles
+    const int64_t ds_off = (L.total + BWD_DS_ALIGN - 1) / BWD_DS_ALIGN * BWD_DS_ALIGN;
+    int64_t ds_cap = ws_bytes > ds_off ? (ws_bytes - ds_off) / BWD_DS_TILE_BYTES : 0;
+    if (ds_cap > (int64_t(1) << 24)) ds_cap = int64_t(1) << 24;       // TMA row coordinate stays below 2^31
+    __nv_bfloat16 *ds_buf = ds_cap > 0 ? reinterpret_cast<__nv_bfloat16 *>(ws + ds_off) : nullptr;
+    if (ds_buf && (st = make_map_box(&mds, ds_buf, ds_cap * BWD_BN, 1, BWD_BM, 1, BWD_BN)) != PP_OK) return st;
     cudaError_t e;
     k_bwd_pre<<<sm_count * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(o),
                                            static_cast<const __nv_bfloat16 *>(dout), lse, ldg, T, L.rows_pad, hq,
@@ -716,14 +739,25 @@ inline pp_status launch_bwd(const void *q, const void *k, const void *v, const v
         return fail(PP_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     k_bwd_tc<<<sm_count, BWD_THREADS, smem, s>>>(mq, mk, mv, mdo, meta, ldg, dk_acc, dv_acc,
                                                  static_cast<__nv_bfloat16 *>(dk), static_cast<__nv_bfloat16 *>(dv),
-                                                 hq, hkv, L.rows_pad, scale, scale * 1.4426950408889634f);
+                                                 hq, hkv, L.rows_pad, scale, scale * 1.4426950408889634f, ds_buf,
+                                                 ds_cap);
     if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_tc: %s", cudaGetErrorString(e));
     const size_t smem_dq = sizeof(DqSmem) + 1024;
     if ((e = cudaFuncSetAttribute(k_bwd_dq, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_dq))) != cudaSuccess)
         return fail(PP_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     k_bwd_dq<<<sm_count, DQ_THREADS, smem_dq, s>>>(mq, mk, mv, mdo, meta, ldg, static_cast<__nv_bfloat16 *>(dq),
-                                                   hq, hkv, L.rows_pad, scale, scale * 1.4426950408889634f);
+                                                   hq, hkv, L.rows_pad, scale, scale * 1.4426950408889634f, ds_buf,
+                                                   ds_cap);
     if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_dq: %s", cudaGetErrorString(e));
+    if (ds_buf) {
+        const size_t smem_ds = sizeof(DqsSmem) + 1024;
+        if ((e = cudaFuncSetAttribute(k_bwd_dq_ds, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_ds))) !=
+            cudaSuccess)
+            return fail(PP_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        k_bwd_dq_ds<<<sm_count, DQS_THREADS, smem_ds, s>>>(mds, mk, meta, static_cast<__nv_bfloat16 *>(dq), hq, hkv,
+                                                            ds_buf, ds_cap);
+        if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_dq_ds: %s", cudaGetErrorString(e));
+    }
     k_bwd_convert<<<sm_count * 8, 256, 0, s>>>(meta, dk_acc, dv_acc, static_cast<__nv_bfloat16 *>(dk),
                                                static_cast<__nv_bfloat16 *>(dv), hkv);
     if ((e = cudaGetLastError()) != cudaSuccess) return fail(PP_ERR_CUDA, "k_bwd_convert: %s", cudaGetErrorString(e));

@@ -66,11 +66,12 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
 k_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
          const void *__restrict__ meta, const float2 *__restrict__ ldg, __nv_bfloat16 *__restrict__ dQ, int hq,
-         int hkv, int64_t rows_pad, float scale, float sl2) {
+         int hkv, int64_t rows_pad, float scale, float sl2, const void *ds_buf, int64_t ds_cap) {
     extern __shared__ uint8_t smem_raw[];
     DqSmem &sm = *reinterpret_cast<DqSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const MetaHeader hd = *meta_ptr<MetaHeader>(meta, 0);
+    if (ds_buf != nullptr && int64_t(hd.n_slots) * hkv <= ds_cap) return;   // dS kept: k_bwd_dq_ds computes dQ
     const int n_items = hd.n_qt * hq;
     volatile int *abort_flag = &sm.abort_flag;
 
@@ -393,6 +394,165 @@ done:
     if (warp == 17) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------------------------------------------------------
+// dQ from kept dS tiles. When the workspace holds a dS tile per backward step (the key-side kernel wrote each step's
+// dS^T, [128 key rows][128 query columns] bf16, with scale folded in), dQ needs no recomputation:
+//   dQ(query tile, q head) = sum over its key tiles of dS K      (M = 128 queries, N = d, K = 128 keys)
+// A work item is (query tile, q head) in the forward's cost order. Per key tile one dS tile and one K tile come in
+// through a 3-stage TMA ring; dS is the MMA's A operand read M-major (queries run along the tile's rows), K its B
+// operand read N-major. dQ accumulates in one of two TMEM buffers, so the epilogue of an item overlaps the next
+// item's MMAs. The kernel streams the dS tiles once: it is bound by their HBM read.
+constexpr int DQS_STAGES = 3;
+constexpr int DQS_THREADS = 192;     // warps 0-3 epilogue (TMEM lanes 0-127), warp 4 TMA, warp 5 TMEM + MMA issue
+
+struct DqsSmem {
+    static constexpr int TILE = 128 * 128 * 2;
+    static constexpr int CHUNK = 128 * 64 * 2;
+    alignas(1024) uint8_t ds[DQS_STAGES][TILE];
+    alignas(1024) uint8_t k[DQS_STAGES][TILE];
+    uint64_t full[DQS_STAGES], empty[DQS_STAGES], acc_full[2], acc_empty[2];
+    uint32_t tmem_base;
+    int abort_flag;
+};
+static_assert(sizeof(DqsSmem) + 1024 <= 232448, "dQ (kept dS) kernel shared memory exceeds 227 KB");
+
+// tmDS: 3-D map over the dS slots viewed as [slots * 128 rows][1][128 columns], box (64, 1, 128).
+__global__ void __launch_bounds__(DQS_THREADS, 1)
+k_bwd_dq_ds(const __grid_constant__ CUtensorMap tmDS, const __grid_constant__ CUtensorMap tmK,
+            const void *__restrict__ meta, __nv_bfloat16 *__restrict__ dQ, int hq, int hkv, const void *ds_buf,
+            int64_t ds_cap) {
+    extern __shared__ uint8_t smem_raw[];
+    DqsSmem &sm = *reinterpret_cast<DqsSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const MetaHeader hd = *meta_ptr<MetaHeader>(meta, 0);
+    if (hd.dev_err != 0 || ds_buf == nullptr || int64_t(hd.n_slots) * hkv > ds_cap) return;   // k_bwd_dq does dQ
+    const int r = hq / hkv;
+    const int n_items = hd.n_qt * hq;
+    const int32_t *kslot = meta_ptr<int32_t>(meta, hd.off_kslot);
+    const int32_t *kfirst = meta_ptr<int32_t>(meta, hd.off_kfirst);
+    volatile int *abort_flag = &sm.abort_flag;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < DQS_STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], 128);
+        }
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(&sm.tmem_base, 256);
+        tmem_relinquish();
+    }
+    if (warp == 4 && lane == 0) {
+        prefetch_tmap(&tmDS);
+        prefetch_tmap(&tmK);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t u = 0;
+            for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+                const DqItem w = dq_decode(meta, hd, item, hq, hkv);
+                const int n = qtile_nkv(w.t);
+                const int qt = (w.t.row0 - w.t.gstart) / BWD_BM;       // query tile within the group
+                const int k0 = kfirst[w.t.group];
+                for (int j = 0; j < n; ++j, ++u) {
+                    const int kl = qtile_kv(w.t, j);                    // key tile within the group (= its first
+                    const int64_t slot = int64_t(w.kh) * hd.n_slots + kslot[k0 + kl] + int64_t(qt - kl) * r +
+                                         (w.h - w.kh * r);
+                    const int st = u % DQS_STAGES;                     //  attending query tile)
+                    if (!bwait(&sm.empty[st], ((u / DQS_STAGES) & 1) ^ 1, abort_flag)) goto done;
+                    mbar_arrive_expect_tx(&sm.full[st], 2 * DqsSmem::TILE);
+                    for (int c = 0; c < 2; ++c) {
+                        tma_load_3d(sm.ds[st] + c * DqsSmem::CHUNK, &tmDS, c * 64, 0, int32_t(slot * BWD_BN),
+                                    &sm.full[st]);
+                        tma_load_3d(sm.k[st] + c * DqsSmem::CHUNK, &tmK, c * 64, w.kh, w.t.gstart + kl * BWD_BN,
+                                    &sm.full[st]);
+                    }
+                }
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t ID = idesc_bf16(128, 128, 1, 1);        // A = dS (M-major), B = K (N-major)
+            const uint64_t a_desc = smem_desc(smem_u32(sm.ds[0]), DqsSmem::CHUNK, 1024);
+            const uint64_t b_desc = smem_desc(smem_u32(sm.k[0]), DqsSmem::CHUNK, 1024);
+            uint32_t u = 0, it_n = 0;
+            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+                const int n = qtile_nkv(meta_ptr<QTile>(meta, hd.off_qts)[item / hq]);
+                const uint32_t b = it_n & 1;
+                if (!bwait(&sm.acc_empty[b], ((it_n >> 1) & 1) ^ 1, abort_flag)) goto done;
+                for (int j = 0; j < n; ++j, ++u) {
+                    const int st = u % DQS_STAGES;
+                    if (!bwait(&sm.full[st], (u / DQS_STAGES) & 1, abort_flag)) goto done;
+                    tc_fence_after();
+                    const uint64_t a = a_desc + uint64_t(st) * (DqsSmem::TILE >> 4);
+                    const uint64_t bb = b_desc + uint64_t(st) * (DqsSmem::TILE >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_ss(tmem + 128 * b, desc_adv(a, kk * 2048), desc_adv(bb, kk * 2048), ID,
+                                (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&sm.empty[st]);
+                }
+                umma_commit(&sm.acc_full[b]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------ epilogue warps (thread = query row)
+        const uint32_t lane_off = uint32_t(warp * 32) << 16;
+        const int rt = warp * 32 + lane;
+        uint32_t it_n = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+            const DqItem w = dq_decode(meta, hd, item, hq, hkv);
+            const uint32_t b = it_n & 1;
+            const int row = w.t.row0 + rt;
+            const bool in_group = row < w.t.gstart + w.t.glen;
+            if (!bwait(&sm.acc_full[b], (it_n >> 1) & 1, abort_flag)) goto done;
+            tc_fence_after();
+            uint32_t a[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + 128 * b + 32 * c, a[c]);
+            tmem_wait_ld(a[0], a[1], a[2], a[3]);
+            tc_fence_before();
+            mbar_arrive(&sm.acc_empty[b]);
+            if (in_group) {                                            // 256 bytes: eight 32-byte stores
+                __nv_bfloat16 *dst = dQ + (int64_t(row) * hq + w.h) * 128;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const uint32_t *x = a[c] + 16 * e;
+                        st_global_v8(dst + 32 * c + 16 * e, pack_bf16x2(__uint_as_float(x[0]), __uint_as_float(x[1])),
+                                     pack_bf16x2(__uint_as_float(x[2]), __uint_as_float(x[3])),
+                                     pack_bf16x2(__uint_as_float(x[4]), __uint_as_float(x[5])),
+                                     pack_bf16x2(__uint_as_float(x[6]), __uint_as_float(x[7])),
+                                     pack_bf16x2(__uint_as_float(x[8]), __uint_as_float(x[9])),
+                                     pack_bf16x2(__uint_as_float(x[10]), __uint_as_float(x[11])),
+                                     pack_bf16x2(__uint_as_float(x[12]), __uint_as_float(x[13])),
+                                     pack_bf16x2(__uint_as_float(x[14]), __uint_as_float(x[15])));
+                    }
+            }
+        }
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
     }
 }
 

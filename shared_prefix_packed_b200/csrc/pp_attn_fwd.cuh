@@ -398,10 +398,10 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         for (int e = 0; e < 16; ++e)
                             pk[e] = pack_bf16x2(__uint_as_float(rr[2 * e]) * inv_l,
                                                 __uint_as_float(rr[2 * e + 1]) * inv_l);
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        for (int e = 0; e < 2; ++e)                        // 64 bytes: two 32-byte stores
+                            st_global_v8(orow + c * 32 + 16 * e, pk[8 * e], pk[8 * e + 1], pk[8 * e + 2], pk[8 * e + 3],
+                                         pk[8 * e + 4], pk[8 * e + 5], pk[8 * e + 6], pk[8 * e + 7]);
                     }
                 }
             }

@@ -279,6 +279,14 @@ __global__ void __launch_bounds__(NT) k_meta_sort(void *meta, int32_t *chunk_off
     }
     __syncthreads();
 
+    // ---- dS slots: one per backward step (key tile, query tile, q head of the kv head), key tiles in order
+    int32_t *kslot = meta_ptr<int32_t>(meta, h->off_kslot);
+    const int r = h->hq / h->hkv;
+    for (int i = threadIdx.x; i <= nk; i += NT) kslot[i] = i < nk ? (kt[i].qb - kt[i].qa) * r : 0;
+    __syncthreads();
+    const int32_t n_slots = block_exclusive_scan<NT>(kslot, nk + 1, s_tmp);
+    if (threadIdx.x == 0) h->n_slots = n_slots;
+
     // ---- backward chunks: split each key tile's query range [qa, qb) into nch near-equal chunks
     for (int i = threadIdx.x; i < nk; i += NT) chunk_off[i] = kt[i].nch;
     __syncthreads();
@@ -297,7 +305,7 @@ __global__ void __launch_bounds__(NT) k_meta_sort(void *meta, int32_t *chunk_off
             w.row0 = t.row0;
             w.gstart = t.gstart;
             w.glen = t.glen;
-            w.pad = 0;
+            w.slot0 = kslot[i] + (w.qa - t.qa) * r;
             bw_tmp[chunk_off[i] + c] = w;
         }
     }

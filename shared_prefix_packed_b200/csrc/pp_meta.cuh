@@ -60,7 +60,7 @@ struct alignas(16) BWork {      // backward work chunk: key tile kt, query tiles
     int32_t qa, qb;
     int32_t split;    // 1 if the key tile is split over several chunks (partials are added into fp32 scratch)
     int32_t row0, gstart, glen;   // the key tile's first row, group offset and group length (copied from kt)
-    int32_t pad;
+    int32_t slot0;    // dS slot of the chunk's first step (query tile qa, the first q head of the kv head)
 };
 
 struct alignas(16) MetaHeader {
@@ -72,7 +72,8 @@ struct alignas(16) MetaHeader {
     int32_t n_split;     // key tiles split over several chunks
     int32_t cap_qt, cap_kt, cap_bw;
     int32_t dev_err;     // non-zero if the builder found inconsistent input
-    int32_t pad[2];
+    int32_t n_slots;     // backward steps (key tile, query tile, q head): one dS tile each when dS is kept
+    int32_t pad;
     int64_t off_seg_start;   // int32[T]: packed start of each token's segment
     int64_t off_key_end;     // int32[T]: packed end of the query interval that attends each token as a key
     int64_t off_groups;      // GroupInfo[G]
@@ -82,6 +83,8 @@ struct alignas(16) MetaHeader {
     int64_t off_qts;         // QTile[cap_qt]: the query tiles in that order (one load per work item)
     int64_t off_kt;          // KTile[cap_kt]
     int64_t off_bw;          // BWork[cap_bw], sorted by decreasing cost
+    int64_t off_kslot;       // int32[cap_kt + 1]: first dS slot of each key tile (steps in tile order, then total)
+    int64_t off_kfirst;      // int32[G + 1]: first key tile of each group (inside the builder scratch, kept)
     int64_t off_scratch;     // builder scratch: qoff int32[G+1], koff int32[G+1], tmp int32[max(cap_kt, SORT_BINS)]
     int64_t off_bw_tmp;      // builder scratch: BWork[cap_bw] before sorting
     int64_t total_bytes;
@@ -111,7 +114,9 @@ __host__ __device__ inline MetaHeader meta_layout(int64_t T, int32_t G, int32_t 
     h.off_qts = o;       o = align256(o + int64_t(sizeof(QTile)) * h.cap_qt);
     h.off_kt = o;        o = align256(o + int64_t(sizeof(KTile)) * h.cap_kt);
     h.off_bw = o;        o = align256(o + int64_t(sizeof(BWork)) * h.cap_bw);
+    h.off_kslot = o;     o = align256(o + 4 * int64_t(h.cap_kt + 1));
     h.off_scratch = o;
+    h.off_kfirst = o + 4 * int64_t(G + 1);       // the builder's koff, written by k_meta_groups and never reused
     o = align256(o + 4 * (2 * int64_t(G + 1) + (h.cap_kt > SORT_BINS ? h.cap_kt : SORT_BINS)));
     h.off_bw_tmp = o;    o = align256(o + int64_t(sizeof(BWork)) * h.cap_bw);
     h.total_bytes = o;

@@ -274,6 +274,15 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
                        __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
+// One 32-byte global store (sm_100): half the store instructions of 16-byte vectors for the same bytes. addr must be
+// 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void *addr, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t a4, uint32_t a5, uint32_t a6, uint32_t a7) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(addr), "r"(a0), "r"(a1), "r"(a2),
+                 "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+                 : "memory");
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

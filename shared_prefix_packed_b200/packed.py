@@ -31,8 +31,10 @@ class PackedBatch:
         cu = [0]
         for n in lens:
             cu.append(cu[-1] + n)
-        self.groups = torch.tensor(groups, dtype=torch.int32).to(self.device)
-        self.cu_seqlens = torch.tensor(cu, dtype=torch.int32).to(self.device)
+        self.groups_host = torch.tensor(groups, dtype=torch.int32).reshape(-1, 2)
+        self.cu_host = torch.tensor(cu, dtype=torch.int32)
+        self.groups = self.groups_host.to(self.device)
+        self.cu_seqlens = self.cu_host.to(self.device)
         nbytes = _lib.pp_meta_bounds(len(groups), len(lens), self.T, hq, hkv)
         self.meta = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self.pos_ids = torch.empty(max(self.T, 1), dtype=torch.int32, device=self.device)
@@ -46,8 +48,11 @@ class PackedBatch:
 
     @property
     def ws_bwd(self):
+        """Backward workspace: the base scratch plus room to keep every step's dS tile (the faster dq path)."""
         if self._ws_bwd is None:
             n = _lib.pp_workspace_bytes(_lib.PP_PASS_BWD, self.T, self.hq, self.hkv, self.d)
+            if self.d == 128:
+                n += _lib.pp_bwd_ds_bytes(self.groups_host, self.cu_host, self.hq, self.hkv)
             self._ws_bwd = torch.empty(n, dtype=torch.uint8, device=self.device)
         return self._ws_bwd
 

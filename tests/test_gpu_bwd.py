@@ -101,3 +101,29 @@ def test_bwd_rejects_unsupported():
     lse = torch.zeros(4, 15, device="cuda")
     with pytest.raises(PPError, match="UNSUPPORTED"):
         b.backward(x, kv, kv, x, lse, x)
+
+
+@pytest.mark.parametrize("case", [0, 4, 6, 8])
+def test_bwd_both_dq_paths(case):
+    """The same backward with the base workspace (dQ kernel recomputes S and dP) and with room for every step's dS
+    tile (dQ formed from the kept tiles): both within the bound of the oracle, and only the second writes dS."""
+    from shared_prefix_packed_b200 import PackedBatch, _lib, pp_get_status
+    P, S = SMALL[case]
+    hq, hkv, d = 4, 2, 128
+    inp = W.make_inputs("dpo", P, S, seed=700 + case, with_dout=True, heads=(hq, hkv, d))
+    b = PackedBatch(P, S, hq, hkv, d)
+    q, k, v, do = (inp[x].cuda() for x in ("q", "k", "v", "dout"))
+    o, lse = b.forward(q, k, v)
+    base = _lib.pp_workspace_bytes(_lib.PP_PASS_BWD, b.T, hq, hkv, d)
+    extra = _lib.pp_bwd_ds_bytes(b.groups_host, b.cu_host, hq, hkv)
+    ref = oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["dout"], P, S)
+    for ws_bytes in (base, base + extra):
+        ws = torch.full((ws_bytes,), 0xFF, dtype=torch.uint8, device="cuda")
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        _lib.pp_attn_bwd(q, k, v, o, lse, do, b.meta, dq, dk, dv, ws)
+        pp_get_status()
+        for got, want in zip((dq, dk, dv), ref):
+            assert rel_fro(to_np64(got), want) <= REL_TOL
+        if ws_bytes > base:
+            kept = ws[(base + 1023) // 1024 * 1024:]
+            assert bool((kept[: extra - 1024] != 0xFF).any()), "the kept-dS path did not run"

@@ -65,3 +65,27 @@ def test_noalloc_scratch_size_matches_the_header():
     assert m, "PP_NOALLOC_SCRATCH_BYTES not found in pp.h"
     from shared_prefix_packed_b200 import _lib
     assert _lib.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
+def test_bwd_ds_bytes_counts_the_nonempty_tile_pairs():
+    """pp_bwd_ds_bytes (host only) = 1024 + 32 KiB per backward step, a step being a non-empty (query tile, key
+    tile) pair of the mask times the q heads: checked against the oracle's tile set on edge cases and the
+    workloads' group lengths."""
+    import torch
+    import oracle
+    import workloads as W
+    from shared_prefix_packed_b200 import _lib
+    cases = [([3], [[2, 0, 3]]), ([0], [[130, 77]]), ([300], [[]]), ([127, 129, 1], [[1, 255], [3], [0]]),
+             ([2100], [[700, 900]]), ([0], [[0]])]
+    cases += [W.group_lengths(n) for n in ("dpo", "grpo")]
+    for P, S in cases:
+        groups = torch.tensor([(p, len(ss)) for p, ss in zip(P, S)], dtype=torch.int32).reshape(-1, 2)
+        cu = [0]
+        for p, ss in zip(P, S):
+            cu.append(cu[-1] + p)
+            for x in ss:
+                cu.append(cu[-1] + x)
+        pairs = len(oracle.tile_classes(P, S, 128, 128))
+        for hq, hkv in ((4, 2), (32, 8), (7, 1)):
+            got = _lib.pp_bwd_ds_bytes(groups, torch.tensor(cu, dtype=torch.int32), hq, hkv)
+            assert got == 1024 + 32768 * pairs * hq, (P, S, hq, hkv)
