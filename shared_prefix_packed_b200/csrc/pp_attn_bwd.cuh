@@ -220,7 +220,7 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
 // 64 columns of dK (dS^T carried the scale) or dV of one key row, from registers: bf16 for an unsplit key tile,
 // fp32 adds into the workspace for a split one.
 __device__ __forceinline__ void bwd_store_kv64(const uint32_t (&a)[32], const uint32_t (&b)[32], bool split,
-                                               float *acc, __nv_bfloat16 *dst) {
+                                               float *acc, __nv_bfloat16 *dst, bool v8) {
     if (split) {
 #pragma unroll
         for (int e = 0; e < 8; ++e)
@@ -234,11 +234,11 @@ __device__ __forceinline__ void bwd_store_kv64(const uint32_t (&a)[32], const ui
         auto pk = [](const uint32_t *x, int i) { return pack_bf16x2(__uint_as_float(x[i]), __uint_as_float(x[i + 1])); };
 #pragma unroll
         for (int e = 0; e < 2; ++e)
-            st_global_v8(dst + 16 * e, pk(a, 16 * e), pk(a, 16 * e + 2), pk(a, 16 * e + 4), pk(a, 16 * e + 6),
+            st_global_32(dst + 16 * e, v8, pk(a, 16 * e), pk(a, 16 * e + 2), pk(a, 16 * e + 4), pk(a, 16 * e + 6),
                          pk(a, 16 * e + 8), pk(a, 16 * e + 10), pk(a, 16 * e + 12), pk(a, 16 * e + 14));
 #pragma unroll
         for (int e = 0; e < 2; ++e)
-            st_global_v8(dst + 32 + 16 * e, pk(b, 16 * e), pk(b, 16 * e + 2), pk(b, 16 * e + 4), pk(b, 16 * e + 6),
+            st_global_32(dst + 32 + 16 * e, v8, pk(b, 16 * e), pk(b, 16 * e + 2), pk(b, 16 * e + 4), pk(b, 16 * e + 6),
                          pk(b, 16 * e + 8), pk(b, 16 * e + 10), pk(b, 16 * e + 12), pk(b, 16 * e + 14));
     }
 }
@@ -519,6 +519,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
         const int cb = 64 * wx;                                        // first query column of this half
         // dS kept for the dQ kernel: slot s holds the step's dS^T tile, [128 key rows][128 query columns] bf16
         const bool keep_ds = ds_buf != nullptr && int64_t(hd.n_slots) * hkv <= ds_cap;
+        const bool out_v8 = aligned32(wx == 0 ? dK : dV);              // rows are 256 bytes: the base decides
         uint32_t g = 0, it_n = 0;
         const int32_t *key_end = meta_ptr<int32_t>(meta, hd.off_key_end);
         // Item epilogue, run inside the next item's first step (after its P, before its dS), when dK/dV of the
@@ -542,7 +543,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     tc_fence_before();
                     mbar_arrive(&sm.dkv_free);
                 }
-                if (ep_yin) bwd_store_kv64(a, b, ep_split, acc + 64 * half, dst + 64 * half);
+                if (ep_yin) bwd_store_kv64(a, b, ep_split, acc + 64 * half, dst + 64 * half, out_v8);
             }
             return true;
         };
@@ -643,7 +644,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                         __nv_bfloat16 *dst = ds_buf + (slot * BWD_BN + jr) * BWD_BM + cb;   // 32-byte aligned
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            st_global_v8(dst + 16 * e, ds[8 * e], ds[8 * e + 1], ds[8 * e + 2], ds[8 * e + 3],
+                            st_global_32(dst + 16 * e, true, ds[8 * e], ds[8 * e + 1], ds[8 * e + 2], ds[8 * e + 3],
                                          ds[8 * e + 4], ds[8 * e + 5], ds[8 * e + 6], ds[8 * e + 7]);
                     }
                 }

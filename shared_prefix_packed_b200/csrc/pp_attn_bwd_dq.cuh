@@ -514,6 +514,7 @@ k_bwd_dq_ds(const __grid_constant__ CUtensorMap tmDS, const __grid_constant__ CU
         // ------------------------------------------------------------------ epilogue warps (thread = query row)
         const uint32_t lane_off = uint32_t(warp * 32) << 16;
         const int rt = warp * 32 + lane;
+        const bool dq_v8 = aligned32(dQ);                                // rows are 256 bytes: the base decides
         uint32_t it_n = 0;
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
             const DqItem w = dq_decode(meta, hd, item, hq, hkv);
@@ -535,7 +536,7 @@ k_bwd_dq_ds(const __grid_constant__ CUtensorMap tmDS, const __grid_constant__ CU
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const uint32_t *x = a[c] + 16 * e;
-                        st_global_v8(dst + 32 * c + 16 * e, pack_bf16x2(__uint_as_float(x[0]), __uint_as_float(x[1])),
+                        st_global_32(dst + 32 * c + 16 * e, dq_v8, pack_bf16x2(__uint_as_float(x[0]), __uint_as_float(x[1])),
                                      pack_bf16x2(__uint_as_float(x[2]), __uint_as_float(x[3])),
                                      pack_bf16x2(__uint_as_float(x[4]), __uint_as_float(x[5])),
                                      pack_bf16x2(__uint_as_float(x[6]), __uint_as_float(x[7])),

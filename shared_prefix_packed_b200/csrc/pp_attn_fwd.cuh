@@ -275,6 +275,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int rt = lane_base + lane;                       // row within the tile = TMEM lane
         const uint32_t t_s = tmem + (uint32_t(lane_base) << 16) + wg * 128;
         const uint32_t t_o = tmem + (uint32_t(lane_base) << 16) + 256 + wg * 128;
+        const bool o_v8 = aligned32(O);                                  // rows are d * 2 bytes: the base decides
         uint32_t s_cnt = 0, pv_cnt = 0;
         for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
             const FwdItem w = fwd_decode(meta, hd, item, hq, hkv);
@@ -400,7 +401,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                                 __uint_as_float(rr[2 * e + 1]) * inv_l);
 #pragma unroll
                         for (int e = 0; e < 2; ++e)                        // 64 bytes: two 32-byte stores
-                            st_global_v8(orow + c * 32 + 16 * e, pk[8 * e], pk[8 * e + 1], pk[8 * e + 2], pk[8 * e + 3],
+                            st_global_32(orow + c * 32 + 16 * e, o_v8, pk[8 * e], pk[8 * e + 1], pk[8 * e + 2], pk[8 * e + 3],
                                          pk[8 * e + 4], pk[8 * e + 5], pk[8 * e + 6], pk[8 * e + 7]);
                     }
                 }

@@ -274,14 +274,21 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
                        __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
-// One 32-byte global store (sm_100): half the store instructions of 16-byte vectors for the same bytes. addr must be
-// 32-byte aligned.
-__device__ __forceinline__ void st_global_v8(void *addr, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+// 32 bytes to global memory. v8: one 32-byte store (sm_100), addr 32-byte aligned; otherwise two 16-byte stores.
+// The library's tensors need only 16-byte alignment, so kernels test their base pointers once and pass v8.
+__device__ __forceinline__ void st_global_32(void *addr, bool v8, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                              uint32_t a4, uint32_t a5, uint32_t a6, uint32_t a7) {
-    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(addr), "r"(a0), "r"(a1), "r"(a2),
-                 "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
-                 : "memory");
+    if (v8) {
+        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(addr), "r"(a0), "r"(a1),
+                     "r"(a2), "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+                     : "memory");
+    } else {
+        uint4 *p = reinterpret_cast<uint4 *>(addr);
+        p[0] = make_uint4(a0, a1, a2, a3);
+        p[1] = make_uint4(a4, a5, a6, a7);
+    }
 }
+__device__ __forceinline__ bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31) == 0; }
 
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;

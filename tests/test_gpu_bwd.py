@@ -127,3 +127,31 @@ def test_bwd_both_dq_paths(case):
         if ws_bytes > base:
             kept = ws[(base + 1023) // 1024 * 1024:]
             assert bool((kept[: extra - 1024] != 0xFF).any()), "the kept-dS path did not run"
+
+
+def test_fwd_bwd_tensors_16_byte_aligned_only():
+    """Every tensor 16-byte aligned but not 32-byte aligned (views 16 bytes into their buffers): the 32-byte vector
+    loads and stores fall back to 16-byte ones, and the results still match the oracle."""
+    from shared_prefix_packed_b200 import PackedBatch, pp_get_status
+    P, S = SMALL[8]
+    hq, hkv, d = 4, 2, 128
+    inp = W.make_inputs("dpo", P, S, seed=901, with_dout=True, heads=(hq, hkv, d))
+    b = PackedBatch(P, S, hq, hkv, d)
+
+    def offset_like(t):
+        buf = torch.empty(t.numel() + 8, dtype=torch.bfloat16, device="cuda")
+        v = buf[8:].view(t.shape)
+        assert v.data_ptr() % 32 == 16
+        return v
+
+    q, k, v, do = (offset_like(inp[x]) for x in ("q", "k", "v", "dout"))
+    for dst, x in zip((q, k, v, do), ("q", "k", "v", "dout")):
+        dst.copy_(inp[x].cuda())
+    o = offset_like(q)
+    o, lse = b.forward(q, k, v, out=o)
+    dq, dk, dv = offset_like(q), offset_like(k), offset_like(v)
+    b.backward(q, k, v, o, lse, do, dq=dq, dk=dk, dv=dv)
+    pp_get_status()
+    ref = oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["dout"], P, S)
+    for got, want in zip((dq, dk, dv), ref):
+        assert rel_fro(to_np64(got), want) <= REL_TOL
