@@ -264,7 +264,7 @@ def run_gpu(args):
 
     # our kernels per step: metadata (header + 4 stages), RoPE, forward, and the backward's lse/D pass, dK/dV kernel,
     # dQ kernel and split-tile conversion (the workspace memset is a driver memset, not counted)
-    launches_per_step = 5 + (1 if w.rope else 0) + 1 + (4 if w.backward else 0)
+    launches_per_step = 5 + (1 if w.rope else 0) + 1 + (5 if w.backward else 0)
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)                      # nvidia-smi needs a moment before its first sample
@@ -390,7 +390,8 @@ def run_gpu(args):
     dom = "attn_bwd" if w.backward and parts["attn_bwd"] >= parts["attn_fwd"] else "attn_fwd"
     dom_flops = f_bwd if dom == "attn_bwd" else f_fwd
     achieved = dom_flops / (parts[dom] * 1e-3) / 1e12
-    kernels = ["k_bwd_pre", "k_bwd_tc", "k_bwd_dq", "k_bwd_convert"] if dom == "attn_bwd" else ["k_attn_fwd_tc"]
+    kernels = (["k_bwd_pre", "k_bwd_tc", "k_bwd_dq", "k_bwd_dq_ds", "k_bwd_convert"] if dom == "attn_bwd"
+               else ["k_attn_fwd_tc"])
     roofline = {"bound": "tensor", "kernel": f"pp_{dom} ({' + '.join(kernels)})",
                 "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": recorded_traffic(kernels),
