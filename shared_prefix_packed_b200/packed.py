@@ -19,8 +19,12 @@ class PackedBatch:
     """
 
     def __init__(self, prefix_lens: Sequence[int], suffix_lens: Sequence[Sequence[int]], hq: int, hkv: int, d: int,
-                 device="cuda", stream=None):
+                 device="cuda", stream=None, ds_budget_bytes=None):
+        """ds_budget_bytes: most device memory the backward may take to keep every step's dS tile (the faster dq
+        path, ``pp_bwd_ds_bytes``); None means half of the memory free when the backward workspace is first made,
+        0 disables it. Either way the results are the same."""
         self.hq, self.hkv, self.d = hq, hkv, d
+        self.ds_budget_bytes = ds_budget_bytes
         self.device = torch.device(device)
         groups, lens = [], []
         for p, ss in zip(prefix_lens, suffix_lens):
@@ -52,7 +56,12 @@ class PackedBatch:
         if self._ws_bwd is None:
             n = _lib.pp_workspace_bytes(_lib.PP_PASS_BWD, self.T, self.hq, self.hkv, self.d)
             if self.d == 128:
-                n += _lib.pp_bwd_ds_bytes(self.groups_host, self.cu_host, self.hq, self.hkv)
+                extra = _lib.pp_bwd_ds_bytes(self.groups_host, self.cu_host, self.hq, self.hkv)
+                budget = self.ds_budget_bytes
+                if budget is None:
+                    budget = torch.cuda.mem_get_info(self.device)[0] // 2
+                if extra <= budget:
+                    n += extra
             self._ws_bwd = torch.empty(n, dtype=torch.uint8, device=self.device)
         return self._ws_bwd
 

@@ -155,3 +155,21 @@ def test_fwd_bwd_tensors_16_byte_aligned_only():
     ref = oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["dout"], P, S)
     for got, want in zip((dq, dk, dv), ref):
         assert rel_fro(to_np64(got), want) <= REL_TOL
+
+
+def test_bwd_ds_budget_zero_uses_the_recompute_path():
+    """PackedBatch with ds_budget_bytes=0 allocates only the base workspace (the dQ kernel recomputes S and dP); the
+    gradients agree with the oracle either way."""
+    from shared_prefix_packed_b200 import PackedBatch, _lib, pp_get_status
+    P, S = SMALL[6]
+    hq, hkv, d = 4, 2, 128
+    inp = W.make_inputs("dpo", P, S, seed=950, with_dout=True, heads=(hq, hkv, d))
+    b = PackedBatch(P, S, hq, hkv, d, ds_budget_bytes=0)
+    assert b.ws_bwd.numel() == _lib.pp_workspace_bytes(_lib.PP_PASS_BWD, b.T, hq, hkv, d)
+    q, k, v, do = (inp[x].cuda() for x in ("q", "k", "v", "dout"))
+    o, lse = b.forward(q, k, v)
+    dq, dk, dv = b.backward(q, k, v, o, lse, do)
+    pp_get_status()
+    ref = oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["dout"], P, S)
+    for got, want in zip((dq, dk, dv), ref):
+        assert rel_fro(to_np64(got), want) <= REL_TOL
