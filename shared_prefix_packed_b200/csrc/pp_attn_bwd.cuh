@@ -4,11 +4,14 @@
 //   dS_ij = p_ij (dO_i . v_j - D_i),  dQ_i = scale sum_j dS_ij k_j,
 //   dK_j = scale sum_h sum_i dS_ij q_i,  dV_j = sum_h sum_i p_ij dO_i   (h over the q heads of j's kv head).
 //
-// Four kernels:
+// Kernels:
 //   k_bwd_pre     (-lse / scale, -D) per row and head, D = rowsum(dO * O) in fp32 (HBM-bound).
-//   k_bwd_tc      dK and dV: key/value-stationary tensor-core kernel (below).
-//   k_bwd_dq      dQ: query-stationary tensor-core kernel (pp_attn_bwd_dq.cuh); recomputes S and dP per tile so
-//                 that every dQ row is produced by exactly one CTA (no fp32 accumulator, no reduction traffic).
+//   k_bwd_tc      dK and dV: key/value-stationary tensor-core kernel (below); when the workspace has room it also
+//                 keeps every step's dS^T tile there.
+//   k_bwd_dq_ds   dQ = sum dS K from the kept tiles (pp_attn_bwd_dq.cuh), streaming them once.
+//   k_bwd_dq      dQ when the tiles are not kept: query-stationary tensor-core kernel (pp_attn_bwd_dq.cuh) that
+//                 recomputes S and dP per tile. Either way every dQ row is produced by exactly one CTA (no fp32
+//                 accumulator, no reduction traffic).
 //   k_bwd_convert the fp32 dK/dV partials of split key tiles to bf16.
 // k_bwd_tc: a work item is (key tile of 128 rows, kv head, chunk of the query tiles that attend it). Seen from key
 // y the attending queries are one interval [y, e(y)) (pp_meta.cuh), so a key tile's query tiles are one contiguous

@@ -1,4 +1,6 @@
-// pp_attn_bwd_dq.cuh - the dQ half of the backward: query-stationary tcgen05 kernel, no atomics.
+// pp_attn_bwd_dq.cuh - the dQ half of the backward, two ways, neither with atomics. k_bwd_dq_ds (at the end of this
+// file) forms dQ from the dS tiles the dK/dV kernel kept in the workspace; k_bwd_dq, below, recomputes S and dP per
+// tile when the workspace cannot hold those tiles.
 //
 // dQ_i = scale sum_j dS_ij k_j with dS_ij = p_ij (dO_i . v_j - D_i) and p_ij = exp(s_ij - lse_i), over the allowed
 // keys j of query row i (pp_meta.cuh). A work item is (query tile of 128 rows, one q head); it walks the same key
