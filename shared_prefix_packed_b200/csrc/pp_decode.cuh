@@ -26,7 +26,8 @@ namespace pp {
 
 constexpr int DEC_CH = 128;           // keys per chunk (the MMA N of S, the K of P V)
 constexpr int DEC_D = 128;            // head dim
-constexpr int DEC_REC = 132;          // floats per record: max (base 2), sum, two pad, O[128] (16-byte aligned)
+constexpr int DEC_REC = 136;          // floats per record: max (base 2), sum, six pad, O[128] (32-byte aligned)
+constexpr int DEC_REC_O = 8;          // offset of O in a record
 constexpr int DEC_STAGES = 3;         // K and V chunk rings
 constexpr int DEC_THREADS = 320;      // warps 0-7 softmax / records (two warpgroups), warp 8 TMA, warp 9 MMA
 
@@ -429,7 +430,7 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             }
             tc_fence_before();
             mbar_arrive(&sm.p_full[b]);
-            // the job's O (PV(u)) -> its record (max in base-2 units, sum, two pad, O[128])
+            // the job's O (PV(u)) -> its record (max in base-2 units, sum, six pad, O[128])
             if (!bwait(&sm.o_full[b], (u >> 1) & 1, abort_flag)) goto done;
             tc_fence_after();
             if (any) {
@@ -440,11 +441,11 @@ k_dec_chunk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     tmem_ld32(tmem + lane_off + 256 + 128 * b + 32 * c, o);
                     tmem_wait_ld(o);
                     if (valid) {
-                        float4 *dst = reinterpret_cast<float4 *>(part + rec + 4 + 32 * c);
+                        float *dst = part + rec + DEC_REC_O + 32 * c;       // 32-byte aligned
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            dst[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
-                                                 __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+                        for (int e = 0; e < 4; ++e)
+                            st_global_32(dst + 8 * e, true, o[8 * e], o[8 * e + 1], o[8 * e + 2], o[8 * e + 3],
+                                         o[8 * e + 4], o[8 * e + 5], o[8 * e + 6], o[8 * e + 7]);
                     }
                 }
                 if (valid) *reinterpret_cast<float4 *>(part + rec) = make_float4(m, l, 0.f, 0.f);
@@ -519,14 +520,14 @@ __global__ void __launch_bounds__(DEC_COMB_WARPS * 32, 3) k_dec_combine(int hq, 
                     const float *r = rec_of(j + u);
                     m[u] = r[0];
                     l[u] = r[1];
-                    v[u] = *reinterpret_cast<const float4 *>(r + 4 + 4 * lane);
+                    v[u] = *reinterpret_cast<const float4 *>(r + DEC_REC_O + 4 * lane);
                 }
 #pragma unroll
                 for (int u = 0; u < UNROLL; ++u) add(m[u], l[u], v[u]);
             }
             for (; j < n; ++j) {
                 const float *r = rec_of(j);
-                add(r[0], r[1], *reinterpret_cast<const float4 *>(r + 4 + 4 * lane));
+                add(r[0], r[1], *reinterpret_cast<const float4 *>(r + DEC_REC_O + 4 * lane));
             }
         }
         const bool any = L > 0.f;
