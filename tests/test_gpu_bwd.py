@@ -47,7 +47,7 @@ SMALL = [
 
 
 @pytest.mark.parametrize("case", range(len(SMALL)))
-@pytest.mark.parametrize("heads", [(4, 2), (7, 1)])
+@pytest.mark.parametrize("heads", [(4, 2), (7, 1), (2, 2)])
 def test_bwd_small(case, heads):
     P, S = SMALL[case]
     hq, hkv = heads
