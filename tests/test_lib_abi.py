@@ -89,3 +89,18 @@ def test_bwd_ds_bytes_counts_the_nonempty_tile_pairs():
         for hq, hkv in ((4, 2), (32, 8), (7, 1)):
             got = _lib.pp_bwd_ds_bytes(groups, torch.tensor(cu, dtype=torch.int32), hq, hkv)
             assert got == 1024 + 32768 * pairs * hq, (P, S, hq, hkv)
+
+
+def test_bwd_ds_bytes_rejects_inconsistent_descriptors():
+    """Descriptors that disagree with the segment bounds are refused on the host (no size is returned)."""
+    import pytest
+    import torch
+    from shared_prefix_packed_b200 import _lib
+    groups = torch.tensor([[4, 2]], dtype=torch.int32)
+    with pytest.raises(_lib.PPError):                      # prefix length 4, but the first segment holds 3 rows
+        _lib.pp_bwd_ds_bytes(groups, torch.tensor([0, 3, 5, 9], dtype=torch.int32), 4, 2)
+    with pytest.raises(_lib.PPError):                      # two responses declared, one segment present
+        _lib.pp_bwd_ds_bytes(groups, torch.tensor([0, 4, 9], dtype=torch.int32), 4, 2)
+    with pytest.raises(_lib.PPError):                      # hq not a multiple of hkv
+        _lib.pp_bwd_ds_bytes(groups, torch.tensor([0, 4, 6, 9], dtype=torch.int32), 3, 2)
+    assert _lib.pp_bwd_ds_bytes(groups, torch.tensor([0, 4, 6, 9], dtype=torch.int32), 4, 2) == 1024 + 32768 * 4
