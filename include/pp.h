@@ -141,7 +141,7 @@ PP_API pp_status pp_workspace_bytes(int32_t which, int64_t T, int32_t hq, int32_
  * instead of recomputing the scores. A step is (key tile of 128 rows, query tile of 128 rows that attends it, q
  * head), for every kv head; the count follows the mask (same descriptors as pp_build_meta). groups_host,
  * cu_host: host copies of the descriptors and segment bounds; *bytes (host) receives 1024 + steps * 32768.
- * Returns PP_ERR_INVALID_ARG for descriptors that disagree with the segments.
+ * Returns PP_ERR_INVALID_ARG for descriptors that disagree with the segments or segment bounds that decrease.
  */
 PP_API pp_status pp_bwd_ds_bytes(const pp_group_desc *groups_host, int32_t G, const int32_t *cu_host,
                                  int32_t nseg, int32_t hq, int32_t hkv, int64_t *bytes);

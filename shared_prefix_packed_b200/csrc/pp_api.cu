@@ -297,9 +297,11 @@ pp_status pp_bwd_ds_bytes(const pp_group_desc *groups_host, int32_t G, const int
     for (int32_t g = 0; g < G; ++g) {
         const int32_t P = groups_host[g].prefix_len, k = groups_host[g].num_suffixes;
         if (k < 0 || P < 0 || s + 1 + int64_t(k) > nseg) return fail(PP_ERR_INVALID_ARG, "descriptors exceed num_segments");
+        for (int32_t j = s; j <= s + k; ++j)
+            if (cu_host[j + 1] < cu_host[j]) return fail(PP_ERR_INVALID_ARG, "segment bounds must not decrease");
         const int32_t start = cu_host[s], end = cu_host[s + 1 + k];
         const int32_t L = end - start;
-        if (cu_host[s + 1] - start != P || L < P) return fail(PP_ERR_INVALID_ARG, "prefix length disagrees with segments");
+        if (cu_host[s + 1] - start != P) return fail(PP_ERR_INVALID_ARG, "prefix length disagrees with segments");
         int32_t seg = s + 1;                                        // segment of the current key (responses)
         for (int32_t y0 = 0; y0 < L; y0 += pp::BWD_BN) {
             const int32_t ylast = std::min(y0 + pp::BWD_BN, L) - 1;

@@ -101,6 +101,8 @@ def test_bwd_ds_bytes_rejects_inconsistent_descriptors():
         _lib.pp_bwd_ds_bytes(groups, torch.tensor([0, 3, 5, 9], dtype=torch.int32), 4, 2)
     with pytest.raises(_lib.PPError):                      # two responses declared, one segment present
         _lib.pp_bwd_ds_bytes(groups, torch.tensor([0, 4, 9], dtype=torch.int32), 4, 2)
+    with pytest.raises(_lib.PPError):                      # a response with a negative row count
+        _lib.pp_bwd_ds_bytes(groups, torch.tensor([0, 4, 3, 9], dtype=torch.int32), 4, 2)
     with pytest.raises(_lib.PPError):                      # hq not a multiple of hkv
         _lib.pp_bwd_ds_bytes(groups, torch.tensor([0, 4, 6, 9], dtype=torch.int32), 3, 2)
     assert _lib.pp_bwd_ds_bytes(groups, torch.tensor([0, 4, 6, 9], dtype=torch.int32), 4, 2) == 1024 + 32768 * 4
