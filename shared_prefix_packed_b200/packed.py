@@ -90,11 +90,11 @@ class PackedBatch:
     def decode(self, q, k_cache, v_cache, softmax_scale: float = 0.0, out=None, lse=None, stream=None):
         """One decoding step over this layout as a KV cache: q [n_resp, hq, d], one query per response (its newest
         token, the last row of its segment); returns (o [n_resp, hq, d], lse [hq, n_resp])."""
-        n_resp = self.cu_seqlens.numel() - 1 - self.groups.shape[0]
+        n_resp = self.cu_host.numel() - 1 - self.groups_host.shape[0]
         o = torch.empty_like(q) if out is None else out
         l = torch.empty(self.hq, n_resp, dtype=torch.float32, device=q.device) if lse is None else lse
         if getattr(self, "_ws_dec", None) is None:
-            n = _lib.pp_decode_workspace_bytes(self.groups.cpu(), self.cu_seqlens.cpu(), self.hq)
+            n = _lib.pp_decode_workspace_bytes(self.groups_host, self.cu_host, self.hq)
             self._ws_dec = torch.empty(n, dtype=torch.uint8, device=self.device)
         _lib.pp_decode_attn(q, k_cache, v_cache, self.groups, self.cu_seqlens, o, l, self._ws_dec, softmax_scale,
                             stream)
