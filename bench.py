@@ -128,9 +128,9 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernels):
+def recorded_traffic(kernels, workload):
     """DRAM bytes per launch summed over `kernels`, from the committed ncu summary, if every one of them was taken
-    on the current kernel sources (None otherwise)."""
+    on the current kernel sources and on this workload (None otherwise)."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
@@ -139,7 +139,7 @@ def recorded_traffic(kernels):
     with open(path) as f:
         for ln in f:
             parts = dict(p.split("=", 1) for p in ln.strip().split() if "=" in p)
-            if parts.get("kernel") in kernels and parts.get("sources") == src:
+            if parts.get("kernel") in kernels and parts.get("sources") == src and parts.get("workload") == workload:
                 try:
                     found[parts["kernel"]] = float(parts["dram_bytes_per_launch"])
                 except (KeyError, ValueError):
@@ -394,7 +394,7 @@ def run_gpu(args):
                else ["k_attn_fwd_tc"])
     roofline = {"bound": "tensor", "kernel": f"pp_{dom} ({' + '.join(kernels)})",
                 "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": recorded_traffic(kernels),
+                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": recorded_traffic(kernels, name),
                 "peak_source": peaks["source"] + " bf16_tflops (burst)",
                 "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4)
                 if peaks.get("bf16_tflops_sustained") else None,
@@ -813,8 +813,7 @@ def run_logprobs(args):
                    "l2": f"logits {T * V * 2 / 2**30:.1f} GiB, larger than L2, no flush"},
         "roofline": {"bound": "hbm", "kernel": "k_response_logprobs", "achieved": round(gbs, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                     "traffic": recorded_traffic(["k_response_logprobs"]) if V == W.LOGPROB_VOCAB and
-                     name == "dpo" else None,
+                     "traffic": recorded_traffic(["k_response_logprobs"], f"{name}-layout-vocab{V}"),
                      "peak_source": peaks["source"] + " hbm_gbs", "bytes_per_launch": nbytes},
         "gpu_launches": args.steps, "clocks": clocks}))
 
