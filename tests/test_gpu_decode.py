@@ -101,3 +101,35 @@ def test_decode_rejects_inconsistent_bounds():
     with pytest.raises(PPError, match="DEVICE_INPUT"):
         pp_get_status()
     assert torch.isnan(lse).all()
+
+
+EMPTY_RESP = [
+    ([5], [[0, 3, 0]]),             # zero-length responses: their query sees the prefix alone
+    ([0, 130], [[0, 2], [0]]),      # no prefix and no rows: no key at all; a prefix of two chunks alone
+]
+
+
+@pytest.mark.parametrize("case", range(len(EMPTY_RESP)))
+@pytest.mark.parametrize("heads", [(8, 2), (4, 4)])
+def test_decode_zero_length_responses(case, heads):
+    """A response with no cached row decodes against its group's prefix alone, which is what the prefix's last row
+    attends in the packed forward; with no prefix either it sees no key and gets O = 0 and LSE = -inf."""
+    P, S = EMPTY_RESP[case]
+    hq, hkv = heads
+    inp, qd, last_rows, T, o, lse = _decode_case(P, S, hq, hkv, 700 + case)
+    rows, i, start = [], 0, 0
+    for p, ss in zip(P, S):
+        for _ in ss:
+            rows.append(last_rows[i] if last_rows[i] is not None else (start + p - 1 if p > 0 else None))
+            i += 1
+        start += p + sum(ss)
+    assert any(r is None for r in last_rows)
+    for i, row in enumerate(rows):
+        if row is None:
+            assert torch.all(o[i].float() == 0) and torch.all(torch.isneginf(lse[:, i]))
+            continue
+        qp = torch.zeros((T, hq, 128), dtype=torch.bfloat16)
+        qp[row] = qd[i]
+        O_ref, L_ref = oracle.attention_forward_rows(qp, inp["k"], inp["v"], P, S, [row])
+        assert np.max(np.abs(to_np64(o[i : i + 1]) - O_ref) - 0.5 * bf16_ulp(O_ref)) <= O_TOL
+        assert np.max(np.abs(lse[:, i : i + 1].double().numpy() - L_ref)) <= LSE_TOL
