@@ -465,7 +465,7 @@ k_bwd_dq_ds(const __grid_constant__ CUtensorMap tmDS, const __grid_constant__ CU
         // ------------------------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t u = 0;
-            for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+            for (int rnd = 0, item = blockIdx.x; item < n_items; item = alt_item(++rnd, blockIdx.x, gridDim.x)) {
                 const DqItem w = dq_decode(meta, hd, item, hq, hkv);
                 const int n = qtile_nkv(w.t);
                 const int qt = (w.t.row0 - w.t.gstart) / BWD_BM;       // query tile within the group
@@ -493,7 +493,7 @@ k_bwd_dq_ds(const __grid_constant__ CUtensorMap tmDS, const __grid_constant__ CU
             const uint64_t a_desc = smem_desc(smem_u32(sm.ds[0]), DqsSmem::CHUNK, 1024);
             const uint64_t b_desc = smem_desc(smem_u32(sm.k[0]), DqsSmem::CHUNK, 1024);
             uint32_t u = 0, it_n = 0;
-            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+            for (int rnd = 0, item = blockIdx.x; item < n_items; item = alt_item(++rnd, blockIdx.x, gridDim.x), ++it_n) {
                 const int n = qtile_nkv(meta_ptr<QTile>(meta, hd.off_qts)[item / hq]);
                 const uint32_t b = it_n & 1;
                 if (!bwait(&sm.acc_empty[b], ((it_n >> 1) & 1) ^ 1, abort_flag)) goto done;
@@ -518,7 +518,7 @@ k_bwd_dq_ds(const __grid_constant__ CUtensorMap tmDS, const __grid_constant__ CU
         const int rt = warp * 32 + lane;
         const bool dq_v8 = aligned32(dQ);                                // rows are 256 bytes: the base decides
         uint32_t it_n = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it_n) {
+        for (int rnd = 0, item = blockIdx.x; item < n_items; item = alt_item(++rnd, blockIdx.x, gridDim.x), ++it_n) {
             const DqItem w = dq_decode(meta, hd, item, hq, hkv);
             const uint32_t b = it_n & 1;
             const int row = w.t.row0 + rt;

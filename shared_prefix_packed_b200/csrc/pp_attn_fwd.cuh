@@ -168,11 +168,12 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (hd.dev_err == 0 && warp == 8 && lane == 0) {
         // ------------------------------------------------------------------ TMA producer
         uint32_t kv_it = 0, n_it = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        for (int rnd = 0, item = blockIdx.x; item < n_items; item = alt_item(++rnd, blockIdx.x, gridDim.x)) {
             const FwdItem w = fwd_decode(meta, hd, item, hq, hkv);
             const int n = qtile_nkv(w.t);
-            if (item + int(gridDim.x) < n_items) {                     // the next item's Q into L2 (read once, so
-                const FwdItem wn = fwd_decode(meta, hd, item + gridDim.x, hq, hkv);   // a miss otherwise)
+            const int nxt = alt_item(rnd + 1, blockIdx.x, gridDim.x);
+            if (nxt < n_items) {                                       // the next item's Q into L2 (read once, so
+                const FwdItem wn = fwd_decode(meta, hd, nxt, hq, hkv);  // a miss otherwise)
                 for (int hs = 0; hs < wn.nh; ++hs)
                     for (int c = 0; c < D / 64; ++c) tma_prefetch_3d(&tmQ, c * 64, wn.h0 + hs, wn.t.row0);
             }
@@ -230,7 +231,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             for (int kk = 0; kk < FWD_BN / 16; ++kk)
                 umma_ts(d, a + kk * 8, desc_adv(b, kk * 2048), IDESC_O, (acc | kk) ? 1u : 0u);
         };
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        for (int rnd = 0, item = blockIdx.x; item < n_items; item = alt_item(++rnd, blockIdx.x, gridDim.x)) {
             const FwdItem w = fwd_decode(meta, hd, item, hq, hkv);
             const int n = qtile_nkv(w.t);
             if (!bwait(&sm.q_full, n_it & 1, abort_flag)) goto done;
@@ -277,7 +278,7 @@ k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const uint32_t t_o = tmem + (uint32_t(lane_base) << 16) + 256 + wg * 128;
         const bool o_v8 = aligned32(O);                                  // rows are d * 2 bytes: the base decides
         uint32_t s_cnt = 0, pv_cnt = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        for (int rnd = 0, item = blockIdx.x; item < n_items; item = alt_item(++rnd, blockIdx.x, gridDim.x)) {
             const FwdItem w = fwd_decode(meta, hd, item, hq, hkv);
             if (wg >= w.nh) continue;
             const int h = w.h0 + wg;

@@ -158,4 +158,9 @@ __host__ __device__ inline int qtile_nkv(const QTile &t) {
 // i-th key tile (in-group tile index) a forward query tile visits: run A, then run B.
 __host__ __device__ inline int qtile_kv(const QTile &t, int i) { return i < t.nA ? i : t.bB + (i - t.nA); }
 
+// Item that CTA b of a persistent grid of g CTAs takes in its round k, for items in decreasing cost order: each
+// round deals the next g items, in alternating directions, so that the CTAs that took the costlier items of one
+// round take the cheaper ones of the next (plain round-robin gives CTA 0 the costliest item of every round).
+__host__ __device__ inline int alt_item(int k, int b, int g) { return k * g + ((k & 1) ? g - 1 - b : b); }
+
 }  // namespace pp
