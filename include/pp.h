@@ -173,7 +173,8 @@ PP_API pp_status pp_attn_fwd(const void *q, const void *k, const void *v, const 
  *   one CTA (no reduction). If ws_bytes also covers pp_bwd_ds_bytes(...) for the batch, the dK/dV kernel keeps
  *   every step's dS tile after the base workspace and dq is formed from them (the fast path); otherwise the dq
  *   kernel recomputes the tile's scores and dP. The choice is made on the device from the batch's step count, so
- *   either size is valid. The result is deterministic except for the order of the dK/dV adds.
+ *   either size is valid. A batch of T tokens that could exceed 2^31 - 1 steps per kv head (about 4.2 M tokens at
+ *   hq/hkv = 4) always takes the recompute path. The result is deterministic except for the order of the dK/dV adds.
  */
 PP_API pp_status pp_attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
                       const void *dout, const void *meta_d, int64_t T, int32_t hq, int32_t hkv, int32_t d,

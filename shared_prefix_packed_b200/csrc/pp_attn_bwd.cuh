@@ -731,6 +731,9 @@ inline pp_status launch_bwd(const void *q, const void *k, const void *v, const v
     const int64_t ds_off = (L.total + BWD_DS_ALIGN - 1) / BWD_DS_ALIGN * BWD_DS_ALIGN;
     int64_t ds_cap = ws_bytes > ds_off ? (ws_bytes - ds_off) / BWD_DS_TILE_BYTES : 0;
     if (ds_cap > (int64_t(1) << 24)) ds_cap = int64_t(1) << 24;       // TMA row coordinate stays below 2^31
+    // the schedule builder counts steps and slot offsets in int32: keep no dS tiles where a batch of T tokens could
+    // have more (T above about 4.2 M tokens at r = 4)
+    if (bwd_steps_bound(T, hq / hkv) > int64_t(0x7fffffff)) ds_cap = 0;
     __nv_bfloat16 *ds_buf = ds_cap > 0 ? reinterpret_cast<__nv_bfloat16 *>(ws + ds_off) : nullptr;
     if (ds_buf && (st = make_map_box(&mds, ds_buf, ds_cap * BWD_BN, 1, BWD_BM, 1, BWD_BN)) != PP_OK) return st;
     cudaError_t e;

@@ -158,6 +158,15 @@ __host__ __device__ inline int qtile_nkv(const QTile &t) {
 // i-th key tile (in-group tile index) a forward query tile visits: run A, then run B.
 __host__ __device__ inline int qtile_kv(const QTile &t, int i) { return i < t.nA ? i : t.bB + (i - t.nA); }
 
+// Upper bound, from T alone, on the backward steps of one kv head (sum over key tiles of the query tiles that attend
+// them, times r). A group of n key tiles has at most n (n + 1) / 2 (key tile, query tile) pairs; joining two groups
+// of two or more tiles each never lowers the count, and groups of one tile add at most one pair per token, so
+// T + N (N + 1) / 2 pairs with N = ceil(T / BWD_BN) bound any batch of T tokens.
+__host__ __device__ inline int64_t bwd_steps_bound(int64_t T, int r) {
+    const int64_t n = (T + BWD_BN - 1) / BWD_BN;
+    return int64_t(r) * (T + n * (n + 1) / 2);
+}
+
 // Item that CTA b of a persistent grid of g CTAs takes in its round k, for items in decreasing cost order: each
 // round deals the next g items, in alternating directions, so that the CTAs that took the costlier items of one
 // round take the cheaper ones of the next (plain round-robin gives CTA 0 the costliest item of every round).
